@@ -1,0 +1,449 @@
+"""Benchmark: Flux single-stream block forward at S=4608, dim 3072, 24 x 128,
+MLP 12288, bf16, on B200 through the C ABI (libdit.so).
+
+One step = one block forward (adaLN modulation, LayerNorm+modulate, fused
+QKV|MLP-in GEMM with GELU, QK RMSNorm+RoPE, flash attention, output GEMM
+with the gated residual) over one synthetic batch-1 input already resident in
+HBM.  The weights of one block (282 MB) and its activations exceed the 126 MB
+L2, so every step streams them from HBM.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 runs under torch.distributed.run, one independent replica per GPU (the
+block is data-parallel over samples; there is no exchange step), and reports
+the whole-job throughput (weak scaling).  --impl reference times the fp64 CPU
+oracle on the host cores instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "Flux single-stream block ms & TFLOP/s at S=4608 bf16; % of tensor/HBM roofline"
+UNIT = "TFLOP/s"
+WORKLOAD = "flux_single_block_S4608_D3072_H24_M12288_bf16"
+S_TXT, GRID, D, H, M = 512, 64, 3072, 24, 12288
+S = S_TXT + GRID * GRID
+KERNELS = ["adaln_modulation", "modulate_norm", "gemm_qkv_mlp_gelu", "qk_norm_rope", "attention",
+           "gemm_out_gated_residual"]
+
+
+def block_flops(S_=S):
+    gemm1 = 2.0 * S_ * D * (3 * D + M)
+    attn = 4.0 * S_ * S_ * H * 128
+    gemm2 = 2.0 * S_ * (D + M) * D
+    mod = 2.0 * D * 3 * D
+    return {"adaln_modulation": mod, "modulate_norm": 0.0, "gemm_qkv_mlp_gelu": gemm1, "qk_norm_rope": 0.0,
+            "attention": attn, "gemm_out_gated_residual": gemm2}
+
+
+def block_bytes(S_=S):
+    """Algorithmic HBM bytes per launch (read once + write once)."""
+    return {
+        "adaln_modulation": 3 * D * D * 2 + D * 2 + 3 * D * 4,
+        "modulate_norm": 2 * S_ * D * 2,
+        "gemm_qkv_mlp_gelu": S_ * D * 2 + (3 * D + M) * D * 2 + S_ * (3 * D + M) * 2,
+        "qk_norm_rope": 4 * S_ * D * 2 + S_ * 64 * 8,
+        "attention": 4 * S_ * D * 2,
+        "gemm_out_gated_residual": S_ * (D + M) * 2 + D * (D + M) * 2 + 2 * S_ * D * 2,
+    }
+
+
+KERNEL_BOUND = {"adaln_modulation": "hbm", "modulate_norm": "hbm", "gemm_qkv_mlp_gelu": "tensor",
+                "qk_norm_rope": "hbm", "attention": "tensor", "gemm_out_gated_residual": "tensor"}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return {"hbm_gbs": float(j["hbm_gbs"]), "bf16_tflops": float(j["bf16_tflops"]),
+                "bf16_tflops_sustained": float(j.get("bf16_tflops_sustained", j["bf16_tflops"])),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ----------------------------------------------------------------------------
+# Clock sampling during the timed region
+# ----------------------------------------------------------------------------
+
+REASON_COLS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+
+
+class ClockSampler:
+    def __init__(self, index: int):
+        self.index = index
+        self.samples = []
+        self.proc = None
+        self.t = None
+
+    def start(self):
+        q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+             "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+             "clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.t = threading.Thread(target=self._read, daemon=True)
+        self.t.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 7:
+                self.samples.append((time.time(), parts))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self, t0, t1):
+        rows = [p for (t, p) in self.samples if t0 - 0.05 <= t <= t1 + 0.05] or [p for (_, p) in self.samples]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[0]) for r in rows if num(r[0]) is not None]
+        busy = [v for v in sm if v > 500] or sm
+        reasons = sorted({REASON_COLS[i] for r in rows for i in range(4) if r[3 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(busy) if busy else None,
+                "sm_max_mhz": num(rows[0][1]), "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------
+# Our arm
+# ----------------------------------------------------------------------------
+
+
+def make_block(torch, dev, seed):
+    """Random-init weights of the block (N(0, 0.02) linears, zero biases, unit
+    norm scales) and N(0, 1) inputs, drawn on the device from a seeded
+    generator."""
+    g = torch.Generator(device=dev)
+    g.manual_seed(seed)
+
+    def nrm(*shape, std=1.0):
+        return (torch.randn(*shape, generator=g, device=dev, dtype=torch.float32) * std).to(torch.bfloat16)
+
+    w = {"W_mod": nrm(3 * D, D, std=0.02), "b_mod": torch.zeros(3 * D, device=dev, dtype=torch.bfloat16),
+         "W1": nrm(3 * D + M, D, std=0.02), "b1": torch.zeros(3 * D + M, device=dev, dtype=torch.bfloat16),
+         "q_scale": torch.ones(128, device=dev, dtype=torch.bfloat16),
+         "k_scale": torch.ones(128, device=dev, dtype=torch.bfloat16),
+         "W2": nrm(D, D + M, std=0.02), "b2": torch.zeros(D, device=dev, dtype=torch.bfloat16)}
+    x = nrm(S, D)
+    vec = nrm(1, D)
+    return w, x, vec
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import diffusion_transformer_block_flux_b200 as dit
+    from diffusion_transformer_block_flux_b200 import synth
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    dit.lib()  # raises if the CUDA library is missing
+    w, x, vec = make_block(torch, dev, seed=1234 + rank)
+    ids = torch.from_numpy(synth.flux_ids(S_TXT, GRID, GRID)).to(dev)
+    rope = torch.empty((S, 64, 2), dtype=torch.float32, device=dev)
+    dit.dit_rope_table(ids, (8, 28, 28), 10000.0, rope)
+    cfg = dit.block_cfg(1, S, D, H, M)
+    ws = torch.empty(dit.dit_single_block_workspace(cfg), dtype=torch.uint8, device=dev)
+    out = torch.empty_like(x)
+    cw = dit.single_weights(w)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(evs=None):
+        dit.dit_single_block_fwd(cfg, cw, x, vec, rope, out, ws, events=evs)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st, code = dit.dit_get_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error word {code:#x} after warm-up")
+
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(K)]
+    for row in evs:  # torch creates the CUDA event on first record
+        for e in row:
+            e.record(stream)
+    torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    time.sleep(0.3)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    wall0 = time.time()
+    t_start.record(stream)
+    for i in range(K):
+        step(evs[i])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    wall1 = time.time()
+    if world > 1:
+        torch.distributed.barrier()
+    time.sleep(0.2)
+    sampler.stop()
+    clocks = sampler.summary(wall0, wall1)
+    elapsed_ms = t_start.elapsed_time(t_end)
+    per_kernel = {k: statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(K))
+                  for j, k in enumerate(KERNELS)}
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    st, code = dit.dit_get_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error word {code:#x} in the timed region")
+
+    # ---- end to end through the C ABI with host buffers ----
+    x_h = torch.empty((S, D), dtype=torch.bfloat16).pin_memory()
+    x_h.copy_(x.cpu())
+    vec_h = vec.cpu().pin_memory()
+    out_h = torch.empty_like(x_h).pin_memory()
+    x_d = torch.empty_like(x)
+    vec_d = torch.empty_like(vec)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    Ke = max(1, min(K, 200))
+
+    def e2e_step():
+        x_d.copy_(x_h, non_blocking=True)
+        vec_d.copy_(vec_h, non_blocking=True)
+        dit.dit_single_block_fwd(cfg, cw, x_d, vec_d, rope, out, ws)
+        out_h.copy_(out, non_blocking=True)
+
+    for _ in range(max(3, min(args.warmup, 10))):
+        e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    e0.record(stream)
+    for _ in range(Ke):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    flops = block_flops()
+    total_flops = sum(flops.values())
+    ms_per_step = elapsed_ms / K
+    value = world * total_flops * K / (elapsed_ms * 1e-3) / 1e12
+    e2e_value = world * total_flops * Ke / (e2e_ms * 1e-3) / 1e12
+
+    pk = peaks()
+    dom = max(per_kernel, key=per_kernel.get)
+    nbytes = block_bytes()
+    if KERNEL_BOUND[dom] == "tensor":
+        achieved = flops[dom] / (per_kernel[dom] * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": round(achieved / pk["bf16_tflops"], 4)}
+    else:
+        achieved = nbytes[dom] / (per_kernel[dom] * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": round(achieved / pk["hbm_gbs"], 4)}
+    roof["kernel"] = dom
+    roof["traffic"] = TRAFFIC.get(dom)
+    roof["peak_source"] = pk["source"] + " burst (MEASURED_PEAKS.json)" if pk["source"] == "measured" else "fallback"
+    kernels = {}
+    for k in KERNELS:
+        ent = {"ms": round(per_kernel[k], 4), "share": round(per_kernel[k] / sum(per_kernel.values()), 4)}
+        if KERNEL_BOUND[k] == "tensor":
+            a = flops[k] / (per_kernel[k] * 1e-3) / 1e12
+            ent.update({"tflops": round(a, 1), "frac_of_bf16_peak": round(a / pk["bf16_tflops"], 4)})
+        else:
+            a = nbytes[k] / (per_kernel[k] * 1e-3) / 1e9
+            ent.update({"gbs": round(a, 1), "frac_of_hbm_peak": round(a / pk["hbm_gbs"], 4)})
+        kernels[k] = ent
+    block_frac = (total_flops / (ms_per_step * 1e-3) / 1e12) / pk["bf16_tflops"]
+    res = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "global_batch": world, "seq_len": S, "parallelism": f"replicas{world}",
+                   "l2": "inputs larger than L2 (282 MB of block weights + 0.25 GB activations per step)"},
+        "ms_per_block": round(ms_per_step, 4), "blocks_per_s": round(world * 1e3 / ms_per_step, 1),
+        "block_frac_of_bf16_peak": round(block_frac, 4),
+        "gpu_launches": 6 * K,
+        "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": S * D * 2 + D * 2,
+                "d2h_bytes_per_step": S * D * 2, "steps": Ke},
+        "roofline": roof, "kernels": kernels, "clocks": clocks,
+    }
+    return res
+
+
+TRAFFIC: dict = {}
+
+
+# ----------------------------------------------------------------------------
+# CPU oracle (reference arm and cpu_baseline leg)
+# ----------------------------------------------------------------------------
+
+
+def oracle_inputs(n_tokens):
+    """Seeded cfg-2 weights and the first n_tokens tokens (text first, then
+    image rows) of the cfg-2 input, widened to fp64."""
+    from diffusion_transformer_block_flux_b200 import synth
+    shape = synth.FLUX
+    w = synth.to_f64(synth.single_block_weights(shape))
+    a = synth.block_activations(shape)
+    x = synth.bf16_bits_to_f64(a["x"][:n_tokens])
+    vec = synth.bf16_bits_to_f64(a["vec"])
+    return w, x, vec, a["ids"][:n_tokens]
+
+
+def oracle_block_time(n_tokens, reps, w=None):
+    from oracle import dit_oracle as O
+    if w is None:
+        w, x, vec, ids = oracle_inputs(n_tokens)
+    else:
+        w, x, vec, ids = w
+    times = []
+    for _ in range(reps):
+        t0 = time.perf_counter()
+        O.single_block(x, vec, ids, w, H)
+        times.append(time.perf_counter() - t0)
+    return times
+
+
+def cores_used():
+    for var in ("OPENBLAS_NUM_THREADS", "OMP_NUM_THREADS", "MKL_NUM_THREADS"):
+        if os.environ.get(var):
+            return int(os.environ[var])
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n and n[0]:
+            return int(n[0])
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+def sub_flops(n):
+    return sum(block_flops(n).values())
+
+
+def cpu_baseline(n_tokens=1024, reps=2):
+    inp = oracle_inputs(n_tokens)
+    oracle_block_time(64, 1, (inp[0], inp[1][:64], inp[2], inp[3][:64]))  # warm BLAS threads
+    times = oracle_block_time(n_tokens, reps, inp)
+    t = statistics.mean(times)
+    return {"value": round(sub_flops(n_tokens) / t / 1e12, 5), "unit": UNIT, "cores": cores_used(),
+            "kind": "oracle",
+            "sample": f"fp64 numpy oracle single-stream block on the first {n_tokens} of the 4608 tokens "
+                      f"(full dim 3072, 24 heads, MLP 12288, same weights), mean of {reps} runs "
+                      f"of {t:.2f} s; TFLOP/s = algorithmic FLOPs of that sub-block / time"}
+
+
+def run_reference(args):
+    """Reference arm: the fp64 oracle as it stands, on the host cores.  Each
+    step runs the block on a leading token window sized so the whole
+    --steps/--warmup run stays within about two minutes."""
+    budget_s = 120.0
+    calib_n = 128
+    inp = oracle_inputs(S)
+    full_w = inp[0]
+    t_cal = min(oracle_block_time(calib_n, 2, (full_w, inp[1][:calib_n], inp[2], inp[3][:calib_n])))
+    per_token = t_cal / calib_n
+    per_step = budget_s / max(1, args.steps + args.warmup)
+    n = int(max(64, min(S, (per_step / per_token) // 64 * 64)))
+    sub = (full_w, inp[1][:n], inp[2], inp[3][:n])
+    oracle_block_time(n, args.warmup, sub)
+    times = oracle_block_time(n, args.steps, sub)
+    total = sum(times)
+    value = sub_flops(n) * args.steps / total / 1e12
+    sample = (f"fp64 numpy oracle single-stream block on the first {n} of the 4608 tokens per step "
+              f"(full dim 3072, 24 heads, MLP 12288); TFLOP/s = algorithmic FLOPs of that sub-block / time")
+    return {
+        "metric": METRIC, "value": round(value, 5), "unit": UNIT, "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(total / args.steps * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "global_batch": 1, "seq_len": S, "parallelism": "none",
+                   "tokens_per_step": n},
+        "impl": "reference",
+        "cpu_baseline": {"value": round(value, 5), "unit": UNIT, "cores": cores_used(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 5), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        print(json.dumps(run_reference(args)), flush=True)
+        return 0
+
+    if world != args.gpus:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}; using WORLD_SIZE", file=sys.stderr)
+    if world > 1:
+        import datetime
+        import torch
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        traffic_file = os.path.join(ROOT, "profiles", "traffic.json")
+        if os.path.exists(traffic_file):
+            with open(traffic_file) as f:
+                TRAFFIC.update(json.load(f).get("per_launch_bytes", {}))
+        res = run_ours(args, rank, world, local_rank)
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            res["cpu_baseline"] = cpu_baseline()
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            import torch
+            torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

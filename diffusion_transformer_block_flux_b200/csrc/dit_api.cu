@@ -1,0 +1,396 @@
+// C ABI of libdit: argument checks, TMA descriptor encoding and kernel
+// launches for every entry point declared in include/dit.h.
+//
+// Every entry point validates its arguments before enqueuing anything, never
+// allocates device memory, never synchronises (except dit_get_device_error)
+// and reports CUDA failures as DIT_ERR_CUDA.
+#include <math.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "attention.cuh"
+#include "common.cuh"
+#include "elementwise.cuh"
+#include "gemm.cuh"
+
+using dit::bf16;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int kVecSmemMax = 200 * 1024;  // staged input vectors of dit_vec_linear (B * K fp32)
+uint64_t g_wait_limit_ns = 2000000000ull;
+
+struct DeviceInfo {
+  bool init = false;
+  bool supported = false;
+  int num_sms = 0;
+  bool attrs_set = false;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_mu;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+#define DIT_CUDA_CHECK(expr)                 \
+  do {                                       \
+    cudaError_t e_ = (expr);                 \
+    if (e_ != cudaSuccess) return DIT_ERR_CUDA; \
+  } while (0)
+
+dit_status launch_status() {
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? DIT_OK : DIT_ERR_CUDA;
+}
+
+// Per-device setup: SM count, capability check, kernel attributes, driver
+// entry point for tensor-map encoding.
+dit_status device_setup(int* num_sms) {
+  int dev = 0;
+  DIT_CUDA_CHECK(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDevices) return DIT_ERR_UNSUPPORTED;
+  DeviceInfo& d = g_dev[dev];
+  if (!d.init) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!d.init) {
+      int major = 0, sms = 0;
+      DIT_CUDA_CHECK(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev));
+      DIT_CUDA_CHECK(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+      d.supported = (major == 10);
+      d.num_sms = sms;
+      if (d.supported) {
+        DIT_CUDA_CHECK(cudaFuncSetAttribute(dit::gemm::gemm_kernel<DIT_EPI_NONE>,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize, dit::gemm::SMEM_BYTES));
+        DIT_CUDA_CHECK(cudaFuncSetAttribute(dit::gemm::gemm_kernel<DIT_EPI_BIAS>,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize, dit::gemm::SMEM_BYTES));
+        DIT_CUDA_CHECK(cudaFuncSetAttribute(dit::gemm::gemm_kernel<DIT_EPI_BIAS_GELU_COLS>,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize, dit::gemm::SMEM_BYTES));
+        DIT_CUDA_CHECK(cudaFuncSetAttribute(dit::gemm::gemm_kernel<DIT_EPI_BIAS_GATED_RESIDUAL>,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize, dit::gemm::SMEM_BYTES));
+        DIT_CUDA_CHECK(cudaFuncSetAttribute(dit::attn::attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            dit::attn::SMEM_BYTES));
+        for (int nb = 1; nb <= 8; nb *= 2) {
+          void* f = nb == 1   ? (void*)dit::vec_linear_kernel<1>
+                    : nb == 2 ? (void*)dit::vec_linear_kernel<2>
+                    : nb == 4 ? (void*)dit::vec_linear_kernel<4>
+                              : (void*)dit::vec_linear_kernel<8>;
+          DIT_CUDA_CHECK(cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, kVecSmemMax));
+        }
+        if (g_encode == nullptr) {
+          void* fn = nullptr;
+          cudaDriverEntryPointQueryResult q;
+          DIT_CUDA_CHECK(cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q));
+          if (q != cudaDriverEntryPointSuccess || fn == nullptr) return DIT_ERR_CUDA;
+          g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+        }
+      }
+      d.init = true;
+    }
+  }
+  if (!d.supported) return DIT_ERR_UNSUPPORTED;
+  if (num_sms) *num_sms = d.num_sms;
+  return DIT_OK;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// 2-D bf16 tensor map: rows x cols (cols contiguous, row stride ld elements),
+// box = box_rows x 64 columns, 128-byte swizzle, zero fill out of bounds.
+dit_status make_map_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, int64_t ld, uint32_t box_rows) {
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? DIT_OK : DIT_ERR_CUDA;
+}
+
+// 3-D bf16 tensor map over [batch][rows][cols] with row stride ld elements and
+// batch stride rows*ld; box = 128 rows x 64 columns x 1.
+dit_status make_map_3d(CUtensorMap* m, const void* base, uint64_t batch, uint64_t rows, uint64_t cols, int64_t ld) {
+  cuuint64_t dims[3] = {cols, rows, batch};
+  cuuint64_t strides[2] = {(cuuint64_t)ld * 2, (cuuint64_t)ld * 2 * rows};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? DIT_OK : DIT_ERR_CUDA;
+}
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Internal RoPE-only / norm+RoPE launch shared by the public call and blocks.
+dit_status launch_qk(const bf16* q, const bf16* k, int64_t ld_in, const bf16* qs, const bf16* ks, const float* rope,
+                     bf16* qo, bf16* ko, int64_t ld_out, int B, int S, int H, float eps, int do_norm,
+                     cudaStream_t st) {
+  const int64_t n_vecs = (int64_t)B * S * H * 2;
+  const int threads = 256;
+  const int64_t blocks = (n_vecs * 16 + threads - 1) / threads;
+  dit::qk_norm_rope_kernel<<<(unsigned)blocks, threads, 0, st>>>(q, k, ld_in, qs, ks,
+                                                                  reinterpret_cast<const float2*>(rope), qo, ko,
+                                                                  ld_out, S, H, n_vecs, eps, do_norm);
+  return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* dit_status_string(dit_status s) {
+  switch (s) {
+    case DIT_OK: return "ok";
+    case DIT_ERR_INVALID_ARG: return "invalid argument";
+    case DIT_ERR_SHAPE: return "unsupported shape";
+    case DIT_ERR_ALIGNMENT: return "pointer or stride not 16-byte aligned";
+    case DIT_ERR_UNSUPPORTED: return "unsupported configuration or device";
+    case DIT_ERR_CUDA: return "CUDA runtime error";
+    case DIT_ERR_NOT_CAPTURABLE: return "not allowed while the stream is capturing";
+    case DIT_ERR_TIMEOUT: return "device-side wait timed out";
+    case DIT_ERR_WORKSPACE: return "workspace missing or too small";
+  }
+  return "unknown status";
+}
+
+int dit_version(void) { return 100; }
+
+dit_status dit_get_device_error(void* stream, uint32_t* code) {
+  if (code == nullptr) return DIT_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  DIT_CUDA_CHECK(cudaStreamIsCapturing(st, &cs));
+  if (cs != cudaStreamCaptureStatusNone) return DIT_ERR_NOT_CAPTURABLE;
+  unsigned int v = 0;
+  DIT_CUDA_CHECK(cudaMemcpyFromSymbolAsync(&v, dit::g_dit_error, sizeof(v), 0, cudaMemcpyDeviceToHost, st));
+  DIT_CUDA_CHECK(cudaStreamSynchronize(st));
+  *code = v;
+  return v == 0 ? DIT_OK : DIT_ERR_TIMEOUT;
+}
+
+dit_status dit_clear_device_error(void* stream) {
+  static const unsigned int zero = 0;
+  DIT_CUDA_CHECK(cudaMemcpyToSymbolAsync(dit::g_dit_error, &zero, sizeof(zero), 0, cudaMemcpyHostToDevice,
+                                         (cudaStream_t)stream));
+  DIT_CUDA_CHECK(cudaStreamSynchronize((cudaStream_t)stream));
+  return DIT_OK;
+}
+
+dit_status dit_set_wait_limit_ns(uint64_t limit_ns) {
+  if (limit_ns == 0) return DIT_ERR_INVALID_ARG;
+  g_wait_limit_ns = limit_ns;
+  return DIT_OK;
+}
+
+dit_status dit_selftest_wait_timeout(uint64_t limit_ns, void* stream) {
+  if (limit_ns == 0 || limit_ns > 10000000000ull) return DIT_ERR_INVALID_ARG;
+  dit_status s = device_setup(nullptr);
+  if (s != DIT_OK) return s;
+  dit::selftest_wait_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(limit_ns);
+  return launch_status();
+}
+
+dit_status dit_rope_table(const int32_t* ids, int S, int n_axes, const int* axes_pairs, double theta, float* rope,
+                          void* stream) {
+  if (ids == nullptr || rope == nullptr || axes_pairs == nullptr) return DIT_ERR_INVALID_ARG;
+  if (S <= 0 || n_axes < 1 || n_axes > 3 || !(theta > 0)) return DIT_ERR_INVALID_ARG;
+  int p[3] = {0, 0, 0};
+  for (int a = 0; a < n_axes; ++a) {
+    if (axes_pairs[a] < 0) return DIT_ERR_INVALID_ARG;
+    p[a] = axes_pairs[a];
+  }
+  if (p[0] + p[1] + p[2] <= 0) return DIT_ERR_INVALID_ARG;
+  dit_status s = device_setup(nullptr);
+  if (s != DIT_OK) return s;
+  const int64_t n = (int64_t)S * (p[0] + p[1] + p[2]);
+  dit::rope_table_kernel<<<(unsigned)((n + 255) / 256), 256, 0, (cudaStream_t)stream>>>(
+      ids, S, n_axes, p[0], p[1], p[2], theta, reinterpret_cast<float2*>(rope));
+  return launch_status();
+}
+
+dit_status dit_vec_linear(const dit_bf16* x, int64_t ldx, const dit_bf16* W, int64_t ldw, const dit_bf16* bias,
+                          void* out, int64_t ldo, int B, int N, int K, int flags, void* stream) {
+  if (x == nullptr || W == nullptr || out == nullptr) return DIT_ERR_INVALID_ARG;
+  if (B < 1 || B > 8 || N < 1 || K < 8 || K > 8192 || (K % 8) != 0) return DIT_ERR_SHAPE;
+  if ((size_t)B * K * sizeof(float) > (size_t)kVecSmemMax) return DIT_ERR_SHAPE;
+  if (ldx < K || ldw < K || ldo < N || (ldw % 8) != 0) return DIT_ERR_SHAPE;
+  if (!aligned16(W)) return DIT_ERR_ALIGNMENT;
+  if (flags & ~(DIT_VEC_SILU_IN | DIT_VEC_OUT_BF16)) return DIT_ERR_INVALID_ARG;
+  int sms = 0;
+  dit_status s = device_setup(&sms);
+  if (s != DIT_OK) return s;
+  const int threads = 256, wpb = threads / 32;
+  int blocks = (N + wpb - 1) / wpb;
+  if (blocks > sms * 8) blocks = sms * 8;
+  const size_t smem = (size_t)B * K * sizeof(float);
+  cudaStream_t st = (cudaStream_t)stream;
+  const bf16* xb = reinterpret_cast<const bf16*>(x);
+  const bf16* Wb = reinterpret_cast<const bf16*>(W);
+  const bf16* bb = reinterpret_cast<const bf16*>(bias);
+  if (B == 1)
+    dit::vec_linear_kernel<1><<<blocks, threads, smem, st>>>(xb, ldx, Wb, ldw, bb, out, ldo, B, N, K, flags);
+  else if (B <= 2)
+    dit::vec_linear_kernel<2><<<blocks, threads, smem, st>>>(xb, ldx, Wb, ldw, bb, out, ldo, B, N, K, flags);
+  else if (B <= 4)
+    dit::vec_linear_kernel<4><<<blocks, threads, smem, st>>>(xb, ldx, Wb, ldw, bb, out, ldo, B, N, K, flags);
+  else
+    dit::vec_linear_kernel<8><<<blocks, threads, smem, st>>>(xb, ldx, Wb, ldw, bb, out, ldo, B, N, K, flags);
+  return launch_status();
+}
+
+dit_status dit_adaln_modulation(const dit_bf16* vec, int64_t ldv, const dit_bf16* W, int64_t ldw,
+                                const dit_bf16* bias, float* out, int64_t ldo, int B, int N, int K, void* stream) {
+  return dit_vec_linear(vec, ldv, W, ldw, bias, out, ldo, B, N, K, DIT_VEC_SILU_IN, stream);
+}
+
+dit_status dit_modulate_norm(const dit_bf16* x, int64_t ldx, const float* shift, const float* scale,
+                             int64_t mod_stride, dit_bf16* y, int64_t ldy, int B, int S, int D, float eps,
+                             void* stream) {
+  if (x == nullptr || y == nullptr) return DIT_ERR_INVALID_ARG;
+  if ((shift == nullptr) != (scale == nullptr)) return DIT_ERR_INVALID_ARG;
+  if (B < 1 || S < 1 || D < 8 || D > 8192 || (D % 8) != 0) return DIT_ERR_SHAPE;
+  if (ldx < D || ldy < D || (ldx % 8) != 0 || (ldy % 8) != 0) return DIT_ERR_SHAPE;
+  if (!aligned16(x) || !aligned16(y)) return DIT_ERR_ALIGNMENT;
+  if (shift != nullptr && (!aligned16(shift) || !aligned16(scale) || (mod_stride % 4) != 0))
+    return DIT_ERR_ALIGNMENT;
+  if (!(eps >= 0)) return DIT_ERR_INVALID_ARG;
+  if ((const void*)x == (const void*)y) return DIT_ERR_INVALID_ARG;
+  dit_status s = device_setup(nullptr);
+  if (s != DIT_OK) return s;
+  const int threads = ((D / 8 + 31) / 32) * 32;
+  dit::modulate_norm_kernel<<<(unsigned)((int64_t)B * S), threads, 0, (cudaStream_t)stream>>>(
+      reinterpret_cast<const bf16*>(x), ldx, shift, scale, mod_stride, reinterpret_cast<bf16*>(y), ldy, S, D, eps);
+  return launch_status();
+}
+
+dit_status dit_qk_norm_rope(const dit_bf16* q, const dit_bf16* k, int64_t ld_in, const dit_bf16* q_scale,
+                            const dit_bf16* k_scale, const float* rope, dit_bf16* q_out, dit_bf16* k_out,
+                            int64_t ld_out, int B, int S, int H, int head_dim, float eps, void* stream) {
+  if (q == nullptr || k == nullptr || q_out == nullptr || k_out == nullptr) return DIT_ERR_INVALID_ARG;
+  if (head_dim != 128) return DIT_ERR_UNSUPPORTED;
+  if (B < 1 || S < 1 || H < 1) return DIT_ERR_SHAPE;
+  if (ld_in < (int64_t)H * 128 || ld_out < (int64_t)H * 128 || (ld_in % 8) != 0 || (ld_out % 8) != 0)
+    return DIT_ERR_SHAPE;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(q_out) || !aligned16(k_out)) return DIT_ERR_ALIGNMENT;
+  if ((q_scale && !aligned16(q_scale)) || (k_scale && !aligned16(k_scale)) || (rope && !aligned16(rope)))
+    return DIT_ERR_ALIGNMENT;
+  if (!(eps >= 0)) return DIT_ERR_INVALID_ARG;
+  dit_status s = device_setup(nullptr);
+  if (s != DIT_OK) return s;
+  return launch_qk(reinterpret_cast<const bf16*>(q), reinterpret_cast<const bf16*>(k), ld_in,
+                   reinterpret_cast<const bf16*>(q_scale), reinterpret_cast<const bf16*>(k_scale), rope,
+                   reinterpret_cast<bf16*>(q_out), reinterpret_cast<bf16*>(k_out), ld_out, B, S, H, eps, 1,
+                   (cudaStream_t)stream);
+}
+
+dit_status dit_attention(const dit_bf16* q, const dit_bf16* k, const dit_bf16* v, int64_t ldq, int64_t ldk,
+                         int64_t ldv, dit_bf16* o, int64_t ldo, float* lse, int B, int Sq, int Skv, int H,
+                         int head_dim, float softmax_scale, void* stream) {
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr) return DIT_ERR_INVALID_ARG;
+  if (head_dim != 128) return DIT_ERR_UNSUPPORTED;
+  if (B < 1 || Sq < 1 || Skv < 1 || H < 1 || B > 65535 || H > 65535) return DIT_ERR_SHAPE;
+  const int64_t D = (int64_t)H * 128;
+  if (ldq < D || ldk < D || ldv < D || ldo < D) return DIT_ERR_SHAPE;
+  if ((ldq % 8) || (ldk % 8) || (ldv % 8) || (ldo % 8)) return DIT_ERR_ALIGNMENT;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return DIT_ERR_ALIGNMENT;
+  if (!(softmax_scale > 0)) return DIT_ERR_INVALID_ARG;
+  dit_status s = device_setup(nullptr);
+  if (s != DIT_OK) return s;
+  CUtensorMap tq, tk, tv;
+  if ((s = make_map_3d(&tq, q, B, Sq, D, ldq)) != DIT_OK) return s;
+  if ((s = make_map_3d(&tk, k, B, Skv, D, ldk)) != DIT_OK) return s;
+  if ((s = make_map_3d(&tv, v, B, Skv, D, ldv)) != DIT_OK) return s;
+  dit::attn::Params p;
+  p.o = reinterpret_cast<bf16*>(o);
+  p.ldo = ldo;
+  p.lse = lse;
+  p.Sq = Sq;
+  p.Skv = Skv;
+  p.H = H;
+  p.scale_log2 = softmax_scale * 1.4426950408889634f;
+  dim3 grid((unsigned)((Sq + 2 * dit::attn::BQ - 1) / (2 * dit::attn::BQ)), (unsigned)H, (unsigned)B);
+  dit::attn::attention_kernel<<<grid, dit::attn::NUM_THREADS, dit::attn::SMEM_BYTES, (cudaStream_t)stream>>>(
+      tq, tk, tv, p, g_wait_limit_ns);
+  return launch_status();
+}
+
+dit_status dit_gemm_epilogue(const dit_gemm_args* a, void* stream) {
+  if (a == nullptr || a->A == nullptr || a->W == nullptr || a->C == nullptr) return DIT_ERR_INVALID_ARG;
+  if (a->M < 1 || a->N < 32 || a->K < 8 || (a->N % 32) != 0 || (a->K % 8) != 0) return DIT_ERR_SHAPE;
+  if (a->lda < a->K || a->ldw < a->K || (a->lda % 8) || (a->ldw % 8)) return DIT_ERR_SHAPE;
+  if (!aligned16(a->A) || !aligned16(a->W) || !aligned16(a->C)) return DIT_ERR_ALIGNMENT;
+  const int split = a->C2 ? a->split_col : a->N;
+  if (a->C2 != nullptr) {
+    if (split < 0 || split > a->N || (split % 32) != 0) return DIT_ERR_SHAPE;
+    if (!aligned16(a->C2) || (a->ldc2 % 8) != 0 || a->ldc2 < a->N - split) return DIT_ERR_ALIGNMENT;
+  }
+  if ((a->ldc % 8) != 0 || a->ldc < split) return DIT_ERR_SHAPE;
+  if (a->bias && !aligned16(a->bias)) return DIT_ERR_ALIGNMENT;
+  switch (a->epi) {
+    case DIT_EPI_NONE:
+    case DIT_EPI_BIAS:
+      break;
+    case DIT_EPI_BIAS_GELU_COLS:
+      if (a->gelu_col_begin < 0 || (a->gelu_col_begin % 32) != 0) return DIT_ERR_SHAPE;
+      break;
+    case DIT_EPI_BIAS_GATED_RESIDUAL:
+      if (a->resid == nullptr || a->rows_per_batch < 1) return DIT_ERR_INVALID_ARG;
+      if (!aligned16(a->resid) || (a->ldr % 8) != 0 || a->ldr < a->N) return DIT_ERR_ALIGNMENT;
+      if (a->gate && (!aligned16(a->gate) || (a->gate_stride % 4) != 0)) return DIT_ERR_ALIGNMENT;
+      if (a->C2 != nullptr) return DIT_ERR_INVALID_ARG;
+      break;
+    default:
+      return DIT_ERR_INVALID_ARG;
+  }
+  int sms = 0;
+  dit_status s = device_setup(&sms);
+  if (s != DIT_OK) return s;
+  CUtensorMap tA, tB;
+  if ((s = make_map_2d(&tA, a->A, a->M, a->K, a->lda, dit::gemm::BM)) != DIT_OK) return s;
+  if ((s = make_map_2d(&tB, a->W, a->N, a->K, a->ldw, dit::gemm::BN)) != DIT_OK) return s;
+  dit::gemm::Epi ep;
+  ep.C = reinterpret_cast<bf16*>(a->C);
+  ep.ldc = a->ldc;
+  ep.C2 = reinterpret_cast<bf16*>(a->C2);
+  ep.ldc2 = a->ldc2;
+  ep.split_col = split;
+  ep.bias = reinterpret_cast<const bf16*>(a->bias);
+  ep.gelu_col_begin = a->gelu_col_begin;
+  ep.gate = a->gate;
+  ep.gate_stride = a->gate_stride;
+  ep.resid = reinterpret_cast<const bf16*>(a->resid);
+  ep.ldr = a->ldr;
+  ep.rows_per_batch = a->rows_per_batch > 0 ? a->rows_per_batch : a->M;
+  const int tiles = ((a->M + dit::gemm::BM - 1) / dit::gemm::BM) * ((a->N + dit::gemm::BN - 1) / dit::gemm::BN);
+  const int grid = tiles < sms ? tiles : sms;
+  cudaStream_t st = (cudaStream_t)stream;
+  const int smem = dit::gemm::SMEM_BYTES;
+  const int nt = dit::gemm::NUM_THREADS;
+  switch (a->epi) {
+    case DIT_EPI_NONE:
+      dit::gemm::gemm_kernel<DIT_EPI_NONE><<<grid, nt, smem, st>>>(tA, tB, a->M, a->N, a->K, ep, g_wait_limit_ns);
+      break;
+    case DIT_EPI_BIAS:
+      dit::gemm::gemm_kernel<DIT_EPI_BIAS><<<grid, nt, smem, st>>>(tA, tB, a->M, a->N, a->K, ep, g_wait_limit_ns);
+      break;
+    case DIT_EPI_BIAS_GELU_COLS:
+      dit::gemm::gemm_kernel<DIT_EPI_BIAS_GELU_COLS><<<grid, nt, smem, st>>>(tA, tB, a->M, a->N, a->K, ep,
+                                                                            g_wait_limit_ns);
+      break;
+    default:
+      dit::gemm::gemm_kernel<DIT_EPI_BIAS_GATED_RESIDUAL><<<grid, nt, smem, st>>>(tA, tB, a->M, a->N, a->K, ep,
+                                                                                 g_wait_limit_ns);
+      break;
+  }
+  return launch_status();
+}
+
+}  // extern "C"
+
+#include "blocks.inc"

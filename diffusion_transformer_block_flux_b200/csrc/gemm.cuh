@@ -1,0 +1,284 @@
+// bf16 GEMM C = A W^T on the 5th-generation tensor cores (tcgen05), with the
+// block's memory-bound tail fused into the epilogue: bias, GELU-tanh on a
+// column range, and the gated residual x + gate * y.
+//
+// Page: "compile_graph" (chenyy20.com), §1.1 and §2 — the block's linears are
+// the large kernels, and the elementwise tail around them is a separate HBM
+// round trip unless fused into the producing kernel.
+//
+// Design (sm_100a):
+//   - persistent CTAs, one per SM, tiles of 128 x 256 taken in M-fastest order
+//     so the CTAs running together share B tiles in L2;
+//   - warp 0: TMA producer (4-stage ring of 128x64 A and 256x64 B tiles,
+//     128-byte swizzle); warp 1: TMEM allocator + single-thread MMA issuer
+//     (tcgen05.mma 128x256x16, fp32 accumulators in TMEM); warps 2-5: epilogue
+//     (tcgen05.ld -> registers -> fused math -> bf16 stores);
+//   - two TMEM accumulators (2 x 256 columns) so the epilogue of tile i
+//     overlaps the main loop of tile i+1.
+#pragma once
+
+#include "common.cuh"
+
+namespace dit {
+namespace gemm {
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK = 64;  // 64 bf16 = 128 bytes = one swizzle row
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;
+constexpr int B_BYTES = BN * BK * 2;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int NUM_THREADS = 192;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr int BAR_BYTES = 256;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;  // + alignment slack
+constexpr uint32_t IDESC = idesc_bf16(BM, BN, 0, 0);
+
+struct Epi {
+  bf16* C;
+  int64_t ldc;
+  bf16* C2;
+  int64_t ldc2;
+  int split_col;
+  const bf16* bias;
+  int gelu_col_begin;
+  const float* gate;
+  int64_t gate_stride;
+  const bf16* resid;
+  int64_t ldr;
+  int rows_per_batch;
+};
+
+template <int EPI>
+__device__ __forceinline__ void epilogue_chunk(const uint32_t (&r)[32], int m, int n0, const Epi& ep) {
+  float v[32];
+#pragma unroll
+  for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+  if (EPI != DIT_EPI_NONE && ep.bias != nullptr) {
+    const uint4* bp = reinterpret_cast<const uint4*>(ep.bias + n0);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint4 u = __ldg(bp + q);
+      v[8 * q + 0] += bf16_lo(u.x); v[8 * q + 1] += bf16_hi(u.x);
+      v[8 * q + 2] += bf16_lo(u.y); v[8 * q + 3] += bf16_hi(u.y);
+      v[8 * q + 4] += bf16_lo(u.z); v[8 * q + 5] += bf16_hi(u.z);
+      v[8 * q + 6] += bf16_lo(u.w); v[8 * q + 7] += bf16_hi(u.w);
+    }
+  }
+  if (EPI == DIT_EPI_BIAS_GELU_COLS) {
+    if (n0 >= ep.gelu_col_begin) {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = gelu_tanh(v[j]);
+    }
+  }
+  if (EPI == DIT_EPI_BIAS_GATED_RESIDUAL) {
+    // gate == nullptr: plain residual add (gate 1)
+    const int b = m / ep.rows_per_batch;
+    const float4* gp = reinterpret_cast<const float4*>(ep.gate + b * ep.gate_stride + n0);
+    const uint4* rp = reinterpret_cast<const uint4*>(ep.resid + (int64_t)m * ep.ldr + n0);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint4 u = rp[q];
+      float4 g0 = make_float4(1.f, 1.f, 1.f, 1.f), g1 = g0;
+      if (ep.gate != nullptr) {
+        g0 = __ldg(gp + 2 * q);
+        g1 = __ldg(gp + 2 * q + 1);
+      }
+      v[8 * q + 0] = fmaf(g0.x, v[8 * q + 0], bf16_lo(u.x));
+      v[8 * q + 1] = fmaf(g0.y, v[8 * q + 1], bf16_hi(u.x));
+      v[8 * q + 2] = fmaf(g0.z, v[8 * q + 2], bf16_lo(u.y));
+      v[8 * q + 3] = fmaf(g0.w, v[8 * q + 3], bf16_hi(u.y));
+      v[8 * q + 4] = fmaf(g1.x, v[8 * q + 4], bf16_lo(u.z));
+      v[8 * q + 5] = fmaf(g1.y, v[8 * q + 5], bf16_hi(u.z));
+      v[8 * q + 6] = fmaf(g1.z, v[8 * q + 6], bf16_lo(u.w));
+      v[8 * q + 7] = fmaf(g1.w, v[8 * q + 7], bf16_hi(u.w));
+    }
+  }
+  bf16* dst;
+  if (ep.C2 != nullptr && n0 >= ep.split_col)
+    dst = ep.C2 + (int64_t)m * ep.ldc2 + (n0 - ep.split_col);
+  else
+    dst = ep.C + (int64_t)m * ep.ldc + n0;
+  uint4* dp = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint4 w;
+    w.x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
+    w.y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
+    w.z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
+    w.w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
+    dp[q] = w;
+  }
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M, int N,
+                int K, Epi ep, uint64_t wait_limit) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * A_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;   // [2]
+  uint64_t* tempty = tfull + 2;       // [2]
+  uint64_t* drain = tempty + 2;       // [1] abort-path MMA drain
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 4);  // one arrival per epilogue warp
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int num_m = (M + BM - 1) / BM;
+  const int num_n = (N + BN - 1) / BN;
+  const int num_tiles = num_m * num_n;
+  const int num_kb = (K + BK - 1) / BK;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer ----------------
+      int stage = 0;
+      uint32_t phase = 0;
+      // per stage: parity of the most recent fill we issued (for the abort drain)
+      uint32_t issued_mask = 0, issued_parity = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        const int tm = tile % num_m, tn = tile / num_m;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, wait_limit, abort_flag, SITE_GEMM_PRODUCER)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
+          tma_load_2d(sA + stage * A_BYTES, &tmA, &full[stage], kb * BK, tm * BM);
+          tma_load_2d(sB + stage * B_BYTES, &tmB, &full[stage], kb * BK, tn * BN);
+          issued_mask |= 1u << stage;
+          issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (!ok) {
+        // Let every copy we started land before the CTA exits.
+        for (int s = 0; s < STAGES; ++s)
+          if (issued_mask & (1u << s))
+            (void)mbar_wait(&full[s], (issued_parity >> s) & 1u, wait_limit, nullptr, SITE_GEMM_DRAIN);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer ----------------
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      bool issued_any = false;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1, wait_limit, abort_flag, SITE_GEMM_MMA)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(&full[stage], phase, wait_limit, abort_flag, SITE_GEMM_MMA)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + stage * A_BYTES);
+          const uint32_t b0 = smem_u32(sB + stage * B_BYTES);
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            const uint64_t ad = sdesc_sw128(a0 + k * 32, 16, 1024);
+            const uint64_t bd = sdesc_sw128(b0 + k * 32, 16, 1024);
+            umma_ss(d_tmem, ad, bd, IDESC, (kb | k) != 0 ? 1u : 0u);
+          }
+          issued_any = true;
+          umma_commit(&empty[stage]);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&tfull[acc]);
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1;
+        }
+      }
+      if (!ok && issued_any) {
+        // Make sure no MMA still writes TMEM when it is released.
+        umma_commit(drain);
+        (void)mbar_wait(drain, 0, wait_limit, nullptr, SITE_GEMM_DRAIN);
+      }
+    }
+  } else {
+    // ---------------- epilogue warps 2..5 ----------------
+    const int quad = warp & 3;  // TMEM lanes quad*32 .. quad*32+31
+    const int row_in_tile = quad * 32 + lane;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+      const int tm = tile % num_m, tn = tile / num_m;
+      bool ok = mbar_wait(&tfull[acc], acc_phase, wait_limit, abort_flag, SITE_GEMM_EPILOGUE);
+      if (!__all_sync(0xffffffffu, ok)) break;  // keep the warp converged for tcgen05.ld
+      tc_fence_after();
+      const int m = tm * BM + row_in_tile;
+      const uint32_t t_row = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * BN);
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        const int n0 = tn * BN + c * 32;
+        if (n0 >= N) break;  // warp-uniform
+        uint32_t r[32];
+        tmem_ld32(t_row + (uint32_t)(c * 32), r);
+        if (m < M) epilogue_chunk<EPI>(r, m, n0, ep);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, TMEM_COLS);
+}
+
+}  // namespace gemm
+}  // namespace dit

@@ -1,0 +1,357 @@
+/*
+ * dit.h — C ABI of the B200 (sm_100a) Flux-style DiT block forward.
+ *
+ * Sources of the operations (web pages, cited by title and section):
+ *   [CG]  "compile_graph" write-up on ChituDiffusion / Flux.1-dev (chenyy20.com):
+ *         §1.1 the memory-bound tail fused around each GEMM/attention
+ *         (LayerNorm, GELU, adaLN modulation (1+scale)*x+shift);
+ *         §2 the traced single-stream block (S=4608, dim 3072, 24 x 128, bf16)
+ *         and the 57-block model; §3.1 RoPE as complex arithmetic from position
+ *         ids, the double-stream and single-stream block lists; §6.3 attention
+ *         operands (B, S, H, D); §1.2 and §4 CUDA-graph capture with static
+ *         buffers, fixed shapes and addresses, no host sync, no allocation.
+ *   [WAN] Wan2.1 local-acceleration page (mhpq.cn), §1.1: video DiT blocks over
+ *         long (t, h, w) token sequences, dominated by self-attention.
+ *
+ * Conventions shared by every call
+ *   - dit_bf16 is the raw bit pattern of a bfloat16 value.
+ *   - Every pointer named as a device buffer must point to memory of the
+ *     current CUDA device.  The caller owns all memory; the library keeps no
+ *     pointer after a call returns, except the graph object, which keeps the
+ *     pointers it was created with until it is destroyed.
+ *   - Matrices are row-major; a leading dimension (ld*) is the distance between
+ *     rows in elements.  Unless a call says otherwise, every device pointer and
+ *     every ld * sizeof(element) must be a multiple of 16 bytes (TMA rule).
+ *   - stream is a cudaStream_t (NULL = legacy default stream).  Calls enqueue
+ *     work on it and return; they neither allocate device memory nor
+ *     synchronise, so they can be captured into a CUDA graph.  Exceptions are
+ *     named: dit_get_device_error synchronises, dit_forward_graph_create
+ *     captures on a private stream.
+ *   - No call aborts or traps.  Argument errors return a status before any work
+ *     is enqueued.  A kernel that waits longer than the wait limit (default 2 s)
+ *     on an internal barrier records DIT_ERR_TIMEOUT in the device error word,
+ *     releases its resources and exits; dit_get_device_error reports it.
+ */
+#ifndef DIT_H_
+#define DIT_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* The library is built with hidden visibility; everything declared here is
+ * exported. */
+#if defined(DIT_BUILD) && defined(__GNUC__)
+#pragma GCC visibility push(default)
+#endif
+
+typedef uint16_t dit_bf16;
+
+typedef enum {
+  DIT_OK = 0,
+  DIT_ERR_INVALID_ARG = 1,   /* null pointer, negative size, bad enum */
+  DIT_ERR_SHAPE = 2,         /* size outside what the kernel supports */
+  DIT_ERR_ALIGNMENT = 3,     /* pointer or stride not 16-byte aligned */
+  DIT_ERR_UNSUPPORTED = 4,   /* e.g. head_dim != 128, no sm_100 device */
+  DIT_ERR_CUDA = 5,          /* a CUDA runtime call failed */
+  DIT_ERR_NOT_CAPTURABLE = 6,/* the call cannot run while the stream captures */
+  DIT_ERR_TIMEOUT = 7,       /* a device-side wait ran out (device error word) */
+  DIT_ERR_WORKSPACE = 8      /* workspace pointer null or too small */
+} dit_status;
+
+const char* dit_status_string(dit_status s);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int dit_version(void);
+
+/* ------------------------------------------------------------------------
+ * Device error word and wait limit
+ * ------------------------------------------------------------------------ */
+
+/* Synchronises `stream`, then reads the device error word of the current
+ * device into *code (0 = no error; otherwise DIT_ERR_TIMEOUT in the low byte
+ * and the waiting site in the upper bytes).  Returns DIT_ERR_TIMEOUT when the
+ * word is set, DIT_OK otherwise.  Not capturable. */
+dit_status dit_get_device_error(void* stream, uint32_t* code);
+
+/* Clears the device error word of the current device (enqueued on stream). */
+dit_status dit_clear_device_error(void* stream);
+
+/* Upper bound, in nanoseconds, on any single wait inside a kernel (default
+ * 2e9).  Applies to kernels launched after the call. */
+dit_status dit_set_wait_limit_ns(uint64_t limit_ns);
+
+/* Failure-detection self test: launches one CTA that waits on a barrier that
+ * nothing ever arrives on, with the given limit.  The kernel must give up,
+ * record DIT_ERR_TIMEOUT in the device error word and exit.  Enqueued on
+ * stream; read the result with dit_get_device_error. */
+dit_status dit_selftest_wait_timeout(uint64_t limit_ns, void* stream);
+
+/* ------------------------------------------------------------------------
+ * RoPE table ([CG] §3.1: positions from ids, rotation as complex product)
+ * ------------------------------------------------------------------------ */
+
+/* rope[t][p] = (cos phi, sin phi) as two floats, phi = ids[t][a] * theta^(-2j/2P_a)
+ * for pair p = (sum of P_b for b < a) + j, where P_a = axes_pairs[a] and the
+ * pairs sum to head_dim/2 (Flux: 8, 28, 28; video: 22, 21, 21).
+ *   ids   device int32 [S][n_axes] (n_axes <= 3; each row t holds (t, h, w)).
+ *   rope  device float [S][sum P][2].  Computed in double, stored as float.
+ * Alignment: 4 bytes suffices. */
+dit_status dit_rope_table(const int32_t* ids, int S, int n_axes, const int* axes_pairs,
+                          double theta, float* rope, void* stream);
+
+/* ------------------------------------------------------------------------
+ * adaLN modulation vector ([CG] §1.1: the modulation that feeds (1+scale)*x+shift)
+ * ------------------------------------------------------------------------ */
+
+/* out[b][n] = sum_k W[n][k] * silu(vec[b][k]) + bias[n]  in fp32.
+ *   vec   device bf16 [B][ldv], W device bf16 [N][ldw] (nn.Linear layout),
+ *   bias  device bf16 [N] or NULL (= 0), out device float [B][ldo].
+ * The single block uses N = 3D chunks (shift, scale, gate); the double block
+ * and video block N = 6D (shift1, scale1, gate1, shift2, scale2, gate2).
+ * Requires K % 8 == 0, 1 <= B <= 8, K <= 8192, B * K <= 51200.  HBM-bound on
+ * the weight read. */
+dit_status dit_adaln_modulation(const dit_bf16* vec, int64_t ldv, const dit_bf16* W, int64_t ldw,
+                                const dit_bf16* bias, float* out, int64_t ldo,
+                                int B, int N, int K, void* stream);
+
+/* Same contraction with the input map and the output type chosen by flags:
+ *   DIT_VEC_SILU_IN   apply silu to the input before the product
+ *   DIT_VEC_OUT_BF16  write bf16 (round-to-nearest-even) instead of fp32 */
+enum { DIT_VEC_SILU_IN = 1, DIT_VEC_OUT_BF16 = 2 };
+dit_status dit_vec_linear(const dit_bf16* x, int64_t ldx, const dit_bf16* W, int64_t ldw,
+                          const dit_bf16* bias, void* out, int64_t ldo,
+                          int B, int N, int K, int flags, void* stream);
+
+/* ------------------------------------------------------------------------
+ * LayerNorm + adaLN modulate ([CG] §1.1)
+ * ------------------------------------------------------------------------ */
+
+/* y[r] = (1 + scale[b]) * (x[r] - mean) / sqrt(var + eps) + shift[b]
+ * per row r of D elements, b = r / S (rows of batch b are contiguous), biased
+ * variance, no LayerNorm affine.  shift/scale: device float, row b at
+ * shift + b * mod_stride; pass shift = scale = NULL for a plain LayerNorm.
+ *   x, y device bf16 [B*S][ld].  y must not alias x.  D % 8 == 0, D <= 8192. */
+dit_status dit_modulate_norm(const dit_bf16* x, int64_t ldx, const float* shift, const float* scale,
+                             int64_t mod_stride, dit_bf16* y, int64_t ldy,
+                             int B, int S, int D, float eps, void* stream);
+
+/* ------------------------------------------------------------------------
+ * QK RMSNorm + 3-axis RoPE ([CG] §3.1)
+ * ------------------------------------------------------------------------ */
+
+/* For every token t (of B*S rows) and head h, for q and for k:
+ *   u = x / sqrt(mean(x^2) + eps) * s          (x = head vector of head_dim 128)
+ *   (u[2p], u[2p+1]) <- (u0 cos - u1 sin, u0 sin + u1 cos), (cos, sin) = rope[t mod S][p]
+ *   q, k       device bf16, head h of token r at q + r*ld_in + h*128 (same for k)
+ *   q_scale, k_scale device bf16 [128] or NULL (= 1)
+ *   rope       device float [S][64][2] from dit_rope_table, or NULL (no rotation)
+ *   q_out, k_out device bf16 with row stride ld_out; may equal q, k (in place).
+ * head_dim must be 128. */
+dit_status dit_qk_norm_rope(const dit_bf16* q, const dit_bf16* k, int64_t ld_in,
+                            const dit_bf16* q_scale, const dit_bf16* k_scale, const float* rope,
+                            dit_bf16* q_out, dit_bf16* k_out, int64_t ld_out,
+                            int B, int S, int H, int head_dim, float eps, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Attention ([CG] §2 joint full attention, 24 x 128; §6.3 operands (B, S, H, D))
+ * ------------------------------------------------------------------------ */
+
+/* o[b, i, h, :] = sum_j softmax_j(scale * q[b,i,h,:] . k[b,j,h,:]) v[b,j,h,:]
+ * No mask.  Token i of batch b, head h lives at q + (b*Sq + i)*ldq + h*128 (same
+ * for k, v with Skv and o with Sq).  lse: NULL or device float [B][H][Sq] that
+ * receives the natural-log sum-exp of the scaled logits per query.
+ * head_dim must be 128; Sq, Skv >= 1 (any value: ragged tails are masked).
+ * Tensor cores (tcgen05, TMEM accumulators), online softmax.  o must not
+ * alias q, k or v. */
+dit_status dit_attention(const dit_bf16* q, const dit_bf16* k, const dit_bf16* v,
+                         int64_t ldq, int64_t ldk, int64_t ldv, dit_bf16* o, int64_t ldo,
+                         float* lse, int B, int Sq, int Skv, int H, int head_dim,
+                         float softmax_scale, void* stream);
+
+/* ------------------------------------------------------------------------
+ * GEMM with fused epilogue ([CG] §1.1 tail fused into the producing kernel;
+ * the block's linears: QKV|MLP-in and the output projection)
+ * ------------------------------------------------------------------------ */
+
+typedef enum {
+  DIT_EPI_NONE = 0,            /* C = A W^T */
+  DIT_EPI_BIAS = 1,            /* C = A W^T + bias */
+  DIT_EPI_BIAS_GELU_COLS = 2,  /* C = A W^T + bias; gelu_tanh on columns >= gelu_col_begin */
+  DIT_EPI_BIAS_GATED_RESIDUAL = 3 /* C = resid + gate[b] * (A W^T + bias) */
+} dit_epilogue;
+
+typedef struct {
+  const dit_bf16* A; int64_t lda;   /* device [M][lda], K used columns */
+  const dit_bf16* W; int64_t ldw;   /* device [N][ldw] (nn.Linear weight) */
+  const dit_bf16* bias;             /* device [N] or NULL (= 0) */
+  dit_bf16* C; int64_t ldc;         /* output of columns [0, split_col) */
+  dit_bf16* C2; int64_t ldc2;       /* output of columns [split_col, N), column n at
+                                       C2 + (n - split_col); NULL = every column to C */
+  int split_col;                    /* multiple of 32 when C2 != NULL */
+  int M, N, K;                      /* N % 32 == 0, K % 8 == 0 */
+  dit_epilogue epi;
+  int gelu_col_begin;               /* multiple of 32 */
+  const float* gate;                /* device fp32, row b at gate + b*gate_stride */
+  int64_t gate_stride;
+  const dit_bf16* resid; int64_t ldr; /* device [M][ldr]; may equal C (in place) */
+  int rows_per_batch;               /* row m belongs to batch m / rows_per_batch */
+} dit_gemm_args;
+
+/* bf16 x bf16 -> fp32 accumulate on tcgen05 (128 x 256 tiles, TMA-fed, TMEM
+ * accumulators, persistent CTAs); epilogue rounds to bf16 (nearest-even). */
+dit_status dit_gemm_epilogue(const dit_gemm_args* args, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Blocks ([CG] §2 single-stream block; §3.1 double-stream blocks; [WAN] §1.1)
+ * ------------------------------------------------------------------------ */
+
+typedef struct {
+  int B;          /* batch */
+  int S;          /* tokens per sample (text + image) */
+  int n_txt;      /* text tokens (double block: the first n_txt tokens of the
+                     joint sequence; image tokens = S - n_txt) */
+  int D;          /* model dim = H * head_dim */
+  int H;          /* heads */
+  int head_dim;   /* 128 */
+  int M;          /* MLP hidden */
+  float eps;      /* LayerNorm and RMSNorm epsilon (1e-6) */
+} dit_block_cfg;
+
+typedef struct {
+  const dit_bf16 *W_mod, *b_mod;     /* [3D][D], [3D]   (shift, scale, gate) */
+  const dit_bf16 *W1, *b1;           /* [3D+M][D], [3D+M]  rows: q | k | v | mlp */
+  const dit_bf16 *q_scale, *k_scale; /* [head_dim] */
+  const dit_bf16 *W2, *b2;           /* [D][D+M], [D]   input: attn | gelu(mlp) */
+} dit_single_weights;
+
+typedef struct {
+  const dit_bf16 *W_mod, *b_mod;     /* [6D][D] (shift1, scale1, gate1, shift2, scale2, gate2) */
+  const dit_bf16 *W_qkv, *b_qkv;     /* [3D][D] */
+  const dit_bf16 *q_scale, *k_scale; /* [head_dim] */
+  const dit_bf16 *W_proj, *b_proj;   /* [D][D] */
+  const dit_bf16 *W_mlp1, *b_mlp1;   /* [M][D] */
+  const dit_bf16 *W_mlp2, *b_mlp2;   /* [D][M] */
+} dit_stream_weights;
+
+typedef struct {
+  dit_stream_weights txt, img;
+} dit_double_weights;
+
+typedef struct {
+  const dit_bf16 *W_mod, *b_mod;     /* [6D][D] */
+  const dit_bf16 *W_qkv, *b_qkv;     /* [3D][D] self-attention q | k | v */
+  const dit_bf16 *W_o, *b_o;         /* [D][D] */
+  const dit_bf16 *W_cq, *b_cq;       /* [D][D] cross-attention query */
+  const dit_bf16 *W_ckv, *b_ckv;     /* [2D][D] cross-attention key | value (from ctx) */
+  const dit_bf16 *W_co, *b_co;       /* [D][D] */
+  const dit_bf16 *W_f1, *b_f1;       /* [M][D] */
+  const dit_bf16 *W_f2, *b_f2;       /* [D][M] */
+} dit_video_weights;
+
+/* Workspace sizes in bytes (256-byte aligned pointer required). */
+size_t dit_single_block_workspace(const dit_block_cfg* cfg);
+size_t dit_double_block_workspace(const dit_block_cfg* cfg);
+size_t dit_video_block_workspace(const dit_block_cfg* cfg, int n_ctx);
+
+/* Flux single-stream block:
+ *   (shift, scale, gate) = W_mod silu(vec) + b_mod
+ *   h = ((1+scale) LN(x) + shift) W1^T + b1 = [q | k | v | mlp]
+ *   o = attention(rope(rms(q)), rope(rms(k)), v); a = gelu_tanh(mlp)
+ *   out = x + gate * ([o | a] W2^T + b2)
+ * x, out: device bf16 [B*S][D] (out may equal x); vec: device bf16 [B][D];
+ * rope: device float [S][64][2] from dit_rope_table.  Six kernels. */
+dit_status dit_single_block_fwd(const dit_block_cfg* cfg, const dit_single_weights* w,
+                                const dit_bf16* x, const dit_bf16* vec, const float* rope,
+                                dit_bf16* out, void* ws, size_t ws_bytes, void* stream);
+
+/* Same call that additionally records events[i] (cudaEvent_t, may not be NULL)
+ * on the stream before kernel i and events[n_kernels] after the last one, so a
+ * caller can time every kernel.  n_events must be >= 7. */
+dit_status dit_single_block_fwd_profiled(const dit_block_cfg* cfg, const dit_single_weights* w,
+                                         const dit_bf16* x, const dit_bf16* vec, const float* rope,
+                                         dit_bf16* out, void* ws, size_t ws_bytes,
+                                         void* const* events, int n_events, void* stream);
+
+/* Flux double-stream block: per stream s in (txt, img) its own adaLN (6
+ * chunks), LN-modulate, QKV, QK RMSNorm; RoPE + joint attention over the
+ * sequence txt | img (rope rows in that order); then
+ *   x_s += gate1 (o_s W_proj^T + b_proj);  x_s += gate2 MLP((1+scale2) LN(x_s) + shift2)
+ * img: [B][S-n_txt][D], txt: [B][n_txt][D] device bf16; outputs may equal
+ * the inputs. */
+dit_status dit_double_block_fwd(const dit_block_cfg* cfg, const dit_double_weights* w,
+                                const dit_bf16* img, const dit_bf16* txt, const dit_bf16* vec,
+                                const float* rope, dit_bf16* img_out, dit_bf16* txt_out,
+                                void* ws, size_t ws_bytes, void* stream);
+
+/* Wan-style video block ([WAN] §1.1):
+ *   x += gate1 * SelfAttn(RoPE q, RoPE k, v) W_o^T       on (1+scale1) LN(x) + shift1
+ *   x += CrossAttn(LN(x) W_cq^T, ctx W_ckv^T) W_co^T      (no RoPE, no gate)
+ *   x += gate2 * W_f2 gelu(W_f1 ((1+scale2) LN(x) + shift2))
+ * x, out: device bf16 [B*S][D]; ctx: device bf16 [B*n_ctx][D]; no QK norm. */
+dit_status dit_video_block_fwd(const dit_block_cfg* cfg, const dit_video_weights* w,
+                               const dit_bf16* x, const dit_bf16* ctx, int n_ctx,
+                               const dit_bf16* vec, const float* rope, dit_bf16* out,
+                               void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Whole denoising loop in one CUDA graph ([CG] §1.2, §4, §7: capture once with
+ * static buffers and replay; flowmatch-euler steps)
+ * ------------------------------------------------------------------------ */
+
+typedef struct {
+  int D, H, head_dim, M;             /* block dims */
+  int channels;                      /* latent channels (16); patch 2x2 */
+  int txt_dim;                       /* raw text feature dim (4096) */
+  int t_dim;                         /* timestep embedding dim (256) */
+  int n_double, n_single;
+  const dit_double_weights* double_blocks;   /* host array [n_double] */
+  const dit_single_weights* single_blocks;   /* host array [n_single] */
+  const dit_bf16 *W_img_in, *b_img_in;       /* [D][4*channels] */
+  const dit_bf16 *W_txt_in, *b_txt_in;       /* [D][txt_dim] */
+  const dit_bf16 *W_t1, *b_t1;               /* [D][t_dim] */
+  const dit_bf16 *W_t2, *b_t2;               /* [D][D] */
+  const dit_bf16 *W_fmod, *b_fmod;           /* [2D][D] final (shift, scale) */
+  const dit_bf16 *W_out, *b_out;             /* [4*channels][D] */
+  float eps;
+} dit_model;
+
+typedef struct {
+  int n_txt, grid_h, grid_w;         /* text tokens; image grid (latent / 2) */
+  int steps;                         /* Euler steps over t_i = 1 - i/steps */
+  const dit_bf16* latent_in;         /* device bf16 [channels][2 grid_h][2 grid_w] */
+  const dit_bf16* txt;               /* device bf16 [n_txt][txt_dim] */
+  const int32_t* ids;                /* device int32 [n_txt + grid_h grid_w][3] */
+  float* latent_out;                 /* device float [channels][2 grid_h][2 grid_w] */
+} dit_loop_io;
+
+typedef struct dit_graph dit_graph;
+
+size_t dit_forward_workspace(const dit_model* m, const dit_loop_io* io);
+
+/* Runs the loop eagerly (kernel by kernel) on stream. */
+dit_status dit_forward_eager(const dit_model* m, const dit_loop_io* io, void* ws, size_t ws_bytes,
+                             void* stream);
+
+/* Captures the same kernel sequence into one CUDA graph (on a private
+ * stream) and instantiates it.  All pointers are baked in: refill io's input
+ * buffers in place between launches.  *out receives the handle. */
+dit_status dit_forward_graph_create(const dit_model* m, const dit_loop_io* io, void* ws,
+                                    size_t ws_bytes, dit_graph** out);
+dit_status dit_forward_graph_launch(dit_graph* g, void* stream);
+/* Number of kernel nodes in the graph (*n). */
+dit_status dit_forward_graph_nodes(const dit_graph* g, size_t* n);
+dit_status dit_forward_graph_destroy(dit_graph* g);
+
+#if defined(DIT_BUILD) && defined(__GNUC__)
+#pragma GCC visibility pop
+#endif
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DIT_H_ */

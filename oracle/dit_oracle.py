@@ -217,7 +217,7 @@ def single_block(x, vec, ids, w, n_heads, axes_dim=(16, 56, 56), theta=10000.0,
 
 
 def double_block(img, txt, vec, ids, w, n_heads, axes_dim=(16, 56, 56),
-                 theta=10000.0, eps=1e-6):
+                 theta=10000.0, eps=1e-6, rows_img=None, rows_txt=None):
     """Flux double-stream block ([CG] §3.1 "transformer_blocks").
 
     Each stream s in (txt, img) has its own adaLN (6 chunks), QKV linear,
@@ -228,7 +228,8 @@ def double_block(img, txt, vec, ids, w, n_heads, axes_dim=(16, 56, 56),
     RoPE from ids (ids rows: text first).  Then per stream
       x += gate1 * (o W_proj^T + b_proj)
       x += gate2 * MLP((1 + scale2) LN(x) + shift2),  MLP = W_mlp2 gelu(W_mlp1 . + b) + b.
-    Returns (img', txt')."""
+    Returns (img', txt').  rows_img / rows_txt: optional output-row subsets
+    (given together; every key and value is still computed from all tokens)."""
     streams = {"txt": txt, "img": img}
     D = img.shape[1]
     mods, qs, ks, vs = {}, {}, {}, {}
@@ -245,14 +246,20 @@ def double_block(img, txt, vec, ids, w, n_heads, axes_dim=(16, 56, 56),
     q = apply_rope(np.concatenate([qs["txt"], qs["img"]]), phi, n_heads)
     k = apply_rope(np.concatenate([ks["txt"], ks["img"]]), phi, n_heads)
     v = np.concatenate([vs["txt"], vs["img"]])
-    o = attention(q, k, v, n_heads)
     n_txt = txt.shape[0]
-    outs = {"txt": o[:n_txt], "img": o[n_txt:]}
+    if rows_img is None:
+        sel = {"txt": np.arange(n_txt), "img": np.arange(img.shape[0])}
+    else:
+        sel = {"txt": np.asarray(rows_txt), "img": np.asarray(rows_img)}
+    joint_rows = np.concatenate([sel["txt"], n_txt + sel["img"]])
+    o = attention(q, k, v, n_heads, rows=joint_rows)
+    n_sel_txt = len(sel["txt"])
+    outs = {"txt": o[:n_sel_txt], "img": o[n_sel_txt:]}
     res = {}
     for s in ("txt", "img"):
         ws = w[s]
         _, _, gate1, shift2, scale2, gate2 = mods[s]
-        x = streams[s] + gate1 * linear(outs[s], ws["W_proj"], ws["b_proj"])
+        x = streams[s][sel[s]] + gate1 * linear(outs[s], ws["W_proj"], ws["b_proj"])
         y = modulate(layer_norm(x, eps), shift2, scale2)
         hmid = gelu_tanh(linear(y, ws["W_mlp1"], ws["b_mlp1"]))
         res[s] = x + gate2 * linear(hmid, ws["W_mlp2"], ws["b_mlp2"])

@@ -1,0 +1,69 @@
+"""CPU checks of the C-ABI library: it loads, exports every symbol the header
+declares, and rejects bad arguments before touching the GPU."""
+import ctypes
+
+import pytest
+
+import diffusion_transformer_block_flux_b200 as dit
+from diffusion_transformer_block_flux_b200 import build
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return dit.lib()
+
+
+def test_exports_every_header_symbol(L):
+    names = dit.header_functions()
+    assert len(names) >= 20
+    missing = [n for n in names if not hasattr(L, n)]
+    assert not missing, missing
+    # and the binding declares a signature for each
+    assert set(names) <= set(dit._SIGS), set(names) - set(dit._SIGS)
+
+
+def test_status_strings_and_version(L):
+    assert dit.dit_status_string(0) == "ok"
+    assert "aligned" in dit.dit_status_string(3)
+    assert dit.dit_status_string(99) == "unknown status"
+    assert dit.dit_version() >= 100
+
+
+def test_argument_validation_is_host_side(L):
+    # Null pointers and bad shapes are rejected before any CUDA call.
+    assert L.dit_modulate_norm(None, 8, None, None, 0, None, 8, 1, 1, 8, 1e-6, None) == dit.DIT_ERR_INVALID_ARG
+    assert L.dit_attention(None, None, None, 128, 128, 128, None, 128, None, 1, 1, 1, 1, 128, 0.1,
+                           None) == dit.DIT_ERR_INVALID_ARG
+    bad = ctypes.c_void_p(16)
+    assert L.dit_attention(bad, bad, bad, 128, 128, 128, bad, 128, None, 1, 1, 1, 1, 64, 0.1,
+                           None) == dit.DIT_ERR_UNSUPPORTED
+    assert L.dit_qk_norm_rope(bad, bad, 128, None, None, None, bad, bad, 128, 1, 1, 1, 64, 1e-6,
+                              None) == dit.DIT_ERR_UNSUPPORTED
+    a = dit.dit_gemm_args(A=16, lda=64, W=16, ldw=64, C=16, ldc=64, M=1, N=33, K=64)
+    assert L.dit_gemm_epilogue(ctypes.byref(a), None) == dit.DIT_ERR_SHAPE
+    a = dit.dit_gemm_args(A=24, lda=64, W=16, ldw=64, C=16, ldc=64, M=1, N=64, K=64)
+    assert L.dit_gemm_epilogue(ctypes.byref(a), None) == dit.DIT_ERR_ALIGNMENT
+    assert L.dit_gemm_epilogue(None, None) == dit.DIT_ERR_INVALID_ARG
+    assert L.dit_set_wait_limit_ns(0) == dit.DIT_ERR_INVALID_ARG
+    assert L.dit_selftest_wait_timeout(0, None) == dit.DIT_ERR_INVALID_ARG
+
+
+def test_workspace_sizes(L):
+    cfg = dit.block_cfg(1, 4608, 3072, 24, 12288, n_txt=512)
+    ws = dit.dit_single_block_workspace(cfg)
+    # mod + y + qkv + [attn | mlp]
+    expect = 3 * 3072 * 4 + 4608 * 3072 * 2 * (1 + 3) + 4608 * (3072 + 12288) * 2
+    assert expect <= ws <= expect + 4 * 256
+    assert dit.dit_double_block_workspace(cfg) > 0
+    assert dit.dit_video_block_workspace(dit.block_cfg(1, 28350, 1536, 12, 8960), 512) > 0
+    bad = dit.block_cfg(1, 4608, 3072, 24, 12288)
+    bad.head_dim = 64
+    assert dit.dit_single_block_workspace(bad) == 0
+
+
+def test_block_call_rejects_small_workspace(L):
+    cfg = dit.block_cfg(1, 256, 384, 3, 1536)
+    w = dit.dit_single_weights(*([16] * 8))
+    st = L.dit_single_block_fwd(ctypes.byref(cfg), ctypes.byref(w), 16, 16, 16, 16, 256, 10, None)
+    assert st == dit.DIT_ERR_WORKSPACE

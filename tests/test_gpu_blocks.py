@@ -1,0 +1,244 @@
+"""GPU parity of the block entry points and the denoising loop against the
+fp64 oracle, through the C ABI.  Full-size workloads are checked on sampled
+output rows (the oracle still computes every key and value)."""
+import numpy as np
+import pytest
+
+from oracle import dit_oracle as O
+from diffusion_transformer_block_flux_b200 import synth
+import diffusion_transformer_block_flux_b200 as dit
+from helpers import dev_bf16, dev_tree, host_f64, parity
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def cuda():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.fail("CUDA device required for -m gpu tests")
+    dit.lib()
+    yield
+    torch.cuda.synchronize()
+
+
+def rope_for(ids, pairs=(8, 28, 28)):
+    import torch
+    rope = torch.empty((ids.shape[0], 64, 2), dtype=torch.float32, device="cuda")
+    dit.dit_rope_table(torch.from_numpy(ids).cuda(), pairs, 10000.0, rope)
+    return rope
+
+
+def workspace(nbytes):
+    import torch
+    return torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+
+
+def no_device_error():
+    st, code = dit.dit_get_device_error()
+    assert st == 0, f"device error word {code:#x}"
+
+
+def shrink(bits, e=-6):
+    """Scale bf16 values by 2^e (exact).  LayerNorm makes each branch
+    invariant to this, so the residual x no longer dominates the output and
+    the output tolerance then checks the branch itself rather than being met
+    by x carried through unchanged."""
+    return synth.f32_to_bf16_bits(synth.bf16_bits_to_f32(bits) * np.float32(2.0 ** e))
+
+
+# Branch-dominated outputs (small residual): relative L2 stays at 1e-2; the
+# max-abs bound is derived from the arithmetic.  The branch passes five bf16
+# roundings (LayerNorm out, GEMM1 out, q/k out, attention out, block out), each
+# with relative error <= 2^-9, so an element carries up to ~1% relative error,
+# and the largest elements sit near 5 RMS: max |err| <= 6e-2 RMS.
+BRANCH_MAX_ABS = 6e-2
+
+
+def check_out(got, ref, what, small_x):
+    parity(got, ref, what, max_abs_frac=BRANCH_MAX_ABS if small_x else 3e-2)
+
+
+def sample_rows(S, n_txt, k, seed=0):
+    r = np.random.default_rng(seed)
+    fixed = [0, n_txt - 1, n_txt, S - 1] if n_txt > 0 else [0, S - 1]
+    rest = r.choice(S, size=k, replace=False)
+    return np.unique(np.concatenate([fixed, rest]))
+
+
+# ---------------------------------------------------------------- single-stream block
+
+def run_single(shape, w_bits, a_bits):
+    import torch
+    w = dev_tree(w_bits)
+    x = dev_bf16(a_bits["x"])
+    vec = dev_bf16(a_bits["vec"]).reshape(1, -1)
+    rope = rope_for(a_bits["ids"])
+    cfg = dit.block_cfg(1, shape.S, shape.D, shape.H, shape.M)
+    ws = workspace(dit.dit_single_block_workspace(cfg))
+    out = torch.empty_like(x)
+    dit.dit_single_block_fwd(cfg, dit.single_weights(w), x, vec, rope, out, ws)
+    torch.cuda.synchronize()
+    return x, out
+
+
+@pytest.mark.parametrize("norm_std,small_x", [(0.0, False), (0.1, False), (0.0, True)])
+def test_single_block_tiny(norm_std, small_x):
+    s = synth.TINY
+    wb = synth.single_block_weights(s, norm_scale_std=norm_std)
+    ab = synth.block_activations(s)
+    if small_x:
+        ab["x"] = shrink(ab["x"])
+    x, out = run_single(s, wb, ab)
+    f = synth.to_f64(ab)
+    ref = O.single_block(f["x"], f["vec"], f["ids"], synth.to_f64(wb), s.H)
+    got = host_f64(out)
+    check_out(got, ref, "single block out", small_x)
+    if small_x:
+        assert np.linalg.norm(ref - f["x"]) > 4 * np.linalg.norm(f["x"])  # branch dominates
+    no_device_error()
+
+
+def test_single_block_zero_modulation_is_identity_bitwise():
+    import torch
+    s = synth.TINY
+    wb = synth.single_block_weights(s, zero_mod=True)
+    ab = synth.block_activations(s)
+    x, out = run_single(s, wb, ab)
+    assert torch.equal(out, x)
+
+
+def test_single_block_in_place_matches_out_of_place():
+    import torch
+    s = synth.TINY
+    wb = synth.single_block_weights(s)
+    ab = synth.block_activations(s)
+    x, out = run_single(s, wb, ab)
+    w = dev_tree(wb)
+    xi = dev_bf16(ab["x"])
+    cfg = dit.block_cfg(1, s.S, s.D, s.H, s.M)
+    ws = workspace(dit.dit_single_block_workspace(cfg))
+    dit.dit_single_block_fwd(cfg, dit.single_weights(w), xi, dev_bf16(ab["vec"]), rope_for(ab["ids"]), xi, ws)
+    assert torch.equal(xi, out)
+
+
+@pytest.mark.parametrize("small_x", [False, True])
+def test_single_block_full_shape_sampled_rows(small_x):
+    s = synth.FLUX
+    wb = synth.single_block_weights(s)
+    ab = synth.block_activations(s)
+    if small_x:
+        ab["x"] = shrink(ab["x"])
+    x, out = run_single(s, wb, ab)
+    rows = sample_rows(s.S, s.n_txt, 28)
+    f = synth.to_f64(ab)
+    ref = O.single_block(f["x"], f["vec"], f["ids"], synth.to_f64(wb), s.H, rows=rows)
+    got = host_f64(out)[rows]
+    check_out(got, ref, "full single block out", small_x)
+    no_device_error()
+
+
+# ---------------------------------------------------------------- double-stream block
+
+def run_double(shape, w_bits, a_bits):
+    import torch
+    w = dev_tree(w_bits)
+    img, txt = dev_bf16(a_bits["img"]), dev_bf16(a_bits["txt"])
+    vec = dev_bf16(a_bits["vec"]).reshape(1, -1)
+    rope = rope_for(a_bits["ids"])
+    cfg = dit.block_cfg(1, shape.S, shape.D, shape.H, shape.M, n_txt=shape.n_txt)
+    ws = workspace(dit.dit_double_block_workspace(cfg))
+    img_o, txt_o = torch.empty_like(img), torch.empty_like(txt)
+    dit.dit_double_block_fwd(cfg, dit.double_weights(w), img, txt, vec, rope, img_o, txt_o, ws)
+    torch.cuda.synchronize()
+    return img_o, txt_o
+
+
+@pytest.mark.parametrize("small_x", [False, True])
+def test_double_block_small(small_x):
+    s = synth.BlockShape("small_double", 40, 6, 9, 256, 2, 512)
+    wb = synth.double_block_weights(s)
+    ab = synth.double_block_activations(s)
+    if small_x:
+        ab["img"], ab["txt"] = shrink(ab["img"]), shrink(ab["txt"])
+    img_o, txt_o = run_double(s, wb, ab)
+    f = synth.to_f64(ab)
+    ref_img, ref_txt = O.double_block(f["img"], f["txt"], f["vec"], f["ids"], synth.to_f64(wb), s.H)
+    check_out(host_f64(img_o), ref_img, "double img", small_x)
+    check_out(host_f64(txt_o), ref_txt, "double txt", small_x)
+    no_device_error()
+
+
+def test_double_block_zero_modulation_identity_bitwise():
+    import torch
+    s = synth.BlockShape("small_double", 40, 6, 9, 256, 2, 512)
+    wb = synth.double_block_weights(s, zero_mod=True)
+    ab = synth.double_block_activations(s)
+    img_o, txt_o = run_double(s, wb, ab)
+    assert torch.equal(img_o, dev_bf16(ab["img"])) and torch.equal(txt_o, dev_bf16(ab["txt"]))
+
+
+@pytest.mark.parametrize("small_x", [False, True])
+def test_double_block_full_shape_sampled_rows(small_x):
+    s = synth.FLUX_DOUBLE
+    wb = synth.double_block_weights(s)
+    ab = synth.double_block_activations(s)
+    if small_x:
+        ab["img"], ab["txt"] = shrink(ab["img"]), shrink(ab["txt"])
+    img_o, txt_o = run_double(s, wb, ab)
+    n_img = s.S - s.n_txt
+    ri = sample_rows(n_img, 0, 16, seed=1)
+    rt = sample_rows(s.n_txt, 0, 8, seed=2)
+    f = synth.to_f64(ab)
+    ref_img, ref_txt = O.double_block(f["img"], f["txt"], f["vec"], f["ids"], synth.to_f64(wb), s.H,
+                                      rows_img=ri, rows_txt=rt)
+    check_out(host_f64(img_o)[ri], ref_img, "full double img", small_x)
+    check_out(host_f64(txt_o)[rt], ref_txt, "full double txt", small_x)
+    no_device_error()
+
+
+# ---------------------------------------------------------------- video block
+
+def run_video(vs, w_bits, a_bits):
+    import torch
+    w = dev_tree(w_bits)
+    x, ctx = dev_bf16(a_bits["x"]), dev_bf16(a_bits["ctx"])
+    vec = dev_bf16(a_bits["vec"]).reshape(1, -1)
+    rope = rope_for(a_bits["ids"], (22, 21, 21))
+    cfg = dit.block_cfg(1, vs.S, vs.D, vs.H, vs.M)
+    ws = workspace(dit.dit_video_block_workspace(cfg, vs.n_ctx))
+    out = torch.empty_like(x)
+    dit.dit_video_block_fwd(cfg, dit.video_weights(w), x, ctx, vs.n_ctx, vec, rope, out, ws)
+    torch.cuda.synchronize()
+    return out
+
+
+@pytest.mark.parametrize("small_x", [False, True])
+def test_video_block_small_ragged(small_x):
+    vs = synth.VideoShape("small_video", 3, 7, 9, 256, 2, 384, 40)  # S = 189: ragged tiles
+    wb = synth.video_block_weights(vs)
+    ab = synth.video_activations(vs)
+    if small_x:
+        ab["x"] = shrink(ab["x"])
+    out = run_video(vs, wb, ab)
+    f = synth.to_f64(ab)
+    ref = O.video_block(f["x"], f["ctx"], f["vec"], f["ids"], synth.to_f64(wb), vs.H)
+    got = host_f64(out)
+    check_out(got, ref, "video out", small_x)
+    no_device_error()
+
+
+@pytest.mark.parametrize("small_x", [False, True])
+def test_video_block_full_shape_sampled_rows(small_x):
+    vs = synth.VIDEO
+    wb = synth.video_block_weights(vs)
+    ab = synth.video_activations(vs)
+    if small_x:
+        ab["x"] = shrink(ab["x"])
+    out = run_video(vs, wb, ab)
+    rows = sample_rows(vs.S, 0, 24, seed=3)
+    f = synth.to_f64(ab)
+    ref = O.video_block(f["x"], f["ctx"], f["vec"], f["ids"], synth.to_f64(wb), vs.H, rows=rows)
+    got = host_f64(out)[rows]
+    check_out(got, ref, "full video out", small_x)
+    no_device_error()

@@ -1,0 +1,257 @@
+"""GPU parity of each kernel against the fp64 oracle on seeded inputs, called
+through the C ABI.  Sizes span several tiles with ragged tails."""
+import math
+
+import numpy as np
+import pytest
+
+from oracle import dit_oracle as O
+from diffusion_transformer_block_flux_b200 import synth
+import diffusion_transformer_block_flux_b200 as dit
+from helpers import dev_bf16, host_f64, parity
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def cuda():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.fail("CUDA device required for -m gpu tests")
+    dit.lib()
+    yield
+    torch.cuda.synchronize()
+
+
+def f32dev(a):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).cuda()
+
+
+def assert_no_device_error():
+    st, code = dit.dit_get_device_error()
+    assert st == 0 and code == 0, f"device error word {code:#x}"
+
+
+# ---------------------------------------------------------------- RoPE table
+
+@pytest.mark.parametrize("pairs,axes,ids_fn", [
+    ((8, 28, 28), (16, 56, 56), lambda: synth.flux_ids(64, 12, 16)),
+    ((22, 21, 21), (44, 42, 42), lambda: synth.video_ids(3, 5, 7)),
+])
+def test_rope_table(pairs, axes, ids_fn):
+    import torch
+    ids = ids_fn()
+    S = ids.shape[0]
+    rope = torch.empty((S, 64, 2), dtype=torch.float32, device="cuda")
+    dit.dit_rope_table(torch.from_numpy(ids).cuda(), pairs, 10000.0, rope)
+    phi = O.rope_angles(ids, axes)
+    got = rope.cpu().double().numpy()
+    assert np.abs(got[..., 0] - np.cos(phi)).max() < 1e-6
+    assert np.abs(got[..., 1] - np.sin(phi)).max() < 1e-6
+
+
+# ---------------------------------------------------------------- adaLN
+
+@pytest.mark.parametrize("B,N,K", [(1, 1152, 384), (2, 9216, 3072), (3, 200, 64)])
+def test_adaln_modulation(B, N, K):
+    import torch
+    vec = synth.normal_bf16(1, "vec", (B, K))
+    W = synth.normal_bf16(0, "W", (N, K), 0.02)
+    b = synth.normal_bf16(0, "b", (N,), 0.1)
+    out = torch.empty((B, N), dtype=torch.float32, device="cuda")
+    dit.dit_adaln_modulation(dev_bf16(vec), dev_bf16(W), dev_bf16(b), out)
+    ref = O.linear(O.silu(synth.bf16_bits_to_f64(vec)), synth.bf16_bits_to_f64(W), synth.bf16_bits_to_f64(b))
+    rl2, _ = parity(out.cpu().double().numpy(), ref, "adaln")
+    assert rl2 < 1e-4  # fp32 output, fp32 accumulation
+
+
+def test_vec_linear_bf16_out_no_silu():
+    import torch
+    x = synth.normal_bf16(1, "x", (1, 256))
+    W = synth.normal_bf16(0, "W", (384, 256), 0.02)
+    out = torch.empty((1, 384), dtype=torch.bfloat16, device="cuda")
+    dit.dit_vec_linear(dev_bf16(x), dev_bf16(W), None, out, flags=dit.DIT_VEC_OUT_BF16)
+    ref = O.linear(synth.bf16_bits_to_f64(x), synth.bf16_bits_to_f64(W))
+    parity(host_f64(out), ref, "vec_linear")
+
+
+# ---------------------------------------------------------------- LayerNorm + modulate
+
+@pytest.mark.parametrize("B,S,D", [(2, 100, 384), (1, 37, 3072), (1, 5, 1536), (1, 3, 8)])
+def test_modulate_norm(B, S, D):
+    import torch
+    x = synth.normal_bf16(1, "x", (B * S, D), 2.0, 0.5)
+    sh = synth.bf16_bits_to_f64(synth.normal_bf16(2, "sh", (B, D), 0.7))
+    sc = synth.bf16_bits_to_f64(synth.normal_bf16(3, "sc", (B, D), 0.7))
+    y = torch.empty((B * S, D), dtype=torch.bfloat16, device="cuda")
+    dit.dit_modulate_norm(dev_bf16(x), f32dev(sh), f32dev(sc), y, B, S, mod_stride=D)
+    xf = synth.bf16_bits_to_f64(x).reshape(B, S, D)
+    ref = O.modulate(O.layer_norm(xf), sh[:, None, :], sc[:, None, :]).reshape(B * S, D)
+    parity(host_f64(y), ref, "modulate_norm")
+    # plain LayerNorm (no modulation)
+    dit.dit_modulate_norm(dev_bf16(x), None, None, y, B, S)
+    parity(host_f64(y), O.layer_norm(xf).reshape(B * S, D), "layer_norm")
+
+
+# ---------------------------------------------------------------- QK RMSNorm + RoPE
+
+@pytest.mark.parametrize("B,nt,gh,gw,H", [(1, 64, 12, 16, 3), (2, 5, 3, 7, 2)])
+def test_qk_norm_rope(B, nt, gh, gw, H):
+    import torch
+    ids = synth.flux_ids(nt, gh, gw)
+    S = ids.shape[0]
+    D = H * 128
+    qkv = synth.normal_bf16(1, "qkv", (B * S, 3 * D), 1.5)
+    qs = synth.normal_bf16(0, "qs", (128,), 0.1, 1.0)
+    ks = synth.normal_bf16(0, "ks", (128,), 0.1, 1.0)
+    rope = torch.empty((S, 64, 2), dtype=torch.float32, device="cuda")
+    dit.dit_rope_table(torch.from_numpy(ids).cuda(), (8, 28, 28), 10000.0, rope)
+    d_qkv = dev_bf16(qkv)
+    qo = torch.empty((B * S, D), dtype=torch.bfloat16, device="cuda")
+    ko = torch.empty_like(qo)
+    dit.dit_qk_norm_rope(d_qkv[:, :D], d_qkv[:, D:2 * D], dev_bf16(qs), dev_bf16(ks), rope, qo, ko, B, S, H)
+    phi = O.rope_angles(ids, (16, 56, 56))
+    f = synth.bf16_bits_to_f64(qkv).reshape(B, S, 3 * D)
+    for which, out, sc in ((0, qo, qs), (1, ko, ks)):
+        ref = np.concatenate([O.apply_rope(O.rms_norm_heads(f[b, :, which * D:(which + 1) * D],
+                                                            synth.bf16_bits_to_f64(sc), H), phi, H)
+                              for b in range(B)])
+        parity(host_f64(out), ref, "qk_norm_rope")
+    # in place gives the same bits
+    dit.dit_qk_norm_rope(d_qkv[:, :D], d_qkv[:, D:2 * D], dev_bf16(qs), dev_bf16(ks), rope, d_qkv[:, :D],
+                         d_qkv[:, D:2 * D], B, S, H)
+    assert torch.equal(d_qkv[:, :D], qo) and torch.equal(d_qkv[:, D:2 * D], ko)
+
+
+# ---------------------------------------------------------------- GEMM + epilogues
+
+def _gemm_inputs(M, N, K, seed=0):
+    A = synth.normal_bf16(seed + 1, "A", (M, K))
+    W = synth.normal_bf16(seed, "W", (N, K), 0.02)
+    b = synth.normal_bf16(seed, "b", (N,), 0.1)
+    return A, W, b
+
+
+@pytest.mark.parametrize("M,N,K", [(300, 2688, 384), (128, 256, 64), (1, 32, 8), (256, 512, 15360),
+                                   (777, 96, 200)])
+def test_gemm_bias(M, N, K):
+    import torch
+    A, W, b = _gemm_inputs(M, N, K)
+    C = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    dit.dit_gemm_epilogue(dev_bf16(A), dev_bf16(W), C, dit.DIT_EPI_BIAS, bias=dev_bf16(b))
+    ref = O.linear(synth.bf16_bits_to_f64(A), synth.bf16_bits_to_f64(W), synth.bf16_bits_to_f64(b))
+    parity(host_f64(C), ref, "gemm_bias")
+    dit.dit_gemm_epilogue(dev_bf16(A), dev_bf16(W), C, dit.DIT_EPI_NONE)
+    parity(host_f64(C), O.linear(synth.bf16_bits_to_f64(A), synth.bf16_bits_to_f64(W)), "gemm_none")
+    assert_no_device_error()
+
+
+def test_gemm_gelu_cols_split_output():
+    import torch
+    M, D, Mh = 300, 384, 1536
+    N, K = 3 * D + Mh, D
+    A, W, b = _gemm_inputs(M, N, K, seed=5)
+    qkv = torch.empty((M, 3 * D), dtype=torch.bfloat16, device="cuda")
+    cat = torch.zeros((M, D + Mh), dtype=torch.bfloat16, device="cuda")
+    dit.dit_gemm_epilogue(dev_bf16(A), dev_bf16(W), qkv, dit.DIT_EPI_BIAS_GELU_COLS, bias=dev_bf16(b),
+                          C2=cat[:, D:], split_col=3 * D, gelu_col_begin=3 * D)
+    h = O.linear(synth.bf16_bits_to_f64(A), synth.bf16_bits_to_f64(W), synth.bf16_bits_to_f64(b))
+    parity(host_f64(qkv), h[:, :3 * D], "gemm qkv part")
+    parity(host_f64(cat[:, D:]), O.gelu_tanh(h[:, 3 * D:]), "gemm gelu part")
+    assert torch.count_nonzero(cat[:, :D]) == 0  # columns left of the split untouched
+
+
+@pytest.mark.parametrize("M,rows_per_batch,N,K,inplace", [(300, 150, 384, 1920, False), (256, 256, 3072, 512, True)])
+def test_gemm_gated_residual(M, rows_per_batch, N, K, inplace):
+    import torch
+    A, W, b = _gemm_inputs(M, N, K, seed=9)
+    B = M // rows_per_batch
+    x = synth.normal_bf16(3, "x", (M, N))
+    gate = synth.bf16_bits_to_f64(synth.normal_bf16(4, "g", (B, N), 0.7))
+    d_x = dev_bf16(x)
+    out = d_x if inplace else torch.empty_like(d_x)
+    dit.dit_gemm_epilogue(dev_bf16(A), dev_bf16(W), out, dit.DIT_EPI_BIAS_GATED_RESIDUAL, bias=dev_bf16(b),
+                          gate=f32dev(gate), gate_stride=N, resid=d_x, rows_per_batch=rows_per_batch)
+    y = O.linear(synth.bf16_bits_to_f64(A), synth.bf16_bits_to_f64(W), synth.bf16_bits_to_f64(b))
+    xf = synth.bf16_bits_to_f64(x)
+    g = np.repeat(gate, rows_per_batch, axis=0)
+    ref = xf + g * y
+    got = host_f64(out)
+    parity(got, ref, "gated residual out")
+    # with a small residual the output is the branch itself: same tolerance
+    xs = synth.f32_to_bf16_bits(synth.bf16_bits_to_f32(x) * np.float32(2.0 ** -8))
+    d_xs = dev_bf16(xs)
+    out_s = torch.empty_like(d_xs)
+    dit.dit_gemm_epilogue(dev_bf16(A), dev_bf16(W), out_s, dit.DIT_EPI_BIAS_GATED_RESIDUAL, bias=dev_bf16(b),
+                          gate=f32dev(gate), gate_stride=N, resid=d_xs, rows_per_batch=rows_per_batch)
+    xsf = synth.bf16_bits_to_f64(xs)
+    assert np.linalg.norm(g * y) > 10 * np.linalg.norm(xsf)
+    parity(host_f64(out_s), xsf + g * y, "gated residual, small residual")
+
+
+# ---------------------------------------------------------------- attention
+
+def _attn_case(B, Sq, Skv, H, qmul=1.0, seed=0):
+    D = H * 128
+    q = synth.normal_bf16(seed + 1, "q", (B * Sq, D), qmul)
+    k = synth.normal_bf16(seed + 2, "k", (B * Skv, D))
+    v = synth.normal_bf16(seed + 3, "v", (B * Skv, D))
+    return q, k, v
+
+
+@pytest.mark.parametrize("B,Sq,Skv,H,qmul", [
+    (1, 256, 256, 3, 1.0),     # tiny single-block shape
+    (2, 300, 333, 2, 1.0),     # ragged query and key tails, batch strides
+    (1, 384, 640, 1, 8.0),     # peaky logits: exercises the online max rescale
+    (1, 1000, 512, 2, 1.0),    # cross-attention shape (512 context tokens)
+    (1, 1, 1, 1, 1.0),         # single query, single key
+    (1, 129, 127, 1, 3.0),
+])
+def test_attention(B, Sq, Skv, H, qmul):
+    import torch
+    D = H * 128
+    q, k, v = _attn_case(B, Sq, Skv, H, qmul)
+    o = torch.empty((B * Sq, D), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((B, H, Sq), dtype=torch.float32, device="cuda")
+    dit.dit_attention(dev_bf16(q), dev_bf16(k), dev_bf16(v), o, B, Sq, Skv, H, lse=lse)
+    qf, kf, vf = (synth.bf16_bits_to_f64(t) for t in (q, k, v))
+    got = host_f64(o).reshape(B, Sq, D)
+    lg = lse.cpu().double().numpy()
+    for b in range(B):
+        qs, ks, vs = qf[b * Sq:(b + 1) * Sq], kf[b * Skv:(b + 1) * Skv], vf[b * Skv:(b + 1) * Skv]
+        parity(got[b], O.attention(qs, ks, vs, H), f"attention b={b}")
+        ref_lse = O.attention_lse(qs, ks, H)
+        assert np.abs(lg[b] - ref_lse).max() < 1e-3 * max(1.0, np.abs(ref_lse).max())
+    assert_no_device_error()
+
+
+def test_attention_strided_views_in_packed_buffer():
+    """q, k, v as column slices of one [S, 3D] buffer; o into a wider buffer."""
+    import torch
+    S, H = 200, 2
+    D = H * 128
+    qkv = synth.normal_bf16(7, "qkv", (S, 3 * D))
+    d = dev_bf16(qkv)
+    cat = torch.zeros((S, D + 512), dtype=torch.bfloat16, device="cuda")
+    dit.dit_attention(d[:, :D], d[:, D:2 * D], d[:, 2 * D:], cat[:, :D], 1, S, S, H)
+    f = synth.bf16_bits_to_f64(qkv)
+    parity(host_f64(cat[:, :D]), O.attention(f[:, :D], f[:, D:2 * D], f[:, 2 * D:], H), "attention packed")
+    assert torch.count_nonzero(cat[:, D:]) == 0
+
+
+# ---------------------------------------------------------------- failure detection
+
+def test_selftest_wait_times_out_and_reports():
+    """A wait on a barrier nothing arrives on ends after its limit; the error
+    word reports a timeout from the self-test site; the context stays usable."""
+    import torch
+    dit.dit_clear_device_error()
+    dit.dit_selftest_wait_timeout(50_000_000)  # 50 ms
+    st, code = dit.dit_get_device_error()
+    assert st == dit.DIT_ERR_TIMEOUT
+    assert code & 0xFF == dit.DIT_ERR_TIMEOUT and (code >> 8) == 1
+    dit.dit_clear_device_error()
+    assert dit.dit_get_device_error() == (0, 0)
+    x = torch.ones(4, device="cuda")
+    assert float((x * 2).sum()) == 8.0

@@ -280,6 +280,17 @@ def test_double_block_zero_modulation_and_stream_swap():
     np.testing.assert_allclose(txt2, img1, rtol=1e-10, atol=1e-10)
 
 
+def test_double_block_rows_subset():
+    s = _tiny_shape()
+    a = synth.to_f64(synth.double_block_activations(s))
+    w = synth.to_f64(synth.double_block_weights(s))
+    img, txt = O.double_block(a["img"], a["txt"], a["vec"], a["ids"], w, s.H)
+    ri, rt = np.array([0, 3, 7]), np.array([1, 6])
+    img_r, txt_r = O.double_block(a["img"], a["txt"], a["vec"], a["ids"], w, s.H, rows_img=ri, rows_txt=rt)
+    np.testing.assert_allclose(img_r, img[ri], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(txt_r, txt[rt], rtol=1e-12, atol=1e-12)
+
+
 def test_double_block_per_stream_independence_of_weights():
     """Changing the text stream's MLP weights leaves the image output alone
     (the streams only meet in attention, which precedes the MLP)."""
