@@ -129,6 +129,8 @@ _SIGS = {
     "dit_single_block_fwd_profiled": (i32, [ctypes.POINTER(dit_block_cfg), ctypes.POINTER(dit_single_weights),
                                             c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, size_t,
                                             ctypes.POINTER(c_void_p), i32, c_void_p]),
+    "dit_single_block_fwd_noalloc": (i32, [ctypes.POINTER(dit_block_cfg), ctypes.POINTER(dit_single_weights),
+                                           c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]),
     "dit_double_block_fwd": (i32, [ctypes.POINTER(dit_block_cfg), ctypes.POINTER(dit_double_weights),
                                    c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                    size_t, c_void_p]),
@@ -322,6 +324,14 @@ def dit_single_block_fwd(cfg, w: dit_single_weights, x, vec, rope, out, ws, stre
     else:
         arr = (c_void_p * len(events))(*[e.cuda_event for e in events])
         _call("dit_single_block_fwd_profiled", *args, arr, len(events), _stream(stream))
+
+
+def dit_single_block_fwd_noalloc(cfg, w: dit_single_weights, x, vec, rope, out, stream=None):
+    """Single-stream block without a caller workspace: for callers that may
+    not allocate device memory.  The intermediates live in a fixed 16 MiB
+    array inside the library (shared by all calls; overlapping calls race)."""
+    _call("dit_single_block_fwd_noalloc", ctypes.byref(cfg), ctypes.byref(w), _ptr(x), _ptr(vec), _ptr(rope),
+          _ptr(out), _stream(stream))
 
 
 def dit_double_block_fwd(cfg, w: dit_double_weights, img, txt, vec, rope, img_out, txt_out, ws, stream=None):

@@ -13,8 +13,8 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libdit.so")
-SOURCES = ["dit_api.cu"]
-DEPS = ["dit_api.cu", "blocks.inc", "common.cuh", "elementwise.cuh", "gemm.cuh", "attention.cuh"]
+SOURCES = ["dit_api.cu", "dit_no_alloc.cu"]
+DEPS = ["dit_api.cu", "dit_no_alloc.cu", "blocks.inc", "common.cuh", "elementwise.cuh", "gemm.cuh", "attention.cuh"]
 HEADER = os.path.join(ROOT, "include", "dit.h")
 
 

@@ -276,6 +276,27 @@ dit_status dit_single_block_fwd_profiled(const dit_block_cfg* cfg, const dit_sin
                                          dit_bf16* out, void* ws, size_t ws_bytes,
                                          void* const* events, int n_events, void* stream);
 
+/* Allocation-free variant of dit_single_block_fwd.  (The pages have no
+ * counterpart to this call; it exists for deployment.)  For callers that may
+ * not allocate device memory: plug-ins whose host framework owns all device
+ * memory through its own pool, and serving loops that must not call
+ * cudaMalloc/cudaFree once running (those calls can synchronise the device).
+ * Same inputs and outputs as dit_single_block_fwd, but the intermediates live
+ * in a 16 MiB array inside the library that each device keeps until exit.
+ *   - Configurations whose workspace (dit_single_block_workspace) exceeds
+ *     16 MiB are rejected with DIT_ERR_WORKSPACE (e.g. S=256, D=384 fits;
+ *     S=4608, D=3072 does not).
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress with that device current); make that first call
+ *     before capturing any stream into a graph.
+ *   - All calls share the one array: calls that may overlap on the GPU (other
+ *     streams, other host threads) race and must be serialised by the caller.
+ *     Nothing in the array needs clearing between calls.
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call. */
+dit_status dit_single_block_fwd_noalloc(const dit_block_cfg* cfg, const dit_single_weights* w,
+                                        const dit_bf16* x, const dit_bf16* vec, const float* rope,
+                                        dit_bf16* out, void* stream);
+
 /* Flux double-stream block: per stream s in (txt, img) its own adaLN (6
  * chunks), LN-modulate, QKV, QK RMSNorm; RoPE + joint attention over the
  * sequence txt | img (rope rows in that order); then
