@@ -35,7 +35,7 @@ UNIT = "TFLOP/s"
 WORKLOAD = "flux_single_block_S4608_D3072_H24_M12288_bf16"
 S_TXT, GRID, D, H, M = 512, 64, 3072, 24, 12288
 S = S_TXT + GRID * GRID
-KERNELS = ["adaln_modulation", "modulate_norm", "gemm_qkv_mlp_gelu", "qk_norm_rope", "attention",
+KERNELS = ["adaln_modulation", "modulate_norm", "gemm_qkv_mlp_gelu_qknorm_rope", "attention",
            "gemm_out_gated_residual"]
 
 
@@ -44,7 +44,7 @@ def block_flops(S_=S):
     attn = 4.0 * S_ * S_ * H * 128
     gemm2 = 2.0 * S_ * (D + M) * D
     mod = 2.0 * D * 3 * D
-    return {"adaln_modulation": mod, "modulate_norm": 0.0, "gemm_qkv_mlp_gelu": gemm1, "qk_norm_rope": 0.0,
+    return {"adaln_modulation": mod, "modulate_norm": 0.0, "gemm_qkv_mlp_gelu_qknorm_rope": gemm1,
             "attention": attn, "gemm_out_gated_residual": gemm2}
 
 
@@ -53,15 +53,14 @@ def block_bytes(S_=S):
     return {
         "adaln_modulation": 3 * D * D * 2 + D * 2 + 3 * D * 4,
         "modulate_norm": 2 * S_ * D * 2,
-        "gemm_qkv_mlp_gelu": S_ * D * 2 + (3 * D + M) * D * 2 + S_ * (3 * D + M) * 2,
-        "qk_norm_rope": 4 * S_ * D * 2 + S_ * 64 * 8,
+        "gemm_qkv_mlp_gelu_qknorm_rope": S_ * D * 2 + (3 * D + M) * D * 2 + S_ * (3 * D + M) * 2 + S_ * 64 * 8,
         "attention": 4 * S_ * D * 2,
         "gemm_out_gated_residual": S_ * (D + M) * 2 + D * (D + M) * 2 + 2 * S_ * D * 2,
     }
 
 
-KERNEL_BOUND = {"adaln_modulation": "hbm", "modulate_norm": "hbm", "gemm_qkv_mlp_gelu": "tensor",
-                "qk_norm_rope": "hbm", "attention": "tensor", "gemm_out_gated_residual": "tensor"}
+KERNEL_BOUND = {"adaln_modulation": "hbm", "modulate_norm": "hbm", "gemm_qkv_mlp_gelu_qknorm_rope": "tensor",
+                "attention": "tensor", "gemm_out_gated_residual": "tensor"}
 
 
 def peaks():
@@ -188,7 +187,7 @@ def run_ours(args, rank, world, local_rank):
         raise RuntimeError(f"device error word {code:#x} after warm-up")
 
     K = args.steps
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(K)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(KERNELS) + 1)] for _ in range(K)]
     for row in evs:  # torch creates the CUDA event on first record
         for e in row:
             e.record(stream)
@@ -296,7 +295,7 @@ def run_ours(args, rank, world, local_rank):
                    "l2": "inputs larger than L2 (282 MB of block weights + 0.25 GB activations per step)"},
         "ms_per_block": round(ms_per_step, 4), "blocks_per_s": round(world * 1e3 / ms_per_step, 1),
         "block_frac_of_bf16_peak": round(block_frac, 4),
-        "gpu_launches": 6 * K,
+        "gpu_launches": len(KERNELS) * K,
         "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": S * D * 2 + D * 2,
                 "d2h_bytes_per_step": S * D * 2, "steps": Ke},
         "roofline": roof, "kernels": kernels, "clocks": clocks,
@@ -400,16 +399,239 @@ def run_reference(args):
     }
 
 
+# ----------------------------------------------------------------------------
+# Further workloads (one GPU): the double-stream block, the video block, the
+# whole 57-block x 50-step loop as one CUDA graph, and the HBM-bound kernels
+# in isolation.  Each prints its own JSON line; the default workload above is
+# the headline metric.
+# ----------------------------------------------------------------------------
+
+
+def _event_time(torch, fn, K, W, stream):
+    for _ in range(W):
+        fn()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(K):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / K
+
+
+def _rand(torch, g, dev, *shape, std=1.0):
+    return (torch.randn(*shape, generator=g, device=dev, dtype=torch.float32) * std).to(torch.bfloat16)
+
+
+def _extra_line(workload, ms, flops, K, W, extra=None):
+    pk = peaks()
+    tf = flops / (ms * 1e-3) / 1e12
+    res = {"metric": f"{workload} ms & TFLOP/s (bf16)", "value": round(tf, 2), "unit": "TFLOP/s", "n_gpus": 1,
+           "steps": K, "warmup": W, "ms_per_step": round(ms, 4), "higher_is_better": True, "dtype": "bf16",
+           "data": "synthetic", "config": {"workload": workload},
+           "frac_of_bf16_peak": round(tf / pk["bf16_tflops"], 4), "algorithmic_flops": flops}
+    if extra:
+        res.update(extra)
+    return res
+
+
+def run_double(args):
+    import torch
+    import diffusion_transformer_block_flux_b200 as dit
+    from diffusion_transformer_block_flux_b200 import synth
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device=dev)
+    g.manual_seed(7)
+    w = {}
+    for st in ("txt", "img"):
+        z = lambda n: torch.zeros(n, device=dev, dtype=torch.bfloat16)
+        w[st] = {"W_mod": _rand(torch, g, dev, 6 * D, D, std=0.02), "b_mod": z(6 * D),
+                 "W_qkv": _rand(torch, g, dev, 3 * D, D, std=0.02), "b_qkv": z(3 * D),
+                 "q_scale": torch.ones(128, device=dev, dtype=torch.bfloat16),
+                 "k_scale": torch.ones(128, device=dev, dtype=torch.bfloat16),
+                 "W_proj": _rand(torch, g, dev, D, D, std=0.02), "b_proj": z(D),
+                 "W_mlp1": _rand(torch, g, dev, M, D, std=0.02), "b_mlp1": z(M),
+                 "W_mlp2": _rand(torch, g, dev, D, M, std=0.02), "b_mlp2": z(D)}
+    img, txt = _rand(torch, g, dev, S - S_TXT, D), _rand(torch, g, dev, S_TXT, D)
+    vec = _rand(torch, g, dev, 1, D)
+    ids = torch.from_numpy(synth.flux_ids(S_TXT, GRID, GRID)).to(dev)
+    rope = torch.empty((S, 64, 2), dtype=torch.float32, device=dev)
+    dit.dit_rope_table(ids, (8, 28, 28), 10000.0, rope)
+    cfg = dit.block_cfg(1, S, D, H, M, n_txt=S_TXT)
+    ws = torch.empty(dit.dit_double_block_workspace(cfg), dtype=torch.uint8, device=dev)
+    io, to = torch.empty_like(img), torch.empty_like(txt)
+    cw = dit.double_weights(w)
+    ms = _event_time(torch, lambda: dit.dit_double_block_fwd(cfg, cw, img, txt, vec, rope, io, to, ws),
+                     args.steps, args.warmup, torch.cuda.current_stream())
+    flops = 2.0 * S * D * (3 * D + D + 2 * M) + 4.0 * S * S * H * 128 + 2 * 2.0 * D * 6 * D
+    return _extra_line("flux_double_block_T512_I4096_D3072_bf16", ms, flops, args.steps, args.warmup,
+                       {"gpu_launches_per_step": 15})
+
+
+def run_video(args):
+    import torch
+    import diffusion_transformer_block_flux_b200 as dit
+    from diffusion_transformer_block_flux_b200 import synth
+    vs = synth.VIDEO
+    Dv, Mv, Sv, Hv, C = vs.D, vs.M, vs.S, vs.H, vs.n_ctx
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device=dev)
+    g.manual_seed(9)
+    shapes = {"W_mod": (6 * Dv, Dv), "W_qkv": (3 * Dv, Dv), "W_o": (Dv, Dv), "W_cq": (Dv, Dv),
+              "W_ckv": (2 * Dv, Dv), "W_co": (Dv, Dv), "W_f1": (Mv, Dv), "W_f2": (Dv, Mv)}
+    w = {}
+    for nm, shp in shapes.items():
+        w[nm] = _rand(torch, g, dev, *shp, std=0.02)
+        w["b" + nm[1:]] = torch.zeros(shp[0], device=dev, dtype=torch.bfloat16)
+    x, ctx, vec = _rand(torch, g, dev, Sv, Dv), _rand(torch, g, dev, C, Dv), _rand(torch, g, dev, 1, Dv)
+    ids = torch.from_numpy(synth.video_ids(vs.frames, vs.grid_h, vs.grid_w)).to(dev)
+    rope = torch.empty((Sv, 64, 2), dtype=torch.float32, device=dev)
+    dit.dit_rope_table(ids, (22, 21, 21), 10000.0, rope)
+    cfg = dit.block_cfg(1, Sv, Dv, Hv, Mv)
+    ws = torch.empty(dit.dit_video_block_workspace(cfg, C), dtype=torch.uint8, device=dev)
+    out = torch.empty_like(x)
+    cw = dit.video_weights(w)
+    K = max(3, args.steps // 10)
+    ms = _event_time(torch, lambda: dit.dit_video_block_fwd(cfg, cw, x, ctx, C, vec, rope, out, ws),
+                     K, args.warmup, torch.cuda.current_stream())
+    flops = (2.0 * Sv * Dv * (3 * Dv + Dv + Dv + Dv + 2 * Mv) + 2.0 * C * Dv * 2 * Dv + 4.0 * Sv * Sv * Hv * 128
+             + 4.0 * Sv * C * Hv * 128 + 2.0 * Dv * 6 * Dv)
+    return _extra_line("video_block_S28350_D1536_H12_M8960_ctx512_bf16", ms, flops, K, args.warmup,
+                       {"gpu_launches_per_step": 14})
+
+
+def run_loop(args):
+    """Flux.1-dev-shaped denoising loop at 1024^2: 19 double + 38 single blocks,
+    50 flow-match Euler steps, captured once as one CUDA graph and replayed."""
+    import torch
+    import diffusion_transformer_block_flux_b200 as dit
+    from diffusion_transformer_block_flux_b200 import synth
+    ls = synth.FLUX_LOOP
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device=dev)
+    g.manual_seed(11)
+    z = lambda n: torch.zeros(n, device=dev, dtype=torch.bfloat16)
+    one = lambda n: torch.ones(n, device=dev, dtype=torch.bfloat16)
+    r = lambda *shape: _rand(torch, g, dev, *shape, std=0.02)
+    F = 4 * ls.channels
+    mw = {"W_img_in": r(D, F), "b_img_in": z(D), "W_txt_in": r(D, ls.txt_in), "b_txt_in": z(D),
+          "W_t1": r(D, ls.t_dim), "b_t1": z(D), "W_t2": r(D, D), "b_t2": z(D),
+          "W_fmod": r(2 * D, D), "b_fmod": z(2 * D), "W_out": r(F, D), "b_out": z(F), "double": [], "single": []}
+    for _ in range(ls.n_double):
+        mw["double"].append({st: {"W_mod": r(6 * D, D), "b_mod": z(6 * D), "W_qkv": r(3 * D, D), "b_qkv": z(3 * D),
+                                  "q_scale": one(128), "k_scale": one(128), "W_proj": r(D, D), "b_proj": z(D),
+                                  "W_mlp1": r(M, D), "b_mlp1": z(M), "W_mlp2": r(D, M), "b_mlp2": z(D)}
+                             for st in ("txt", "img")})
+    for _ in range(ls.n_single):
+        mw["single"].append({"W_mod": r(3 * D, D), "b_mod": z(3 * D), "W1": r(3 * D + M, D), "b1": z(3 * D + M),
+                             "q_scale": one(128), "k_scale": one(128), "W2": r(D, D + M), "b2": z(D)})
+    model = dit.Model(mw, D=D, H=H, M=M, channels=ls.channels, txt_dim=ls.txt_in, t_dim=ls.t_dim)
+    lat = _rand(torch, g, dev, ls.channels, 2 * GRID, 2 * GRID, std=1.0)
+    txt = _rand(torch, g, dev, S_TXT, ls.txt_in, std=1.0)
+    ids = torch.from_numpy(synth.flux_ids(S_TXT, GRID, GRID)).to(dev)
+    out = torch.empty((ls.channels, 2 * GRID, 2 * GRID), dtype=torch.float32, device=dev)
+    io = dit.loop_io(S_TXT, GRID, GRID, ls.steps, lat, txt, ids, out)
+    ws = torch.empty(dit.dit_forward_workspace(model, io), dtype=torch.uint8, device=dev)
+    t0 = time.time()
+    graph = dit.Graph(model, io, ws)
+    t_build = time.time() - t0
+    stream = torch.cuda.current_stream()
+    K = max(1, min(3, args.steps))
+    ms = _event_time(torch, lambda: graph.launch(stream.cuda_stream), K, 1, stream)
+    st, code = dit.dit_get_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error word {code:#x}")
+    single = sum(block_flops().values())
+    dbl = 2.0 * S * D * (3 * D + D + 2 * M) + 4.0 * S * S * H * 128 + 2 * 2.0 * D * 6 * D
+    emb = 2.0 * (S_TXT * ls.txt_in * D + (S - S_TXT) * F * D + ls.t_dim * D + D * D) + 2.0 * D * 2 * D \
+        + 2.0 * (S - S_TXT) * D * F
+    flops = ls.steps * (ls.n_double * dbl + ls.n_single * single + emb)
+    n_nodes = graph.nodes()
+    graph.destroy()
+    return _extra_line(ls.name + "_one_cuda_graph", ms, flops, K, 1,
+                       {"s_per_image": round(ms / 1e3, 3), "graph_nodes": n_nodes,
+                        "graph_build_s": round(t_build, 2), "graph_launches_per_image": 1})
+
+
+def run_kernels(args):
+    """HBM-bound kernels alone at the Flux single-block shape.  Each iteration
+    uses the next of 4 buffer sets (> L2 in total), so every launch reads HBM."""
+    import torch
+    import diffusion_transformer_block_flux_b200 as dit
+    from diffusion_transformer_block_flux_b200 import synth
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device=dev)
+    g.manual_seed(3)
+    pk = peaks()
+    NB = 4
+    xs = [_rand(torch, g, dev, S, D) for _ in range(NB)]
+    ys = [torch.empty_like(xs[0]) for _ in range(NB)]
+    mods = [torch.randn(3 * D, generator=g, device=dev) for _ in range(NB)]
+    qkvs = [_rand(torch, g, dev, S, 3 * D) for _ in range(NB)]
+    Ws = [_rand(torch, g, dev, 3 * D, D, std=0.02) for _ in range(NB)]
+    vec = _rand(torch, g, dev, 1, D)
+    mout = torch.empty((1, 3 * D), dtype=torch.float32, device=dev)
+    ones = torch.ones(128, device=dev, dtype=torch.bfloat16)
+    ids = torch.from_numpy(synth.flux_ids(S_TXT, GRID, GRID)).to(dev)
+    rope = torch.empty((S, 64, 2), dtype=torch.float32, device=dev)
+    dit.dit_rope_table(ids, (8, 28, 28), 10000.0, rope)
+    it = [0]
+
+    def nxt():
+        it[0] = (it[0] + 1) % NB
+        return it[0]
+
+    def ln():
+        i = nxt()
+        dit.dit_modulate_norm(xs[i], mods[i][:D], mods[i][D:2 * D], ys[i], 1, S)
+
+    def qk():
+        i = nxt()
+        q = qkvs[i]
+        dit.dit_qk_norm_rope(q[:, :D], q[:, D:2 * D], ones, ones, rope, q[:, :D], q[:, D:2 * D], 1, S, H)
+
+    def ada():
+        i = nxt()
+        dit.dit_adaln_modulation(vec, Ws[i], None, mout)
+
+    K = max(20, args.steps)
+    stream = torch.cuda.current_stream()
+    res = {}
+    for name, fn, nbytes in (("modulate_norm", ln, 2 * S * D * 2),
+                             ("qk_norm_rope", qk, 4 * S * D * 2 + S * 64 * 8),
+                             ("adaln_modulation", ada, 3 * D * D * 2)):
+        ms = _event_time(torch, fn, K, args.warmup, stream)
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        res[name] = {"us": round(ms * 1e3, 2), "gbs": round(gbs, 1), "frac_of_hbm_peak": round(gbs / pk["hbm_gbs"], 4),
+                     "bytes": nbytes}
+    return {"metric": "HBM-bound kernels alone, Flux single-block shape (S=4608, D=3072)", "unit": "GB/s",
+            "n_gpus": 1, "steps": K, "warmup": args.warmup, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "hbm_kernels_S4608_D3072", "l2": "4 rotating buffer sets, > L2 in total"},
+            "hbm_peak_gbs": pk["hbm_gbs"], "kernels": res}
+
+
+EXTRA = {"double": run_double, "video": run_video, "loop": run_loop, "kernels": run_kernels}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=["single"] + sorted(EXTRA), default="single",
+                    help="single = the headline Flux single-stream block (default)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.workload != "single":
+        import torch
+        torch.cuda.set_device(0)
+        print(json.dumps(EXTRA[args.workload](args)), flush=True)
+        return 0
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

@@ -50,7 +50,8 @@ class dit_gemm_args(ctypes.Structure):
         ("C", c_void_p), ("ldc", i64), ("C2", c_void_p), ("ldc2", i64), ("split_col", i32),
         ("M", i32), ("N", i32), ("K", i32), ("epi", i32), ("gelu_col_begin", i32),
         ("gate", c_void_p), ("gate_stride", i64), ("resid", c_void_p), ("ldr", i64),
-        ("rows_per_batch", i32),
+        ("rows_per_batch", i32), ("qk_cols", i32), ("qk_norm", i32), ("qk_eps", f32),
+        ("q_scale", c_void_p), ("k_scale", c_void_p), ("rope", c_void_p), ("rope_rows", i32),
     ]
 
 
@@ -274,7 +275,8 @@ def dit_attention(q, k, v, o, B, Sq, Skv, H, softmax_scale=None, lse=None, strea
 
 
 def dit_gemm_epilogue(A, W, C, epi=DIT_EPI_NONE, bias=None, C2=None, split_col=0, gelu_col_begin=0,
-                      gate=None, gate_stride=0, resid=None, rows_per_batch=0, K=None, stream=None):
+                      gate=None, gate_stride=0, resid=None, rows_per_batch=0, K=None, qk_cols=0, qk_norm=1,
+                      qk_eps=1e-6, q_scale=None, k_scale=None, rope=None, rope_rows=0, stream=None):
     """C[:, :split] (and C2 for the rest) = epilogue(A W^T).  A [M, >=K], W [N, >=K]."""
     M = A.shape[0]
     N = W.shape[0]
@@ -283,7 +285,9 @@ def dit_gemm_epilogue(A, W, C, epi=DIT_EPI_NONE, bias=None, C2=None, split_col=0
         A=_ptr(A), lda=A.stride(0), W=_ptr(W), ldw=W.stride(0), bias=_ptr(bias), C=_ptr(C), ldc=C.stride(0),
         C2=_ptr(C2), ldc2=C2.stride(0) if C2 is not None else 0, split_col=split_col, M=M, N=N, K=K, epi=epi,
         gelu_col_begin=gelu_col_begin, gate=_ptr(gate), gate_stride=gate_stride, resid=_ptr(resid),
-        ldr=resid.stride(0) if resid is not None else 0, rows_per_batch=rows_per_batch or M)
+        ldr=resid.stride(0) if resid is not None else 0, rows_per_batch=rows_per_batch or M,
+        qk_cols=qk_cols, qk_norm=qk_norm, qk_eps=qk_eps, q_scale=_ptr(q_scale), k_scale=_ptr(k_scale),
+        rope=_ptr(rope), rope_rows=rope_rows or M)
     _call("dit_gemm_epilogue", ctypes.byref(a), _stream(stream))
 
 

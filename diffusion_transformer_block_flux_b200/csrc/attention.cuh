@@ -141,9 +141,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else if (warp == 9) {
     if (lane == 0) {
       // ---------------- MMA issuer ----------------
-      const uint32_t tS[2] = {tmem_base + 0, tmem_base + 128};
-      const uint32_t tO[2] = {tmem_base + 256, tmem_base + 384};
-      const uint32_t sQ[2] = {smem_u32(smem + OFF_Q), smem_u32(smem + OFF_Q + TILE_BYTES)};
+      const uint32_t sQ0 = smem_u32(smem + OFF_Q);
       bool ok = true;
       bool issued = false;
       auto issue_qk = [&](int t, int kst) {
@@ -151,8 +149,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
           const uint32_t off = (uint32_t)((kk >> 2) * HALF_BYTES + (kk & 3) * 32);
-          umma_ss(tS[t], sdesc_sw128(sQ[t] + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024), IDESC_QK,
-                  kk > 0 ? 1u : 0u);
+          umma_ss(tmem_base + (uint32_t)(t * 128), sdesc_sw128(sQ0 + (uint32_t)(t * TILE_BYTES) + off, 16, 1024),
+                  sdesc_sw128(kb + off, 16, 1024), IDESC_QK, kk > 0 ? 1u : 0u);
         }
       };
       auto issue_pv = [&](int t, int vst, bool acc) {
@@ -161,8 +159,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int kk = 0; kk < BKV / 16; ++kk) {
           // A: P_t in TMEM, 16 keys = 8 columns of bf16 pairs.
           // B: V MN-major; 64-d halves HALF_BYTES apart (LBO), 8-key groups 1024 B apart (SBO).
-          umma_ts(tO[t], tS[t] + (uint32_t)(kk * 8), sdesc_sw128(vb + (uint32_t)(kk * 2048), HALF_BYTES, 1024),
-                  IDESC_PV, (acc || kk > 0) ? 1u : 0u);
+          umma_ts(tmem_base + 256u + (uint32_t)(t * 128), tmem_base + (uint32_t)(t * 128 + kk * 8),
+                  sdesc_sw128(vb + (uint32_t)(kk * 2048), HALF_BYTES, 1024), IDESC_PV, (acc || kk > 0) ? 1u : 0u);
         }
       };
       if (!mbar_wait(q_full, 0, wait_limit, abort_flag, SITE_ATTN_MMA)) ok = false;
@@ -219,56 +217,83 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint32_t tS = tmem_base + lane_off + (uint32_t)(t * 128);
     const uint32_t tO = tmem_base + lane_off + 256u + (uint32_t)(t * 128);
     const float sl2 = p.scale_log2;
-    float m_run = -INFINITY;  // running max of scaled logits, log2 units
+    // Running max of the scaled logits (log2 units).  It is raised lazily:
+    // only when a tile's max exceeds it by more than 8, so P stays <= 2^8 and
+    // O is rescaled rarely (each thread owns its row, so the decision is
+    // per row; the TMEM round trip runs when any row of the warp needs it).
+    float m_run = -INFINITY;
     float l_run = 0.0f;
     bool ok = true;
     for (int j = 0; j < n_kv; ++j) {
       ok = mbar_wait(&s_full[t], j & 1, wait_limit, abort_flag, SITE_ATTN_SOFTMAX);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
-      float s[128];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tS + (uint32_t)(c * 32), r);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(r[i]);
-      }
+      uint32_t r[4][32];
+      tmem_ld32_nowait(tS + 0u, r[0]);
+      tmem_ld32_nowait(tS + 32u, r[1]);
+      tmem_ld32_nowait(tS + 64u, r[2]);
+      tmem_ld32_nowait(tS + 96u, r[3]);
+      tmem_wait_ld();
+      reg_fence32(r[0]);
+      reg_fence32(r[1]);
+      reg_fence32(r[2]);
+      reg_fence32(r[3]);
       const int valid = p.Skv - j * BKV;  // keys of this tile that exist
       if (valid < BKV) {
 #pragma unroll
-        for (int i = 0; i < 128; ++i)
-          if (i >= valid) s[i] = -INFINITY;
-      }
-      float mx = s[0];
+        for (int c = 0; c < 4; ++c)
 #pragma unroll
-      for (int i = 1; i < 128; ++i) mx = fmaxf(mx, s[i]);
-      const float m_new = fmaxf(m_run, mx * sl2);
-      const float alpha = ex2_fast(m_run - m_new);  // 0 on the first tile
-      float sum = 0.0f;
+          for (int i = 0; i < 32; ++i)
+            if (c * 32 + i >= valid) r[c][i] = __float_as_uint(-INFINITY);
+      }
+      float mx[4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float a0 = __uint_as_float(r[c][0]), a1 = __uint_as_float(r[c][1]);
+#pragma unroll
+        for (int i = 2; i < 32; i += 2) {
+          a0 = fmaxf(a0, __uint_as_float(r[c][i]));
+          a1 = fmaxf(a1, __uint_as_float(r[c][i + 1]));
+        }
+        mx[c] = fmaxf(a0, a1);
+      }
+      const float m_tile = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2;
+      const bool need = m_tile > m_run + 8.0f;  // always true on the first tile
+      const float m_new = need ? m_tile : m_run;
+      const float alpha = need ? ex2_fast(m_run - m_new) : 1.0f;  // 0 on the first tile
+      const float neg = -m_new;
+      float sum[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float p0 = ex2_fast(fmaf(s[c * 32 + 2 * i], sl2, -m_new));
-          const float p1 = ex2_fast(fmaf(s[c * 32 + 2 * i + 1], sl2, -m_new));
-          sum += p0 + p1;
+          const float x0 = fmaf(__uint_as_float(r[c][2 * i]), sl2, neg);
+          const float x1 = fmaf(__uint_as_float(r[c][2 * i + 1]), sl2, neg);
+          float p0, p1;
+          if ((i & 3) == 3) {  // a quarter of the exponentials on the FMA pipe
+            p0 = exp2_poly(x0);
+            p1 = exp2_poly(x1);
+          } else {
+            p0 = ex2_fast(x0);
+            p1 = ex2_fast(x1);
+          }
+          sum[i & 3] += p0 + p1;
           pk[i] = pack_bf16x2(p0, p1);
         }
         tmem_st16(tS + (uint32_t)(c * 16), pk);
       }
-      l_run = l_run * alpha + sum;
+      l_run = l_run * alpha + ((sum[0] + sum[1]) + (sum[2] + sum[3]));
       // Rescale O_t when any row of this warp raised its max (O_t is stable:
       // the commit we waited on covers the previous PV into O_t).
-      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
+      if (j > 0 && __any_sync(0xffffffffu, need)) {
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
-          uint32_t r[32];
-          tmem_ld32(tO + (uint32_t)(c * 32), r);
+          uint32_t o[32];
+          tmem_ld32(tO + (uint32_t)(c * 32), o);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-          tmem_st32(tO + (uint32_t)(c * 32), r);
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st32(tO + (uint32_t)(c * 32), o);
         }
       }
       m_run = m_new;

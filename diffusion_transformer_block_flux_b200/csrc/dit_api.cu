@@ -21,6 +21,7 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 constexpr int kVecSmemMax = 200 * 1024;  // staged input vectors of dit_vec_linear (B * K fp32)
+constexpr int kRowSmemMax = 200 * 1024;  // bulk-staged row rings (8 warps x 2 rows) + vectors
 uint64_t g_wait_limit_ns = 2000000000ull;
 
 struct DeviceInfo {
@@ -80,6 +81,11 @@ dit_status device_setup(int* num_sms) {
                     : nb == 4 ? (void*)dit::vec_linear_kernel<4>
                               : (void*)dit::vec_linear_kernel<8>;
           DIT_CUDA_CHECK(cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, kVecSmemMax));
+          void* fb = nb == 1   ? (void*)dit::vec_linear_bulk_kernel<1>
+                     : nb == 2 ? (void*)dit::vec_linear_bulk_kernel<2>
+                     : nb == 4 ? (void*)dit::vec_linear_bulk_kernel<4>
+                               : (void*)dit::vec_linear_bulk_kernel<8>;
+          DIT_CUDA_CHECK(cudaFuncSetAttribute(fb, cudaFuncAttributeMaxDynamicSharedMemorySize, kRowSmemMax));
         }
         if (g_encode == nullptr) {
           void* fn = nullptr;
@@ -233,6 +239,48 @@ dit_status dit_vec_linear(const dit_bf16* x, int64_t ldx, const dit_bf16* W, int
   const bf16* xb = reinterpret_cast<const bf16*>(x);
   const bf16* Wb = reinterpret_cast<const bf16*>(W);
   const bf16* bb = reinterpret_cast<const bf16*>(bias);
+  if (B == 1 && (K % 256) == 0 && K <= 4096) {
+    int rgrid = (N + 3) / 4;
+    if (rgrid > sms * 3) rgrid = sms * 3;  // three 128-thread CTAs fit per SM at ~160 registers
+#define DIT_VR_CASE(KC_)                                                                                   \
+  case KC_:                                                                                                \
+    dit::vec_linear_reg_kernel<KC_><<<rgrid, 128, 0, st>>>(xb, Wb, ldw, bb, out, N, K, flags);             \
+    return launch_status();
+    switch (K / 256) {
+      DIT_VR_CASE(1)
+      DIT_VR_CASE(2)
+      DIT_VR_CASE(3)
+      DIT_VR_CASE(4)
+      DIT_VR_CASE(6)
+      DIT_VR_CASE(8)
+      DIT_VR_CASE(12)
+      DIT_VR_CASE(16)
+      default:
+        break;
+    }
+#undef DIT_VR_CASE
+  }
+  const size_t bulk_smem = smem + (size_t)dit::kRowWarps * 2 * K * 2 + dit::kRowWarps * 2 * 8;
+  if (bulk_smem <= (size_t)kRowSmemMax) {
+    // weight rows staged through shared memory by bulk copies
+    int bgrid = (N + dit::kRowWarps - 1) / dit::kRowWarps;
+    const int per_sm = (int)(228 * 1024 / (bulk_smem + 1024));
+    const int cap = sms * (per_sm > 0 ? per_sm : 1);
+    if (bgrid > cap) bgrid = cap;
+    if (B == 1)
+      dit::vec_linear_bulk_kernel<1><<<bgrid, 256, bulk_smem, st>>>(xb, ldx, Wb, ldw, bb, out, ldo, B, N, K, flags,
+                                                                    g_wait_limit_ns);
+    else if (B <= 2)
+      dit::vec_linear_bulk_kernel<2><<<bgrid, 256, bulk_smem, st>>>(xb, ldx, Wb, ldw, bb, out, ldo, B, N, K, flags,
+                                                                    g_wait_limit_ns);
+    else if (B <= 4)
+      dit::vec_linear_bulk_kernel<4><<<bgrid, 256, bulk_smem, st>>>(xb, ldx, Wb, ldw, bb, out, ldo, B, N, K, flags,
+                                                                    g_wait_limit_ns);
+    else
+      dit::vec_linear_bulk_kernel<8><<<bgrid, 256, bulk_smem, st>>>(xb, ldx, Wb, ldw, bb, out, ldo, B, N, K, flags,
+                                                                    g_wait_limit_ns);
+    return launch_status();
+  }
   if (B == 1)
     dit::vec_linear_kernel<1><<<blocks, threads, smem, st>>>(xb, ldx, Wb, ldw, bb, out, ldo, B, N, K, flags);
   else if (B <= 2)
@@ -263,10 +311,22 @@ dit_status dit_modulate_norm(const dit_bf16* x, int64_t ldx, const float* shift,
   if ((const void*)x == (const void*)y) return DIT_ERR_INVALID_ARG;
   dit_status s = device_setup(nullptr);
   if (s != DIT_OK) return s;
-  const int threads = ((D / 8 + 31) / 32) * 32;
-  dit::modulate_norm_kernel<<<(unsigned)((int64_t)B * S), threads, 0, (cudaStream_t)stream>>>(
-      reinterpret_cast<const bf16*>(x), ldx, shift, scale, mod_stride, reinterpret_cast<bf16*>(y), ldy, S, D, eps);
-  return launch_status();
+  const int64_t rows = (int64_t)B * S;
+  const bf16* xb = reinterpret_cast<const bf16*>(x);
+  bf16* yb = reinterpret_cast<bf16*>(y);
+  cudaStream_t st = (cudaStream_t)stream;
+  {
+    // persistent row stream: D/8 threads per CTA, modulation held in registers
+    int sms = 0;
+    if ((s = device_setup(&sms)) != DIT_OK) return s;
+    const int threads = ((D / 8 + 31) / 32) * 32;
+    const int per_sm = 2048 / threads;
+    int64_t grid = (int64_t)sms * (per_sm > 0 ? per_sm : 1);
+    if (grid > rows) grid = rows;
+    dit::modulate_norm_stream_kernel<<<(unsigned)grid, threads, 0, st>>>(xb, ldx, shift, scale, mod_stride, yb,
+                                                                         ldy, rows, S, D, eps);
+    return launch_status();
+  }
 }
 
 dit_status dit_qk_norm_rope(const dit_bf16* q, const dit_bf16* k, int64_t ld_in, const dit_bf16* q_scale,
@@ -332,6 +392,15 @@ dit_status dit_gemm_epilogue(const dit_gemm_args* a, void* stream) {
   }
   if ((a->ldc % 8) != 0 || a->ldc < split) return DIT_ERR_SHAPE;
   if (a->bias && !aligned16(a->bias)) return DIT_ERR_ALIGNMENT;
+  if (a->qk_cols != 0) {
+    if (a->qk_cols < 0 || (a->qk_cols % 256) != 0 || a->qk_cols > split) return DIT_ERR_SHAPE;
+    if (a->epi == DIT_EPI_BIAS_GATED_RESIDUAL) return DIT_ERR_INVALID_ARG;
+    if ((a->q_scale && !aligned16(a->q_scale)) || (a->k_scale && !aligned16(a->k_scale)) ||
+        (a->rope && !aligned16(a->rope)))
+      return DIT_ERR_ALIGNMENT;
+    if (a->rope && a->rope_rows < 1) return DIT_ERR_INVALID_ARG;
+    if (!(a->qk_eps >= 0)) return DIT_ERR_INVALID_ARG;
+  }
   switch (a->epi) {
     case DIT_EPI_NONE:
     case DIT_EPI_BIAS:
@@ -367,6 +436,13 @@ dit_status dit_gemm_epilogue(const dit_gemm_args* a, void* stream) {
   ep.resid = reinterpret_cast<const bf16*>(a->resid);
   ep.ldr = a->ldr;
   ep.rows_per_batch = a->rows_per_batch > 0 ? a->rows_per_batch : a->M;
+  ep.qk_cols = a->qk_cols;
+  ep.qk_norm = a->qk_norm;
+  ep.qk_eps = a->qk_eps;
+  ep.q_scale = reinterpret_cast<const bf16*>(a->q_scale);
+  ep.k_scale = reinterpret_cast<const bf16*>(a->k_scale);
+  ep.rope = reinterpret_cast<const float2*>(a->rope);
+  ep.rope_rows = a->rope_rows > 0 ? a->rope_rows : a->M;
   const int tiles = ((a->M + dit::gemm::BM - 1) / dit::gemm::BM) * ((a->N + dit::gemm::BN - 1) / dit::gemm::BN);
   const int grid = tiles < sms ? tiles : sms;
   cudaStream_t st = (cudaStream_t)stream;

@@ -20,72 +20,237 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-__device__ __forceinline__ float block_sum(float v, float* red) {
+
+// ---------------------------------------------------------------------------
+// LayerNorm + modulate, persistent row stream: a CTA of D/8 threads walks rows
+// blockIdx.x, blockIdx.x + gridDim.x, ...; thread t always owns columns
+// [8t, 8t+8), so its 8 shift and 8 scale values stay in registers for every
+// row of the batch, and it loads the next row's 16 bytes before reducing the
+// current one.  Per row the only memory traffic is one 16-byte load and one
+// 16-byte store per thread.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(1024) modulate_norm_stream_kernel(const bf16* __restrict__ x, int64_t ldx,
+                                                                    const float* __restrict__ shift,
+                                                                    const float* __restrict__ scale,
+                                                                    int64_t mod_stride, bf16* __restrict__ y,
+                                                                    int64_t ldy, int64_t rows, int S, int D,
+                                                                    float eps) {
+  __shared__ float red[2][32];
+  const int c0 = threadIdx.x * 8;
+  const bool active = c0 < D;
+  const float invD = 1.0f / (float)D;
+  int64_t r = blockIdx.x;
+  uint4 cur = make_uint4(0, 0, 0, 0);
+  if (active && r < rows) cur = __ldcs(reinterpret_cast<const uint4*>(x + r * ldx + c0));
+  int cur_b = -1;
+  float sh[8], sc1[8];
   const int w = threadIdx.x >> 5, l = threadIdx.x & 31, nw = blockDim.x >> 5;
-  v = warp_sum(v);
-  __syncthreads();  // red may still be read from a previous call
-  if (l == 0) red[w] = v;
-  __syncthreads();
-  float t = (l < nw) ? red[l] : 0.0f;
-  return warp_sum(t);
+  int par = 0;
+  for (; r < rows; r += gridDim.x) {
+    const int64_t rn = r + gridDim.x;
+    uint4 nxt = make_uint4(0, 0, 0, 0);
+    if (active && rn < rows) nxt = __ldcs(reinterpret_cast<const uint4*>(x + rn * ldx + c0));
+    const int b = (int)(r / S);
+    if (b != cur_b) {  // new batch row: refresh this thread's modulation (uniform across the CTA)
+      cur_b = b;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        sh[i] = 0.0f;
+        sc1[i] = 1.0f;
+      }
+      if (active && shift != nullptr) {
+        const float4* ps = reinterpret_cast<const float4*>(shift + b * mod_stride + c0);
+        const float4* pc = reinterpret_cast<const float4*>(scale + b * mod_stride + c0);
+        const float4 a0 = __ldg(ps), a1 = __ldg(ps + 1), b0 = __ldg(pc), b1 = __ldg(pc + 1);
+        sh[0] = a0.x; sh[1] = a0.y; sh[2] = a0.z; sh[3] = a0.w; sh[4] = a1.x; sh[5] = a1.y; sh[6] = a1.z; sh[7] = a1.w;
+        sc1[0] = 1.f + b0.x; sc1[1] = 1.f + b0.y; sc1[2] = 1.f + b0.z; sc1[3] = 1.f + b0.w;
+        sc1[4] = 1.f + b1.x; sc1[5] = 1.f + b1.y; sc1[6] = 1.f + b1.z; sc1[7] = 1.f + b1.w;
+      }
+    }
+    const float v[8] = {bf16_lo(cur.x), bf16_hi(cur.x), bf16_lo(cur.y), bf16_hi(cur.y),
+                        bf16_lo(cur.z), bf16_hi(cur.z), bf16_lo(cur.w), bf16_hi(cur.w)};
+    // mean (inactive threads hold zeros)
+    float t = ((v[0] + v[1]) + (v[2] + v[3])) + ((v[4] + v[5]) + (v[6] + v[7]));
+    t = warp_sum(t);
+    if (l == 0) red[par][w] = t;
+    __syncthreads();
+    float tot = (l < nw) ? red[par][l] : 0.0f;
+    const float mean = warp_sum(tot) * invD;
+    // centred second moment from the same registers
+    float q = 0.0f;
+    if (active) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float d = v[i] - mean;
+        q = fmaf(d, d, q);
+      }
+    }
+    q = warp_sum(q);
+    par ^= 1;  // the other buffer: no thread can still be reading it
+    if (l == 0) red[par][w] = q;
+    __syncthreads();
+    tot = (l < nw) ? red[par][l] : 0.0f;
+    const float rstd = rsqrtf(warp_sum(tot) * invD + eps);
+    par ^= 1;
+    if (active) {
+      uint4 o;
+      o.x = pack_bf16x2(fmaf(sc1[0], (v[0] - mean) * rstd, sh[0]), fmaf(sc1[1], (v[1] - mean) * rstd, sh[1]));
+      o.y = pack_bf16x2(fmaf(sc1[2], (v[2] - mean) * rstd, sh[2]), fmaf(sc1[3], (v[3] - mean) * rstd, sh[3]));
+      o.z = pack_bf16x2(fmaf(sc1[4], (v[4] - mean) * rstd, sh[4]), fmaf(sc1[5], (v[5] - mean) * rstd, sh[5]));
+      o.w = pack_bf16x2(fmaf(sc1[6], (v[6] - mean) * rstd, sh[6]), fmaf(sc1[7], (v[7] - mean) * rstd, sh[7]));
+      *reinterpret_cast<uint4*>(y + r * ldy + c0) = o;
+    }
+    cur = nxt;
+  }
 }
 
 // ---------------------------------------------------------------------------
-// LayerNorm + modulate: one CTA per row, 8 bf16 (16 bytes) per thread.
-// Two-pass statistics from registers (mean, then centred second moment).
+// adaLN / vector x weight with the (mapped) input vector held in registers:
+// lane l of every warp owns input columns {8(l + 32j) .. +8}, j < KC, so each
+// weight row is read with KC 16-byte loads per lane and multiplied against
+// registers; no shared-memory traffic per row.  One warp per output feature,
+// features dealt round-robin over the grid.  B == 1 only (the block's
+// conditioning vector); other batch sizes use vec_linear_kernel.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(1024) modulate_norm_kernel(const bf16* __restrict__ x, int64_t ldx,
-                                                             const float* __restrict__ shift,
-                                                             const float* __restrict__ scale,
-                                                             int64_t mod_stride, bf16* __restrict__ y,
-                                                             int64_t ldy, int S, int D, float eps) {
-  __shared__ float red[32];
-  const int64_t row = blockIdx.x;
-  const int b = (int)(row / S);
-  const int c0 = threadIdx.x * 8;
-  const bool active = c0 < D;
-  float v[8];
-  if (active) {
-    uint4 u = __ldcs(reinterpret_cast<const uint4*>(x + row * ldx + c0));
-    v[0] = bf16_lo(u.x); v[1] = bf16_hi(u.x); v[2] = bf16_lo(u.y); v[3] = bf16_hi(u.y);
-    v[4] = bf16_lo(u.z); v[5] = bf16_hi(u.z); v[6] = bf16_lo(u.w); v[7] = bf16_hi(u.w);
-  } else {
+template <int KC>
+__global__ void __launch_bounds__(128) vec_linear_reg_kernel(const bf16* __restrict__ x,
+                                                             const bf16* __restrict__ W, int64_t ldw,
+                                                             const bf16* __restrict__ bias, void* out, int N, int K,
+                                                             int flags) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float xv[KC * 8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = 0.0f;
-  }
-  float s = 0.0f;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) s += v[i];
-  const float mean = block_sum(s, red) / (float)D;
-  float q = 0.0f;
-  if (active) {
+  for (int j = 0; j < KC; ++j) {
+    const int k0 = (lane + 32 * j) * 8;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      const float d = v[i] - mean;
-      q = fmaf(d, d, q);
+      float z = 0.0f;
+      if (k0 + i < K) {
+        z = __bfloat162float(x[k0 + i]);
+        if (flags & DIT_VEC_SILU_IN) z = silu(z);
+      }
+      xv[j * 8 + i] = z;
     }
   }
-  const float var = block_sum(q, red) / (float)D;
-  const float rstd = rsqrtf(var + eps);
-  if (!active) return;
-  float sh[8], sc[8];
-  if (shift != nullptr) {
-    const float4* ps = reinterpret_cast<const float4*>(shift + b * mod_stride + c0);
-    const float4* pc = reinterpret_cast<const float4*>(scale + b * mod_stride + c0);
-    float4 a0 = __ldg(ps), a1 = __ldg(ps + 1), b0 = __ldg(pc), b1 = __ldg(pc + 1);
-    sh[0] = a0.x; sh[1] = a0.y; sh[2] = a0.z; sh[3] = a0.w; sh[4] = a1.x; sh[5] = a1.y; sh[6] = a1.z; sh[7] = a1.w;
-    sc[0] = b0.x; sc[1] = b0.y; sc[2] = b0.z; sc[3] = b0.w; sc[4] = b1.x; sc[5] = b1.y; sc[6] = b1.z; sc[7] = b1.w;
-  } else {
+  const int nw = gridDim.x * 4;
+  for (int n = blockIdx.x * 4 + warp; n < N; n += nw) {
+    const bf16* wr = W + (int64_t)n * ldw;
+    uint4 wv[KC];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) { sh[i] = 0.0f; sc[i] = 0.0f; }
+    for (int j = 0; j < KC; ++j) {
+      const int k0 = (lane + 32 * j) * 8;
+      wv[j] = (k0 < K) ? __ldcs(reinterpret_cast<const uint4*>(wr + k0)) : make_uint4(0, 0, 0, 0);
+    }
+    float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+    for (int j = 0; j < KC; ++j) {
+      const uint4 u = wv[j];
+      a0 = fmaf(bf16_lo(u.x), xv[j * 8 + 0], a0); a1 = fmaf(bf16_hi(u.x), xv[j * 8 + 1], a1);
+      a0 = fmaf(bf16_lo(u.y), xv[j * 8 + 2], a0); a1 = fmaf(bf16_hi(u.y), xv[j * 8 + 3], a1);
+      a0 = fmaf(bf16_lo(u.z), xv[j * 8 + 4], a0); a1 = fmaf(bf16_hi(u.z), xv[j * 8 + 5], a1);
+      a0 = fmaf(bf16_lo(u.w), xv[j * 8 + 6], a0); a1 = fmaf(bf16_hi(u.w), xv[j * 8 + 7], a1);
+    }
+    const float a = warp_sum(a0 + a1) + (bias ? __bfloat162float(bias[n]) : 0.0f);
+    if (lane == 0) {
+      if (flags & DIT_VEC_OUT_BF16)
+        reinterpret_cast<bf16*>(out)[n] = __float2bfloat16_rn(a);
+      else
+        reinterpret_cast<float*>(out)[n] = a;
+    }
   }
-  float o[8];
+}
+
+// ---------------------------------------------------------------------------
+// Bulk-copy staging of rows: 8 warps per CTA, each warp owns a 2-deep ring of
+// row buffers in shared memory; lane 0 starts the copy of the warp's next row
+// before the warp works on the current one.
+// ---------------------------------------------------------------------------
+constexpr int kRowWarps = 8;
+
+// adaLN / vector x weight with bulk-copy staging of the weight rows (same
+// warp-private 2-deep ring).  out[b][n] = sum_k W[n][k] f(x[b][k]) + bias[n].
+template <int NB>
+__global__ void __launch_bounds__(256) vec_linear_bulk_kernel(const bf16* __restrict__ x, int64_t ldx,
+                                                              const bf16* __restrict__ W, int64_t ldw,
+                                                              const bf16* __restrict__ bias, void* out, int64_t ldo,
+                                                              int B, int N, int K, int flags, uint64_t wait_limit) {
+  extern __shared__ __align__(128) uint8_t sm[];
+  const int ROW_BYTES = K * 2;
+  float* xs = reinterpret_cast<float*>(sm);  // [B][K]
+  uint8_t* rings = sm + (size_t)B * K * 4;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint8_t* buf = rings + (size_t)warp * 2 * ROW_BYTES;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(rings + (size_t)kRowWarps * 2 * ROW_BYTES) + warp * 2;
+  const int64_t nw = (int64_t)gridDim.x * kRowWarps;
+  int64_t n = (int64_t)blockIdx.x * kRowWarps + warp;
+  if (lane == 0) {
+    mbar_init(&bar[0], 1);
+    mbar_init(&bar[1], 1);
+    fence_mbar_init();
+    if (n < N) {
+      mbar_arrive_expect_tx(&bar[0], ROW_BYTES);
+      bulk_load(buf, W + n * ldw, ROW_BYTES, &bar[0]);
+    }
+  }
+  for (int i = threadIdx.x; i < B * K; i += blockDim.x) {
+    const int b = i / K, kk = i % K;
+    float z = __bfloat162float(x[b * ldx + kk]);
+    if (flags & DIT_VEC_SILU_IN) z = silu(z);
+    xs[i] = z;
+  }
+  __syncthreads();
+  int st = 0;
+  uint32_t ph0 = 0, ph1 = 0;
+  for (; n < N; n += nw) {
+    const int64_t nn = n + nw;
+    if (nn < N && lane == 0) {
+      fence_proxy_async_smem();
+      mbar_arrive_expect_tx(&bar[st ^ 1], ROW_BYTES);
+      bulk_load(buf + (st ^ 1) * ROW_BYTES, W + nn * ldw, ROW_BYTES, &bar[st ^ 1]);
+    }
+    const uint32_t ph = st ? ph1 : ph0;
+    bool ok = mbar_wait(&bar[st], ph, wait_limit, nullptr, SITE_ROWS);
+    if (!__all_sync(0xffffffffu, ok)) {
+      if (lane == 0 && nn < N) (void)mbar_wait(&bar[st ^ 1], st ? ph0 : ph1, wait_limit, nullptr, SITE_ROWS);
+      break;
+    }
+    if (st) ph1 ^= 1; else ph0 ^= 1;
+    const uint4* wp = reinterpret_cast<const uint4*>(buf + st * ROW_BYTES);
+    float acc[NB];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) o[i] = fmaf(1.0f + sc[i], (v[i] - mean) * rstd, sh[i]);
-  uint4 w;
-  w.x = pack_bf16x2(o[0], o[1]); w.y = pack_bf16x2(o[2], o[3]);
-  w.z = pack_bf16x2(o[4], o[5]); w.w = pack_bf16x2(o[6], o[7]);
-  *reinterpret_cast<uint4*>(y + row * ldy + c0) = w;
+    for (int b = 0; b < NB; ++b) acc[b] = 0.0f;
+    for (int v = lane; v < K / 8; v += 32) {
+      const uint4 u = wp[v];
+      const float w8[8] = {bf16_lo(u.x), bf16_hi(u.x), bf16_lo(u.y), bf16_hi(u.y),
+                           bf16_lo(u.z), bf16_hi(u.z), bf16_lo(u.w), bf16_hi(u.w)};
+#pragma unroll
+      for (int b = 0; b < NB; ++b) {
+        if (b < B) {
+          const float4* xp = reinterpret_cast<const float4*>(xs + b * K + v * 8);
+          const float4 x0 = xp[0], x1 = xp[1];
+          acc[b] = fmaf(w8[0], x0.x, acc[b]); acc[b] = fmaf(w8[1], x0.y, acc[b]);
+          acc[b] = fmaf(w8[2], x0.z, acc[b]); acc[b] = fmaf(w8[3], x0.w, acc[b]);
+          acc[b] = fmaf(w8[4], x1.x, acc[b]); acc[b] = fmaf(w8[5], x1.y, acc[b]);
+          acc[b] = fmaf(w8[6], x1.z, acc[b]); acc[b] = fmaf(w8[7], x1.w, acc[b]);
+        }
+      }
+    }
+    const float bv = bias ? __bfloat162float(bias[n]) : 0.0f;
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      if (b < B) {
+        const float a = warp_sum(acc[b]) + bv;
+        if (lane == 0) {
+          if (flags & DIT_VEC_OUT_BF16)
+            reinterpret_cast<bf16*>(out)[b * ldo + n] = __float2bfloat16_rn(a);
+          else
+            reinterpret_cast<float*>(out)[b * ldo + n] = a;
+        }
+      }
+    }
+    __syncwarp();
+    st ^= 1;
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -200,6 +365,35 @@ __global__ void __launch_bounds__(256) vec_linear_kernel(const bf16* __restrict_
 #pragma unroll
     for (int b = 0; b < NB; ++b) acc[b] = 0.0f;
     const bf16* wr = W + (int64_t)n * ldw;
+    if (K <= 16 * 256) {
+      // issue the whole row's loads first (up to 16 x 16 bytes per lane)
+      uint4 wv[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int k0 = j * 256 + lane * 8;
+        wv[j] = (k0 < K) ? __ldcs(reinterpret_cast<const uint4*>(wr + k0)) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int k0 = j * 256 + lane * 8;
+        if (k0 < K) {
+          const uint4 u = wv[j];
+          const float w[8] = {bf16_lo(u.x), bf16_hi(u.x), bf16_lo(u.y), bf16_hi(u.y),
+                              bf16_lo(u.z), bf16_hi(u.z), bf16_lo(u.w), bf16_hi(u.w)};
+#pragma unroll
+          for (int b = 0; b < NB; ++b) {
+            if (b < B) {
+              const float4* xp = reinterpret_cast<const float4*>(xs + b * K + k0);
+              const float4 x0 = xp[0], x1 = xp[1];
+              acc[b] = fmaf(w[0], x0.x, acc[b]); acc[b] = fmaf(w[1], x0.y, acc[b]);
+              acc[b] = fmaf(w[2], x0.z, acc[b]); acc[b] = fmaf(w[3], x0.w, acc[b]);
+              acc[b] = fmaf(w[4], x1.x, acc[b]); acc[b] = fmaf(w[5], x1.y, acc[b]);
+              acc[b] = fmaf(w[6], x1.z, acc[b]); acc[b] = fmaf(w[7], x1.w, acc[b]);
+            }
+          }
+        }
+      }
+    } else
     for (int k0 = lane * 8; k0 < K; k0 += 256) {
       uint4 u = __ldcs(reinterpret_cast<const uint4*>(wr + k0));
       float w[8] = {bf16_lo(u.x), bf16_hi(u.x), bf16_lo(u.y), bf16_hi(u.y),

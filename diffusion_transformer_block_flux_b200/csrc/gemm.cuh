@@ -48,7 +48,90 @@ struct Epi {
   const bf16* resid;
   int64_t ldr;
   int rows_per_batch;
+  // fused QK RMSNorm + RoPE on output columns [0, qk_cols) (0 = off):
+  // [0, qk_cols/2) are q heads, [qk_cols/2, qk_cols) k heads, 128 columns each
+  int qk_cols;
+  int qk_norm;
+  float qk_eps;
+  const bf16* q_scale;
+  const bf16* k_scale;
+  const float2* rope;  // [rope_rows][64] (cos, sin); row of output row m = m % rope_rows
+  int rope_rows;
 };
+
+// One 128-column head of q or k for output row m: bias, optional RMSNorm with
+// its per-dimension scale, rotation of each pair (2p, 2p+1) by the RoPE table,
+// bf16 store.  Two passes over TMEM (sum of squares, then transform) keep the
+// register footprint at one 32-column chunk.
+__device__ __forceinline__ void epilogue_qk_head(uint32_t t_head, int m, int n_head, const Epi& ep, bool row_ok) {
+  float ss = 0.0f;
+  if (ep.qk_norm) {
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+      uint32_t r[32];
+      tmem_ld32(t_head + (uint32_t)(c * 32), r);
+      const uint4* bp = reinterpret_cast<const uint4*>(ep.bias + n_head + c * 32);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint4 u = ep.bias ? __ldg(bp + q) : make_uint4(0, 0, 0, 0);
+        const float b8[8] = {bf16_lo(u.x), bf16_hi(u.x), bf16_lo(u.y), bf16_hi(u.y),
+                             bf16_lo(u.z), bf16_hi(u.z), bf16_lo(u.w), bf16_hi(u.w)};
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float v = __uint_as_float(r[8 * q + j]) + b8[j];
+          ss = fmaf(v, v, ss);
+        }
+      }
+    }
+  }
+  const float rs = ep.qk_norm ? rsqrtf(ss * (1.0f / 128.0f) + ep.qk_eps) : 1.0f;
+  const bool is_k = n_head >= (ep.qk_cols >> 1);
+  const bf16* sc = is_k ? ep.k_scale : ep.q_scale;
+  const float2* rrow = ep.rope ? ep.rope + (int64_t)(m % ep.rope_rows) * 64 : nullptr;
+  bf16* dst = ep.C + (int64_t)m * ep.ldc + n_head;
+#pragma unroll 1
+  for (int c = 0; c < 4; ++c) {
+    uint32_t r[32];
+    tmem_ld32(t_head + (uint32_t)(c * 32), r);
+    if (!row_ok) continue;
+    float v[32];
+    const uint4* bp = reinterpret_cast<const uint4*>(ep.bias + n_head + c * 32);
+    const uint4* sp = reinterpret_cast<const uint4*>(sc + c * 32);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint4 u = ep.bias ? __ldg(bp + q) : make_uint4(0, 0, 0, 0);
+      uint4 w = sc ? __ldg(sp + q) : make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
+      const float b8[8] = {bf16_lo(u.x), bf16_hi(u.x), bf16_lo(u.y), bf16_hi(u.y),
+                           bf16_lo(u.z), bf16_hi(u.z), bf16_lo(u.w), bf16_hi(u.w)};
+      const float s8[8] = {bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y),
+                           bf16_lo(w.z), bf16_hi(w.z), bf16_lo(w.w), bf16_hi(w.w)};
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[8 * q + j] = (__uint_as_float(r[8 * q + j]) + b8[j]) * rs * s8[j];
+    }
+    if (rrow != nullptr) {
+      const float4* tp = reinterpret_cast<const float4*>(rrow + c * 16);
+#pragma unroll
+      for (int p2 = 0; p2 < 8; ++p2) {
+        const float4 cs = __ldg(tp + p2);  // pairs 2*p2, 2*p2+1 of this chunk
+        const float a0 = v[4 * p2], a1 = v[4 * p2 + 1], b0 = v[4 * p2 + 2], b1 = v[4 * p2 + 3];
+        v[4 * p2] = a0 * cs.x - a1 * cs.y;
+        v[4 * p2 + 1] = a0 * cs.y + a1 * cs.x;
+        v[4 * p2 + 2] = b0 * cs.z - b1 * cs.w;
+        v[4 * p2 + 3] = b0 * cs.w + b1 * cs.z;
+      }
+    }
+    uint4* dp = reinterpret_cast<uint4*>(dst + c * 32);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint4 w;
+      w.x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
+      w.y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
+      w.z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
+      w.w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
+      dp[q] = w;
+    }
+  }
+}
 
 template <int EPI>
 __device__ __forceinline__ void epilogue_chunk(const uint32_t (&r)[32], int m, int n0, const Epi& ep) {
@@ -260,6 +343,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int c = 0; c < BN / 32; ++c) {
         const int n0 = tn * BN + c * 32;
         if (n0 >= N) break;  // warp-uniform
+        if (EPI != DIT_EPI_BIAS_GATED_RESIDUAL && n0 < ep.qk_cols) {
+          // a whole 128-column q/k head (heads are 128-aligned, tiles 256-aligned)
+          epilogue_qk_head(t_row + (uint32_t)(c * 32), m, n0, ep, m < M);
+          c += 3;
+          continue;
+        }
         uint32_t r[32];
         tmem_ld32(t_row + (uint32_t)(c * 32), r);
         if (m < M) epilogue_chunk<EPI>(r, m, n0, ep);

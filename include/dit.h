@@ -199,6 +199,18 @@ typedef struct {
   int64_t gate_stride;
   const dit_bf16* resid; int64_t ldr; /* device [M][ldr]; may equal C (in place) */
   int rows_per_batch;               /* row m belongs to batch m / rows_per_batch */
+  /* Optional QK RMSNorm + RoPE fused into the epilogue ([CG] §3.1), the same
+   * operation as dit_qk_norm_rope applied to output columns [0, qk_cols):
+   * columns [0, qk_cols/2) are q heads and [qk_cols/2, qk_cols) k heads, 128
+   * columns per head.  qk_cols = 0 disables it; otherwise qk_cols % 256 == 0,
+   * epi is DIT_EPI_NONE/BIAS/BIAS_GELU_COLS and those columns go to C. */
+  int qk_cols;
+  int qk_norm;                      /* 1: RMSNorm each head (eps qk_eps) then scale */
+  float qk_eps;
+  const dit_bf16* q_scale;          /* device [128] or NULL (= 1) */
+  const dit_bf16* k_scale;
+  const float* rope;                /* device [rope_rows][64][2] or NULL (no rotation) */
+  int rope_rows;                    /* output row m uses rope row m % rope_rows */
 } dit_gemm_args;
 
 /* bf16 x bf16 -> fp32 accumulate on tcgen05 (128 x 256 tiles, TMA-fed, TMEM
@@ -263,14 +275,16 @@ size_t dit_video_block_workspace(const dit_block_cfg* cfg, int n_ctx);
  *   o = attention(rope(rms(q)), rope(rms(k)), v); a = gelu_tanh(mlp)
  *   out = x + gate * ([o | a] W2^T + b2)
  * x, out: device bf16 [B*S][D] (out may equal x); vec: device bf16 [B][D];
- * rope: device float [S][64][2] from dit_rope_table.  Six kernels. */
+ * rope: device float [S][64][2] from dit_rope_table.  Five kernels: the QK
+ * RMSNorm + RoPE runs inside the GEMM1 epilogue. */
 dit_status dit_single_block_fwd(const dit_block_cfg* cfg, const dit_single_weights* w,
                                 const dit_bf16* x, const dit_bf16* vec, const float* rope,
                                 dit_bf16* out, void* ws, size_t ws_bytes, void* stream);
 
 /* Same call that additionally records events[i] (cudaEvent_t, may not be NULL)
- * on the stream before kernel i and events[n_kernels] after the last one, so a
- * caller can time every kernel.  n_events must be >= 7. */
+ * on the stream before kernel i and events[5] after the last of its five
+ * kernels (adaLN, LN-modulate, GEMM1 with fused QK-norm+RoPE, attention,
+ * GEMM2), so a caller can time every kernel.  n_events must be >= 6. */
 dit_status dit_single_block_fwd_profiled(const dit_block_cfg* cfg, const dit_single_weights* w,
                                          const dit_bf16* x, const dit_bf16* vec, const float* rope,
                                          dit_bf16* out, void* ws, size_t ws_bytes,

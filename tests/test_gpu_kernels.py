@@ -162,6 +162,40 @@ def test_gemm_gelu_cols_split_output():
     assert torch.count_nonzero(cat[:, :D]) == 0  # columns left of the split untouched
 
 
+@pytest.mark.parametrize("norm,B", [(1, 1), (0, 2)])
+def test_gemm_fused_qk_norm_rope(norm, B):
+    """QKV|MLP GEMM with RMSNorm + RoPE fused into the epilogue for the q and k
+    columns (and GELU on the MLP columns, written through the split output)."""
+    import torch
+    ids = synth.flux_ids(44, 16, 16)  # 300 tokens: ragged last row tile
+    S = ids.shape[0]
+    H, Mh = 2, 512
+    D = H * 128
+    N, K = 3 * D + Mh, D
+    A, W, b = _gemm_inputs(B * S, N, K, seed=11)
+    qs = synth.normal_bf16(0, "qs", (128,), 0.1, 1.0)
+    ks = synth.normal_bf16(0, "ks", (128,), 0.1, 1.0)
+    rope = torch.empty((S, 64, 2), dtype=torch.float32, device="cuda")
+    dit.dit_rope_table(torch.from_numpy(ids).cuda(), (8, 28, 28), 10000.0, rope)
+    qkv = torch.empty((B * S, 3 * D), dtype=torch.bfloat16, device="cuda")
+    mlp = torch.empty((B * S, Mh), dtype=torch.bfloat16, device="cuda")
+    dit.dit_gemm_epilogue(dev_bf16(A), dev_bf16(W), qkv, dit.DIT_EPI_BIAS_GELU_COLS, bias=dev_bf16(b), C2=mlp,
+                          split_col=3 * D, gelu_col_begin=3 * D, qk_cols=2 * D, qk_norm=norm,
+                          q_scale=dev_bf16(qs), k_scale=dev_bf16(ks), rope=rope, rope_rows=S)
+    h = O.linear(synth.bf16_bits_to_f64(A), synth.bf16_bits_to_f64(W), synth.bf16_bits_to_f64(b))
+    phi = np.tile(O.rope_angles(ids, (16, 56, 56)), (B, 1))
+    got = host_f64(qkv)
+    for which, sc in ((0, qs), (1, ks)):
+        x = h[:, which * D:(which + 1) * D]
+        if norm:
+            x = O.rms_norm_heads(x, synth.bf16_bits_to_f64(sc), H)
+        else:
+            x = x * np.tile(synth.bf16_bits_to_f64(sc), H)
+        parity(got[:, which * D:(which + 1) * D], O.apply_rope(x, phi, H), f"fused {'qk'[which]}")
+    parity(got[:, 2 * D:], h[:, 2 * D:3 * D], "v columns")
+    parity(host_f64(mlp), O.gelu_tanh(h[:, 3 * D:]), "gelu columns")
+
+
 @pytest.mark.parametrize("M,rows_per_batch,N,K,inplace", [(300, 150, 384, 1920, False), (256, 256, 3072, 512, True)])
 def test_gemm_gated_residual(M, rows_per_batch, N, K, inplace):
     import torch
