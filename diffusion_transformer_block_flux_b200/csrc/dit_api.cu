@@ -75,6 +75,14 @@ dit_status device_setup(int* num_sms) {
                                             cudaFuncAttributeMaxDynamicSharedMemorySize, dit::gemm::SMEM_BYTES));
         DIT_CUDA_CHECK(cudaFuncSetAttribute(dit::attn::attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                             dit::attn::SMEM_BYTES));
+        DIT_CUDA_CHECK(cudaFuncSetAttribute(dit::gemm::pair::gemm_pair_kernel<DIT_EPI_NONE>,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize, dit::gemm::pair::SMEM_BYTES));
+        DIT_CUDA_CHECK(cudaFuncSetAttribute(dit::gemm::pair::gemm_pair_kernel<DIT_EPI_BIAS>,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize, dit::gemm::pair::SMEM_BYTES));
+        DIT_CUDA_CHECK(cudaFuncSetAttribute(dit::gemm::pair::gemm_pair_kernel<DIT_EPI_BIAS_GELU_COLS>,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize, dit::gemm::pair::SMEM_BYTES));
+        DIT_CUDA_CHECK(cudaFuncSetAttribute(dit::gemm::pair::gemm_pair_kernel<DIT_EPI_BIAS_GATED_RESIDUAL>,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize, dit::gemm::pair::SMEM_BYTES));
         for (int nb = 1; nb <= 8; nb *= 2) {
           void* f = nb == 1   ? (void*)dit::vec_linear_kernel<1>
                     : nb == 2 ? (void*)dit::vec_linear_kernel<2>
@@ -420,9 +428,13 @@ dit_status dit_gemm_epilogue(const dit_gemm_args* a, void* stream) {
   int sms = 0;
   dit_status s = device_setup(&sms);
   if (s != DIT_OK) return s;
+  // SM-pair kernel (256 x 256 tiles over two CTAs) once there are at least
+  // two 128-row blocks; the one-CTA kernel (128 x 256 tiles) otherwise.
+  const bool use_pair = a->M > dit::gemm::BM && sms >= 2;
   CUtensorMap tA, tB;
   if ((s = make_map_2d(&tA, a->A, a->M, a->K, a->lda, dit::gemm::BM)) != DIT_OK) return s;
-  if ((s = make_map_2d(&tB, a->W, a->N, a->K, a->ldw, dit::gemm::BN)) != DIT_OK) return s;
+  if ((s = make_map_2d(&tB, a->W, a->N, a->K, a->ldw, use_pair ? dit::gemm::pair::BN_CTA : dit::gemm::BN)) != DIT_OK)
+    return s;
   dit::gemm::Epi ep;
   ep.C = reinterpret_cast<bf16*>(a->C);
   ep.ldc = a->ldc;
@@ -443,9 +455,34 @@ dit_status dit_gemm_epilogue(const dit_gemm_args* a, void* stream) {
   ep.k_scale = reinterpret_cast<const bf16*>(a->k_scale);
   ep.rope = reinterpret_cast<const float2*>(a->rope);
   ep.rope_rows = a->rope_rows > 0 ? a->rope_rows : a->M;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (use_pair) {
+    namespace P = dit::gemm::pair;
+    const int tiles = ((a->M + P::BM - 1) / P::BM) * ((a->N + P::BN - 1) / P::BN);
+    const int clusters = tiles < sms / 2 ? tiles : sms / 2;
+    const int grid = 2 * clusters;
+    switch (a->epi) {
+      case DIT_EPI_NONE:
+        P::gemm_pair_kernel<DIT_EPI_NONE><<<grid, P::NUM_THREADS, P::SMEM_BYTES, st>>>(tA, tB, a->M, a->N, a->K, ep,
+                                                                                     g_wait_limit_ns);
+        break;
+      case DIT_EPI_BIAS:
+        P::gemm_pair_kernel<DIT_EPI_BIAS><<<grid, P::NUM_THREADS, P::SMEM_BYTES, st>>>(tA, tB, a->M, a->N, a->K, ep,
+                                                                                     g_wait_limit_ns);
+        break;
+      case DIT_EPI_BIAS_GELU_COLS:
+        P::gemm_pair_kernel<DIT_EPI_BIAS_GELU_COLS><<<grid, P::NUM_THREADS, P::SMEM_BYTES, st>>>(
+            tA, tB, a->M, a->N, a->K, ep, g_wait_limit_ns);
+        break;
+      default:
+        P::gemm_pair_kernel<DIT_EPI_BIAS_GATED_RESIDUAL><<<grid, P::NUM_THREADS, P::SMEM_BYTES, st>>>(
+            tA, tB, a->M, a->N, a->K, ep, g_wait_limit_ns);
+        break;
+    }
+    return launch_status();
+  }
   const int tiles = ((a->M + dit::gemm::BM - 1) / dit::gemm::BM) * ((a->N + dit::gemm::BN - 1) / dit::gemm::BN);
   const int grid = tiles < sms ? tiles : sms;
-  cudaStream_t st = (cudaStream_t)stream;
   const int smem = dit::gemm::SMEM_BYTES;
   const int nt = dit::gemm::NUM_THREADS;
   switch (a->epi) {

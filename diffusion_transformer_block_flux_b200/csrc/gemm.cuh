@@ -369,5 +369,212 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == 1) tmem_dealloc(tmem_base, TMEM_COLS);
 }
 
+// ---------------------------------------------------------------------------
+// Two-CTA variant: a cluster of two CTAs on an SM pair computes a 256 x 256
+// tile.  CTA r loads rows [128r, 128r+128) of the A tile and rows
+// [128r, 128r+128) of the B tile (half of N) into its own shared memory; the
+// leader (r = 0) issues tcgen05.mma.cta_group::2 (M=256, N=256, K=16), which
+// reads both halves of each operand and writes each CTA's 128 x 256 part of
+// the accumulator into that CTA's TMEM.  Per SM this halves the B-operand
+// traffic of the one-CTA tile, and with 32 KB stages six fit in shared memory.
+// No TMA multicast: each CTA fetches its own halves.
+//   - full[s] (leader): one arrival (the leader's expect_tx for both CTAs'
+//     bytes) plus the transaction bytes of both CTAs' loads;
+//   - empty[s] (both): committed by the leader's MMA thread to both CTAs;
+//   - tfull[a] (both): committed to both CTAs after the last K block;
+//   - tempty[a] (leader): 8 arrivals, 4 epilogue warps in each CTA.
+// ---------------------------------------------------------------------------
+namespace pair {
+
+constexpr int BM = 256;      // rows per cluster tile
+constexpr int BM_CTA = 128;  // rows per CTA
+constexpr int BN = 256;
+constexpr int BN_CTA = 128;  // B rows loaded per CTA
+constexpr int BK = 64;
+constexpr int STAGES = 6;
+constexpr int A_BYTES = BM_CTA * BK * 2;
+constexpr int B_BYTES = BN_CTA * BK * 2;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int NUM_THREADS = 192;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 256 + 1024;
+constexpr uint32_t IDESC = idesc_bf16(BM, BN, 0, 0);
+
+template <int EPI>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
+    gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M, int N,
+                     int K, Epi ep, uint64_t wait_limit) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * A_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;  // [2]
+  uint64_t* tempty = tfull + 2;      // [2]
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 8);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync_all();  // barrier inits and TMEM allocation visible to both CTAs
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int num_m = (M + BM - 1) / BM;
+  const int num_n = (N + BN - 1) / BN;
+  const int num_tiles = num_m * num_n;
+  const int num_kb = (K + BK - 1) / BK;
+  const int cluster_id = blockIdx.x >> 1;
+  const int n_clusters = gridDim.x >> 1;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer (both CTAs) ----------------
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued_mask = 0, issued_parity = 0;
+      bool ok = true;
+      for (int tile = cluster_id; tile < num_tiles && ok; tile += n_clusters) {
+        const int tm = tile % num_m, tn = tile / num_m;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, wait_limit, abort_flag, SITE_GEMM2_PRODUCER)) {
+            ok = false;
+            break;
+          }
+          if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * STAGE_BYTES);
+          const uint32_t leader_full = mapa_shared(smem_u32(&full[stage]), 0);
+          tma_load_2d_pair(sA + stage * A_BYTES, &tmA, leader_full, kb * BK, tm * BM + (int)rank * BM_CTA);
+          tma_load_2d_pair(sB + stage * B_BYTES, &tmB, leader_full, kb * BK, tn * BN + (int)rank * BN_CTA);
+          issued_mask |= 1u << stage;
+          issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (!ok && rank == 0) {
+        for (int s = 0; s < STAGES; ++s)
+          if (issued_mask & (1u << s))
+            (void)mbar_wait(&full[s], (issued_parity >> s) & 1u, wait_limit, nullptr, SITE_GEMM2_DRAIN);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) {
+      // ---------------- MMA issuer (leader CTA) ----------------
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      bool issued_any = false;
+      for (int tile = cluster_id; tile < num_tiles && ok; tile += n_clusters) {
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1, wait_limit, abort_flag, SITE_GEMM2_MMA)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(&full[stage], phase, wait_limit, abort_flag, SITE_GEMM2_MMA)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + stage * A_BYTES);
+          const uint32_t b0 = smem_u32(sB + stage * B_BYTES);
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            umma_ss_pair(d_tmem, sdesc_sw128(a0 + k * 32, 16, 1024), sdesc_sw128(b0 + k * 32, 16, 1024), IDESC,
+                         (kb | k) != 0 ? 1u : 0u);
+          }
+          issued_any = true;
+          umma_commit_pair(&empty[stage], 0x3);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        umma_commit_pair(&tfull[acc], 0x3);
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1;
+        }
+      }
+      if (!ok && issued_any) {
+        umma_commit(drain);
+        (void)mbar_wait(drain, 0, wait_limit, nullptr, SITE_GEMM2_DRAIN);
+      }
+    }
+  } else {
+    // ---------------- epilogue warps 2..5 (both CTAs) ----------------
+    const int quad = warp & 3;
+    const int row_in_tile = (int)rank * BM_CTA + quad * 32 + lane;
+    const uint32_t leader_tempty0 = mapa_shared(smem_u32(&tempty[0]), 0);
+    const uint32_t leader_tempty1 = mapa_shared(smem_u32(&tempty[1]), 0);
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = cluster_id; tile < num_tiles; tile += n_clusters) {
+      const int tm = tile % num_m, tn = tile / num_m;
+      bool ok = mbar_wait(&tfull[acc], acc_phase, wait_limit, abort_flag, SITE_GEMM2_EPILOGUE);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      const int m = tm * BM + row_in_tile;
+      const uint32_t t_row = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * BN);
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        const int n0 = tn * BN + c * 32;
+        if (n0 >= N) break;  // warp-uniform
+        if (EPI != DIT_EPI_BIAS_GATED_RESIDUAL && n0 < ep.qk_cols) {
+          epilogue_qk_head(t_row + (uint32_t)(c * 32), m, n0, ep, m < M);
+          c += 3;
+          continue;
+        }
+        uint32_t r[32];
+        tmem_ld32(t_row + (uint32_t)(c * 32), r);
+        if (m < M) epilogue_chunk<EPI>(r, m, n0, ep);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(acc ? leader_tempty1 : leader_tempty0);
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1;
+      }
+    }
+  }
+
+  tc_fence_before();
+  cluster_sync_all();  // no CTA leaves while its peer may still touch its memory
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc_pair(tmem_base, TMEM_COLS);
+}
+
+}  // namespace pair
 }  // namespace gemm
 }  // namespace dit
