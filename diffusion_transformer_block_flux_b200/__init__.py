@@ -34,8 +34,8 @@ DIT_VEC_SILU_IN, DIT_VEC_OUT_BF16 = 1, 2
 
 
 class DitError(RuntimeError):
-    def __init__(self, fn: str, code: int):
-        super().__init__(f"{fn} returned {STATUS.get(code, code)}")
+    def __init__(self, fn: str, code: int, detail: str = ""):
+        super().__init__(f"{fn} returned {STATUS.get(code, code)}" + (f" ({detail})" if detail else ""))
         self.code = code
 
 
@@ -106,6 +106,7 @@ class dit_loop_io(ctypes.Structure):
 _SIGS = {
     "dit_status_string": (ctypes.c_char_p, [i32]),
     "dit_version": (i32, []),
+    "dit_last_cuda_error": (ctypes.c_char_p, []),
     "dit_get_device_error": (i32, [c_void_p, ctypes.POINTER(ctypes.c_uint32)]),
     "dit_clear_device_error": (i32, [c_void_p]),
     "dit_set_wait_limit_ns": (i32, [ctypes.c_uint64]),
@@ -177,7 +178,8 @@ def header_functions() -> list[str]:
 
 def _check(name: str, code: int):
     if code != 0:
-        raise DitError(name, code)
+        detail = lib().dit_last_cuda_error().decode() if code == DIT_ERR_CUDA else ""
+        raise DitError(name, code, detail)
 
 
 def _call(name: str, *args):
@@ -208,6 +210,10 @@ def dit_status_string(code: int) -> str:
 
 def dit_version() -> int:
     return lib().dit_version()
+
+
+def dit_last_cuda_error() -> str:
+    return lib().dit_last_cuda_error().decode()
 
 
 def dit_get_device_error(stream=None) -> tuple[int, int]:

@@ -246,44 +246,42 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           for (int i = 0; i < 32; ++i)
             if (c * 32 + i >= valid) r[c][i] = __float_as_uint(-INFINITY);
       }
+      // row max: four independent chains of 3-input max
       float mx[4];
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        float a0 = __uint_as_float(r[c][0]), a1 = __uint_as_float(r[c][1]);
+        float a = fmaxf(__uint_as_float(r[c][0]), __uint_as_float(r[c][1]));
 #pragma unroll
-        for (int i = 2; i < 32; i += 2) {
-          a0 = fmaxf(a0, __uint_as_float(r[c][i]));
-          a1 = fmaxf(a1, __uint_as_float(r[c][i + 1]));
-        }
-        mx[c] = fmaxf(a0, a1);
+        for (int i = 2; i < 32; i += 2) a = max3f(a, __uint_as_float(r[c][i]), __uint_as_float(r[c][i + 1]));
+        mx[c] = a;
       }
       const float m_tile = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2;
       const bool need = m_tile > m_run + 8.0f;  // always true on the first tile
       const float m_new = need ? m_tile : m_run;
       const float alpha = need ? ex2_fast(m_run - m_new) : 1.0f;  // 0 on the first tile
-      const float neg = -m_new;
-      float sum[4] = {0.f, 0.f, 0.f, 0.f};
+      const uint64_t sl2x2 = f2_pack(sl2, sl2);
+      const uint64_t negx2 = f2_pack(-m_new, -m_new);
+      uint64_t sum2[2] = {0ull, 0ull};  // packed (even, odd) partial sums, two chains
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float x0 = fmaf(__uint_as_float(r[c][2 * i]), sl2, neg);
-          const float x1 = fmaf(__uint_as_float(r[c][2 * i + 1]), sl2, neg);
-          float p0, p1;
+          // x = s * scale * log2(e) - m for the pair (2i, 2i+1): one packed FMA
+          const uint64_t x = f2_fma((uint64_t)r[c][2 * i] | ((uint64_t)r[c][2 * i + 1] << 32), sl2x2, negx2);
+          uint64_t pp;
           if ((i & 3) == 3) {  // a quarter of the exponentials on the FMA pipe
-            p0 = exp2_poly(x0);
-            p1 = exp2_poly(x1);
+            pp = exp2_poly2(f2_lo(x), f2_hi(x));
           } else {
-            p0 = ex2_fast(x0);
-            p1 = ex2_fast(x1);
+            pp = f2_pack(ex2_fast(f2_lo(x)), ex2_fast(f2_hi(x)));
           }
-          sum[i & 3] += p0 + p1;
-          pk[i] = pack_bf16x2(p0, p1);
+          sum2[i & 1] = f2_add(sum2[i & 1], pp);
+          pk[i] = pack_bf16x2(f2_lo(pp), f2_hi(pp));
         }
         tmem_st16(tS + (uint32_t)(c * 16), pk);
       }
-      l_run = l_run * alpha + ((sum[0] + sum[1]) + (sum[2] + sum[3]));
+      const uint64_t st2 = f2_add(sum2[0], sum2[1]);
+      l_run = l_run * alpha + (f2_lo(st2) + f2_hi(st2));
       // Rescale O_t when any row of this warp raised its max (O_t is stable:
       // the commit we waited on covers the previous PV into O_t).
       if (j > 0 && __any_sync(0xffffffffu, need)) {

@@ -412,6 +412,47 @@ __device__ __forceinline__ float exp2_poly(float x) {
   return __int_as_float(__float_as_int(p) + ((__float_as_int(t) - 0x4B400000) << 23));
 }
 
+// Packed fp32 pairs (sm_100): one instruction updates two lanes of a 64-bit
+// register pair.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  return (uint64_t)__float_as_uint(lo) | ((uint64_t)__float_as_uint(hi) << 32);
+}
+__device__ __forceinline__ float f2_lo(uint64_t v) { return __uint_as_float((uint32_t)v); }
+__device__ __forceinline__ float f2_hi(uint64_t v) { return __uint_as_float((uint32_t)(v >> 32)); }
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// exp2_poly on a pair: the same Cody-Waite split and cubic, with packed fp32
+// arithmetic; 2^n is added to the exponent field as t_bits << 23 (the magic
+// constant 1.5 * 2^23 contributes nothing modulo 2^32 after the shift).
+__device__ __forceinline__ uint64_t exp2_poly2(float x0, float x1) {
+  const uint64_t x = f2_pack(fmaxf(x0, -126.0f), fmaxf(x1, -126.0f));
+  const uint64_t magic = f2_pack(12582912.0f, 12582912.0f);
+  const uint64_t t = f2_add(x, magic);
+  const uint64_t n = f2_add(t, f2_pack(-12582912.0f, -12582912.0f));
+  const uint64_t f = f2_add(x, n ^ 0x8000000080000000ull);  // x - n
+  uint64_t p = f2_fma(f2_pack(0.0551716648042202f, 0.0551716648042202f), f,
+                      f2_pack(0.2426111251115799f, 0.2426111251115799f));
+  p = f2_fma(p, f, f2_pack(0.6932609677314758f, 0.6932609677314758f));
+  p = f2_fma(p, f, f2_pack(0.9999280571937561f, 0.9999280571937561f));
+  const uint32_t lo = (uint32_t)p + ((uint32_t)t << 23);
+  const uint32_t hi = (uint32_t)(p >> 32) + ((uint32_t)(t >> 32) << 23);
+  return (uint64_t)lo | ((uint64_t)hi << 32);
+}
+
 __device__ __forceinline__ float ex2_fast(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));

@@ -38,15 +38,23 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 EncodeTiledFn g_encode = nullptr;
 
-#define DIT_CUDA_CHECK(expr)                 \
-  do {                                       \
-    cudaError_t e_ = (expr);                 \
-    if (e_ != cudaSuccess) return DIT_ERR_CUDA; \
+// Last CUDA error seen by a library call on this host thread.
+thread_local cudaError_t t_last_cuda_error = cudaSuccess;
+
+inline dit_status cuda_fail(cudaError_t e) {
+  t_last_cuda_error = e;
+  return DIT_ERR_CUDA;
+}
+
+#define DIT_CUDA_CHECK(expr)                      \
+  do {                                            \
+    cudaError_t e_ = (expr);                      \
+    if (e_ != cudaSuccess) return cuda_fail(e_);  \
   } while (0)
 
 dit_status launch_status() {
   cudaError_t e = cudaGetLastError();
-  return e == cudaSuccess ? DIT_OK : DIT_ERR_CUDA;
+  return e == cudaSuccess ? DIT_OK : cuda_fail(e);
 }
 
 // Per-device setup: SM count, capability check, kernel attributes, driver
@@ -174,6 +182,10 @@ const char* dit_status_string(dit_status s) {
 }
 
 int dit_version(void) { return 100; }
+
+const char* dit_last_cuda_error(void) {
+  return t_last_cuda_error == cudaSuccess ? "no error" : cudaGetErrorString(t_last_cuda_error);
+}
 
 dit_status dit_get_device_error(void* stream, uint32_t* code) {
   if (code == nullptr) return DIT_ERR_INVALID_ARG;

@@ -67,6 +67,10 @@ const char* dit_status_string(dit_status s);
 /* Library version as major*10000 + minor*100 + patch. */
 int dit_version(void);
 
+/* Text of the last CUDA runtime error that made a call on this host thread
+ * return DIT_ERR_CUDA ("no error" if none).  Static storage; do not free. */
+const char* dit_last_cuda_error(void);
+
 /* ------------------------------------------------------------------------
  * Device error word and wait limit
  * ------------------------------------------------------------------------ */
