@@ -254,7 +254,19 @@ def test_attention(B, Sq, Skv, H, qmul):
     lg = lse.cpu().double().numpy()
     for b in range(B):
         qs, ks, vs = qf[b * Sq:(b + 1) * Sq], kf[b * Skv:(b + 1) * Skv], vf[b * Skv:(b + 1) * Skv]
-        parity(got[b], O.attention(qs, ks, vs, H), f"attention b={b}")
+        ref = O.attention(qs, ks, vs, H)
+        # Derived max-abs bound for a bf16 attention output: the largest
+        # element carries its own bf16 rounding (<= 2^-9 relative) plus the
+        # bf16 rounding of P that the tensor-core PV product needs (<= 2^-9
+        # relative per term), so allow 2^-7 * max|ref| on top of 3e-2 * RMS
+        # (averaging over many keys makes RMS small next to the largest
+        # element).  rel L2 keeps 1e-2 and must also stay within 2x the error
+        # of the exact result merely rounded to bf16 (+1e-3).
+        rms = np.sqrt(np.mean(ref ** 2))
+        parity(got[b], ref, f"attention b={b}", max_abs_frac=3e-2 + 2.0 ** -7 * np.abs(ref).max() / rms)
+        ref_b = synth.bf16_bits_to_f64(synth.f32_to_bf16_bits(ref.astype(np.float32)))
+        floor = np.linalg.norm(ref_b - ref) / np.linalg.norm(ref)
+        assert np.linalg.norm(got[b] - ref) / np.linalg.norm(ref) <= 2 * floor + 1e-3
         ref_lse = O.attention_lse(qs, ks, H)
         assert np.abs(lg[b] - ref_lse).max() < 1e-3 * max(1.0, np.abs(ref_lse).max())
     assert_no_device_error()
