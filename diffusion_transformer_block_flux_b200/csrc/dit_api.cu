@@ -135,11 +135,12 @@ dit_status make_map_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t
 }
 
 // 3-D bf16 tensor map over [batch][rows][cols] with row stride ld elements and
-// batch stride rows*ld; box = 128 rows x 64 columns x 1.
-dit_status make_map_3d(CUtensorMap* m, const void* base, uint64_t batch, uint64_t rows, uint64_t cols, int64_t ld) {
+// batch stride rows*ld; box = box_rows rows x 64 columns x 1.
+dit_status make_map_3d(CUtensorMap* m, const void* base, uint64_t batch, uint64_t rows, uint64_t cols, int64_t ld,
+                       uint32_t box_rows) {
   cuuint64_t dims[3] = {cols, rows, batch};
   cuuint64_t strides[2] = {(cuuint64_t)ld * 2, (cuuint64_t)ld * 2 * rows};
-  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t box[3] = {64, box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -383,9 +384,9 @@ dit_status dit_attention(const dit_bf16* q, const dit_bf16* k, const dit_bf16* v
   dit_status s = device_setup(nullptr);
   if (s != DIT_OK) return s;
   CUtensorMap tq, tk, tv;
-  if ((s = make_map_3d(&tq, q, B, Sq, D, ldq)) != DIT_OK) return s;
-  if ((s = make_map_3d(&tk, k, B, Skv, D, ldk)) != DIT_OK) return s;
-  if ((s = make_map_3d(&tv, v, B, Skv, D, ldv)) != DIT_OK) return s;
+  if ((s = make_map_3d(&tq, q, B, Sq, D, ldq, dit::attn::BQ)) != DIT_OK) return s;
+  if ((s = make_map_3d(&tk, k, B, Skv, D, ldk, dit::attn::BKV)) != DIT_OK) return s;
+  if ((s = make_map_3d(&tv, v, B, Skv, D, ldv, dit::attn::BKV)) != DIT_OK) return s;
   dit::attn::Params p;
   p.o = reinterpret_cast<bf16*>(o);
   p.ldo = ldo;
