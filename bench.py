@@ -274,7 +274,8 @@ def run_ours(args, rank, world, local_rank):
         roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
                 "frac": round(achieved / pk["hbm_gbs"], 4)}
     roof["kernel"] = dom
-    roof["traffic"] = TRAFFIC.get(dom)
+    roof["traffic"] = traffic_for(dom)
+    roof["traffic_unit"] = "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)"
     roof["peak_source"] = pk["source"] + " burst (MEASURED_PEAKS.json)" if pk["source"] == "measured" else "fallback"
     kernels = {}
     for k in KERNELS:
@@ -303,7 +304,29 @@ def run_ours(args, rank, world, local_rank):
     return res
 
 
-TRAFFIC: dict = {}
+# DRAM bytes (read + write) per launch from one ncu capture of each kernel
+# (profiles/*.ncu.md), with a hash of the kernel's sources at capture time.
+# A kernel whose sources changed since reports traffic null.
+NCU_TRAFFIC = {
+    "gemm_qkv_mlp_gelu_qknorm_rope": (336599808, ("gemm.cuh", "common.cuh"), "5894ad8931c28dfb"),
+    "gemm_out_gated_residual": (586020608, ("gemm.cuh", "common.cuh"), "5894ad8931c28dfb"),
+    "attention": (93017088, ("attention.cuh", "common.cuh"), "52e99483a88ee23f"),
+    "modulate_norm": (28450048, ("elementwise.cuh", "common.cuh"), "3bd8b97de326804d"),
+    "adaln_modulation": (56725504, ("elementwise.cuh", "common.cuh"), "3bd8b97de326804d"),
+}
+
+
+def traffic_for(kernel):
+    import hashlib
+    ent = NCU_TRAFFIC.get(kernel)
+    if ent is None:
+        return None
+    nbytes, files, digest = ent
+    m = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "diffusion_transformer_block_flux_b200", "csrc", f), "rb") as fh:
+            m.update(fh.read())
+    return nbytes if m.hexdigest()[:16] == digest else None
 
 
 # ----------------------------------------------------------------------------
@@ -651,10 +674,6 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local_rank))
     try:
-        traffic_file = os.path.join(ROOT, "profiles", "traffic.json")
-        if os.path.exists(traffic_file):
-            with open(traffic_file) as f:
-                TRAFFIC.update(json.load(f).get("per_launch_bytes", {}))
         res = run_ours(args, rank, world, local_rank)
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
             res["cpu_baseline"] = cpu_baseline()
