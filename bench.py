@@ -158,6 +158,21 @@ def make_block(torch, dev, seed):
     return w, x, vec
 
 
+def max_over_ranks(value, world, device="cpu"):
+    """Largest value over all ranks (the job's time is its slowest rank)."""
+    if world <= 1:
+        return float(value)
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(flops_per_step, steps, world, elapsed_ms):
+    """Whole-job throughput: every rank runs `steps` independent replica steps."""
+    return world * flops_per_step * steps / (elapsed_ms * 1e-3) / 1e12
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import diffusion_transformer_block_flux_b200 as dit
@@ -215,10 +230,7 @@ def run_ours(args, rank, world, local_rank):
     elapsed_ms = t_start.elapsed_time(t_end)
     per_kernel = {k: statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(K))
                   for j, k in enumerate(KERNELS)}
-    if world > 1:
-        t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(elapsed_ms, world, dev)
     st, code = dit.dit_get_device_error()
     if st != 0:
         raise RuntimeError(f"device error word {code:#x} in the timed region")
@@ -250,17 +262,13 @@ def run_ours(args, rank, world, local_rank):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
 
     flops = block_flops()
     total_flops = sum(flops.values())
     ms_per_step = elapsed_ms / K
-    value = world * total_flops * K / (elapsed_ms * 1e-3) / 1e12
-    e2e_value = world * total_flops * Ke / (e2e_ms * 1e-3) / 1e12
+    value = whole_job_tflops(total_flops, K, world, elapsed_ms)
+    e2e_value = whole_job_tflops(total_flops, Ke, world, e2e_ms)
 
     pk = peaks()
     dom = max(per_kernel, key=per_kernel.get)

@@ -262,7 +262,7 @@ dit_status dit_vec_linear(const dit_bf16* x, int64_t ldx, const dit_bf16* W, int
   const bf16* bb = reinterpret_cast<const bf16*>(bias);
   if (B == 1 && (K % 256) == 0 && K <= 4096) {
     int rgrid = (N + 3) / 4;
-    if (rgrid > sms * 3) rgrid = sms * 3;  // three 128-thread CTAs fit per SM at ~160 registers
+    if (rgrid > sms * 2) rgrid = sms * 2;  // two 128-thread CTAs per SM (registers: input + two weight rows)
 #define DIT_VR_CASE(KC_)                                                                                   \
   case KC_:                                                                                                \
     dit::vec_linear_reg_kernel<KC_><<<rgrid, 128, 0, st>>>(xb, Wb, ldw, bb, out, N, K, flags);             \
@@ -340,6 +340,27 @@ dit_status dit_modulate_norm(const dit_bf16* x, int64_t ldx, const float* shift,
     // persistent row stream: D/8 threads per CTA, modulation held in registers
     int sms = 0;
     if ((s = device_setup(&sms)) != DIT_OK) return s;
+    // wide variant: E elements per thread with D/E threads a multiple of 32 (<= 256)
+    const int E = ((D % 1024) == 0 && D / 32 <= 256) ? 32 : ((D % 512) == 0 && D / 16 <= 256) ? 16 : 0;
+    if (E != 0) {
+      const int threads = D / E;
+      int per_sm = 0;
+      if (E == 32)
+        DIT_CUDA_CHECK(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, dit::modulate_norm_wide_kernel<32>,
+                                                                     threads, 0));
+      else
+        DIT_CUDA_CHECK(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, dit::modulate_norm_wide_kernel<16>,
+                                                                     threads, 0));
+      int64_t grid = (int64_t)sms * (per_sm > 0 ? per_sm : 1);  // every CTA resident: a persistent row stream
+      if (grid > rows) grid = rows;
+      if (E == 32)
+        dit::modulate_norm_wide_kernel<32><<<(unsigned)grid, threads, 0, st>>>(xb, ldx, shift, scale, mod_stride,
+                                                                              yb, ldy, rows, S, D, eps);
+      else
+        dit::modulate_norm_wide_kernel<16><<<(unsigned)grid, threads, 0, st>>>(xb, ldx, shift, scale, mod_stride,
+                                                                              yb, ldy, rows, S, D, eps);
+      return launch_status();
+    }
     const int threads = ((D / 8 + 31) / 32) * 32;
     const int per_sm = 2048 / threads;
     int64_t grid = (int64_t)sms * (per_sm > 0 ? per_sm : 1);

@@ -105,6 +105,134 @@ __global__ void __launch_bounds__(1024) modulate_norm_stream_kernel(const bf16* 
 }
 
 // ---------------------------------------------------------------------------
+// LayerNorm + modulate, persistent row stream with E elements per thread
+// (E = 16 or 32; the CTA has D/E threads, a multiple of 32).  Thread t owns
+// the 16-byte chunks t, t + T, t + 2T, ... of every row (T = threads), keeps
+// (1 + scale) and shift for them in registers across rows, and prefetches the
+// next row's chunks before reducing the current one.  Statistics take one
+// reduction per row: each thread forms the exact mean and centred second
+// moment of its own E values, and the (mean, M2) pairs are merged across the
+// CTA with the parallel-variance update (Chan, Golub and LeVeque):
+//   M2 = M2a + M2b + (mean_b - mean_a)^2 * na nb / (na + nb).
+// Output math runs on packed fp32 pairs.
+// ---------------------------------------------------------------------------
+template <int E>
+__global__ void __launch_bounds__(256) modulate_norm_wide_kernel(const bf16* __restrict__ x, int64_t ldx,
+                                                                 const float* __restrict__ shift,
+                                                                 const float* __restrict__ scale,
+                                                                 int64_t mod_stride, bf16* __restrict__ y,
+                                                                 int64_t ldy, int64_t rows, int S, int D,
+                                                                 float eps) {
+  constexpr int NC = E / 8;  // 16-byte chunks per thread
+  __shared__ float2 red[2][8];  // per warp (mean, M2); two buffers alternate by row
+  const int T = blockDim.x;
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31, nw = T >> 5;
+  int64_t r = blockIdx.x;
+  uint4 cur[NC], nxt[NC];
+#pragma unroll
+  for (int c = 0; c < NC; ++c)
+    cur[c] = (r < rows) ? __ldcs(reinterpret_cast<const uint4*>(x + r * ldx) + c * T + threadIdx.x)
+                        : make_uint4(0, 0, 0, 0);
+  int cur_b = -1;
+  uint64_t sc1[E / 2], sh[E / 2];  // packed pairs of (1 + scale) and shift
+  int par = 0;
+  for (; r < rows; r += gridDim.x) {
+    const int64_t rn = r + gridDim.x;
+#pragma unroll
+    for (int c = 0; c < NC; ++c)
+      nxt[c] = (rn < rows) ? __ldcs(reinterpret_cast<const uint4*>(x + rn * ldx) + c * T + threadIdx.x)
+                           : make_uint4(0, 0, 0, 0);
+    const int b = (int)(r / S);
+    if (b != cur_b) {
+      cur_b = b;
+#pragma unroll
+      for (int c = 0; c < NC; ++c) {
+        const int col = (c * T + threadIdx.x) * 8;
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          float4 a = make_float4(0.f, 0.f, 0.f, 0.f), sc = a;
+          if (shift != nullptr) {
+            a = __ldg(reinterpret_cast<const float4*>(shift + b * mod_stride + col) + q);
+            sc = __ldg(reinterpret_cast<const float4*>(scale + b * mod_stride + col) + q);
+          }
+          sh[c * 4 + q * 2] = f2_pack(a.x, a.y);
+          sh[c * 4 + q * 2 + 1] = f2_pack(a.z, a.w);
+          sc1[c * 4 + q * 2] = f2_pack(1.f + sc.x, 1.f + sc.y);
+          sc1[c * 4 + q * 2 + 1] = f2_pack(1.f + sc.z, 1.f + sc.w);
+        }
+      }
+    }
+    // packed (lo, hi) pairs of this thread's E values
+    uint64_t v[E / 2];
+#pragma unroll
+    for (int c = 0; c < NC; ++c) {
+      const uint32_t u[4] = {cur[c].x, cur[c].y, cur[c].z, cur[c].w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) v[c * 4 + q] = f2_pack(bf16_lo(u[q]), bf16_hi(u[q]));
+    }
+    // thread-local exact mean and M2
+    uint64_t s2 = v[0];
+#pragma unroll
+    for (int i = 1; i < E / 2; ++i) s2 = f2_add(s2, v[i]);
+    float mean = (f2_lo(s2) + f2_hi(s2)) * (1.0f / E);
+    const uint64_t negm = f2_pack(-mean, -mean);
+    uint64_t q2 = 0ull;
+#pragma unroll
+    for (int i = 0; i < E / 2; ++i) {
+      const uint64_t d = f2_add(v[i], negm);
+      q2 = f2_fma(d, d, q2);
+    }
+    float m2 = f2_lo(q2) + f2_hi(q2);
+    // merge across the warp: equal counts at every step
+    float n = (float)E;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const float mb = __shfl_xor_sync(0xffffffffu, mean, o);
+      const float qb = __shfl_xor_sync(0xffffffffu, m2, o);
+      const float dlt = mb - mean;
+      m2 = m2 + qb + dlt * dlt * (0.5f * n);
+      mean = 0.5f * (mean + mb);
+      n *= 2.0f;
+    }
+    if (l == 0) red[par][w] = make_float2(mean, m2);
+    __syncthreads();
+    // merge the warps (count 32E each), in order
+    float2 acc = red[par][0];
+    float na = n;
+    for (int k = 1; k < nw; ++k) {
+      const float2 bq = red[par][k];
+      const float dlt = bq.x - acc.x;
+      const float nt = na + n;
+      acc.y = acc.y + bq.y + dlt * dlt * (na * n / nt);
+      acc.x = acc.x + dlt * (n / nt);
+      na = nt;
+    }
+    par ^= 1;  // next row writes the other buffer; no thread still reads it
+    const float mu = acc.x;
+    const float rstd = rsqrtf(acc.y / (float)D + eps);
+    // y = (x - mu) * rstd * (1 + scale) + shift = x * a + (shift - mu * a), a = rstd (1 + scale)
+    const uint64_t rstd2 = f2_pack(rstd, rstd);
+    const uint64_t negmu2 = f2_pack(-mu, -mu);
+    bf16* yr = y + r * ldy;
+#pragma unroll
+    for (int c = 0; c < NC; ++c) {
+      uint32_t pk[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int i = c * 4 + q;
+        const uint64_t a = f2_fma(sc1[i], rstd2, 0ull);              // rstd (1 + scale)
+        const uint64_t bb = f2_fma(negmu2, a, sh[i]);                // shift - mu a
+        const uint64_t o = f2_fma(v[i], a, bb);
+        pk[q] = pack_bf16x2(f2_lo(o), f2_hi(o));
+      }
+      *(reinterpret_cast<uint4*>(yr) + c * T + threadIdx.x) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    }
+#pragma unroll
+    for (int c = 0; c < NC; ++c) cur[c] = nxt[c];
+  }
+}
+
+// ---------------------------------------------------------------------------
 // adaLN / vector x weight with the (mapped) input vector held in registers:
 // lane l of every warp owns input columns {8(l + 32j) .. +8}, j < KC, so each
 // weight row is read with KC 16-byte loads per lane and multiplied against
@@ -113,7 +241,7 @@ __global__ void __launch_bounds__(1024) modulate_norm_stream_kernel(const bf16* 
 // conditioning vector); other batch sizes use vec_linear_kernel.
 // ---------------------------------------------------------------------------
 template <int KC>
-__global__ void __launch_bounds__(128) vec_linear_reg_kernel(const bf16* __restrict__ x,
+__global__ void __launch_bounds__(128, 2) vec_linear_reg_kernel(const bf16* __restrict__ x,
                                                              const bf16* __restrict__ W, int64_t ldw,
                                                              const bf16* __restrict__ bias, void* out, int N, int K,
                                                              int flags) {
@@ -133,13 +261,25 @@ __global__ void __launch_bounds__(128) vec_linear_reg_kernel(const bf16* __restr
     }
   }
   const int nw = gridDim.x * 4;
-  for (int n = blockIdx.x * 4 + warp; n < N; n += nw) {
-    const bf16* wr = W + (int64_t)n * ldw;
+  int n = blockIdx.x * 4 + warp;
+  // the next row's weights are loaded while the current row is multiplied
+  uint4 wn[KC];
+#pragma unroll
+  for (int j = 0; j < KC; ++j) {
+    const int k0 = (lane + 32 * j) * 8;
+    wn[j] = (n < N && k0 < K) ? __ldcs(reinterpret_cast<const uint4*>(W + (int64_t)n * ldw + k0))
+                              : make_uint4(0, 0, 0, 0);
+  }
+  for (; n < N; n += nw) {
     uint4 wv[KC];
+#pragma unroll
+    for (int j = 0; j < KC; ++j) wv[j] = wn[j];
+    const int nn = n + nw;
 #pragma unroll
     for (int j = 0; j < KC; ++j) {
       const int k0 = (lane + 32 * j) * 8;
-      wv[j] = (k0 < K) ? __ldcs(reinterpret_cast<const uint4*>(wr + k0)) : make_uint4(0, 0, 0, 0);
+      wn[j] = (nn < N && k0 < K) ? __ldcs(reinterpret_cast<const uint4*>(W + (int64_t)nn * ldw + k0))
+                                 : make_uint4(0, 0, 0, 0);
     }
     float a0 = 0.f, a1 = 0.f;
 #pragma unroll
