@@ -563,14 +563,16 @@ def run_loop(args):
     txt = _rand(torch, g, dev, S_TXT, ls.txt_in, std=1.0)
     ids = torch.from_numpy(synth.flux_ids(S_TXT, GRID, GRID)).to(dev)
     out = torch.empty((ls.channels, 2 * GRID, 2 * GRID), dtype=torch.float32, device=dev)
-    io = dit.loop_io(S_TXT, GRID, GRID, ls.steps, lat, txt, ids, out)
+    fresh = dit.cached_schedule(ls.steps) if args.cache else None
+    io = dit.loop_io(S_TXT, GRID, GRID, ls.steps, lat, txt, ids, out, fresh=fresh, cache_order=1)
     ws = torch.empty(dit.dit_forward_workspace(model, io), dtype=torch.uint8, device=dev)
     t0 = time.time()
     graph = dit.Graph(model, io, ws)
     t_build = time.time() - t0
     stream = torch.cuda.current_stream()
     K = max(1, min(3, args.steps))
-    ms = _event_time(torch, lambda: graph.launch(stream.cuda_stream), K, 1, stream)
+    W = 3
+    ms = _event_time(torch, lambda: graph.launch(stream.cuda_stream), K, W, stream)
     st, code = dit.dit_get_device_error()
     if st != 0:
         raise RuntimeError(f"device error word {code:#x}")
@@ -578,11 +580,13 @@ def run_loop(args):
     dbl = 2.0 * S * D * (3 * D + D + 2 * M) + 4.0 * S * S * H * 128 + 2 * 2.0 * D * 6 * D
     emb = 2.0 * (S_TXT * ls.txt_in * D + (S - S_TXT) * F * D + ls.t_dim * D + D * D) + 2.0 * D * 2 * D \
         + 2.0 * (S - S_TXT) * D * F
-    flops = ls.steps * (ls.n_double * dbl + ls.n_single * single + emb)
+    n_fwd = sum(fresh) if fresh is not None else ls.steps
+    flops = n_fwd * (ls.n_double * dbl + ls.n_single * single + emb)
     n_nodes = graph.nodes()
     graph.destroy()
-    return _extra_line(ls.name + "_one_cuda_graph", ms, flops, K, 1,
-                       {"s_per_image": round(ms / 1e3, 3), "graph_nodes": n_nodes,
+    name = ls.name + ("_step_cache_%dfresh" % n_fwd if fresh is not None else "") + "_one_cuda_graph"
+    return _extra_line(name, ms, flops, K, W,
+                       {"s_per_image": round(ms / 1e3, 3), "graph_nodes": n_nodes, "model_forwards": n_fwd,
                         "graph_build_s": round(t_build, 2), "graph_launches_per_image": 1})
 
 
@@ -655,6 +659,8 @@ def main():
     ap.add_argument("--workload", choices=["single"] + sorted(EXTRA), default="single",
                     help="single = the headline Flux single-stream block (default)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cache", action="store_true",
+                    help="loop workload: model-level step cache (26 model forwards for 50 steps)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -96,7 +96,8 @@ class dit_model(ctypes.Structure):
 
 class dit_loop_io(ctypes.Structure):
     _fields_ = [("n_txt", i32), ("grid_h", i32), ("grid_w", i32), ("steps", i32),
-                ("latent_in", c_void_p), ("txt", c_void_p), ("ids", c_void_p), ("latent_out", c_void_p)]
+                ("latent_in", c_void_p), ("txt", c_void_p), ("ids", c_void_p), ("latent_out", c_void_p),
+                ("fresh", ctypes.POINTER(ctypes.c_uint8)), ("cache_order", i32)]
 
 
 # ----------------------------------------------------------------------------
@@ -370,9 +371,23 @@ class Model:
                            eps=eps, **kw)
 
 
-def loop_io(n_txt, grid_h, grid_w, steps, latent_in, txt, ids, latent_out) -> dit_loop_io:
-    return dit_loop_io(n_txt=n_txt, grid_h=grid_h, grid_w=grid_w, steps=steps, latent_in=_ptr(latent_in),
-                       txt=_ptr(txt), ids=_ptr(ids), latent_out=_ptr(latent_out))
+def loop_io(n_txt, grid_h, grid_w, steps, latent_in, txt, ids, latent_out, fresh=None,
+            cache_order=1) -> dit_loop_io:
+    """fresh: optional sequence of 0/1 per step (1 = run the model)."""
+    io = dit_loop_io(n_txt=n_txt, grid_h=grid_h, grid_w=grid_w, steps=steps, latent_in=_ptr(latent_in),
+                     txt=_ptr(txt), ids=_ptr(ids), latent_out=_ptr(latent_out), cache_order=cache_order)
+    if fresh is not None:
+        arr = (ctypes.c_uint8 * steps)(*[1 if f else 0 for f in fresh])
+        io._fresh_keep = arr
+        io.fresh = ctypes.cast(arr, ctypes.POINTER(ctypes.c_uint8))
+    return io
+
+
+def cached_schedule(steps: int) -> list:
+    """Fresh at the first two steps and then every other step: 26 model
+    forwards for 50 steps (the count the compile_graph page reports for its
+    step cache, §8)."""
+    return [1 if (i < 2 or i % 2 == 1) else 0 for i in range(steps)]
 
 
 def dit_forward_workspace(model: Model, io: dit_loop_io) -> int:

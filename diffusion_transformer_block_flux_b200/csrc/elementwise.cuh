@@ -612,12 +612,30 @@ __global__ void unpatchify_kernel(const float* __restrict__ state, int C, int Hg
 }
 
 // x += (t_{i+1} - t_i) v, state fp32; also refresh the bf16 copy fed to img_in.
+// vhist (optional): keep the model velocity of this step for the step cache.
 __global__ void euler_kernel(float* __restrict__ state, bf16* __restrict__ tok, const bf16* __restrict__ v,
-                             int64_t n, const float* __restrict__ tsched, int step) {
+                             int64_t n, const float* __restrict__ tsched, int step, float* __restrict__ vhist) {
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= n) return;
   const float dt = tsched[step + 1] - tsched[step];
-  const float s = fmaf(dt, __bfloat162float(v[i]), state[i]);
+  const float vi = __bfloat162float(v[i]);
+  if (vhist != nullptr) vhist[i] = vi;
+  const float s = fmaf(dt, vi, state[i]);
+  state[i] = s;
+  tok[i] = __float2bfloat16_rn(s);
+}
+
+// Cached step: v = ca * va + cb * vb from kept model velocities (vb may be
+// null), then the same Euler update.
+__global__ void euler_cached_kernel(float* __restrict__ state, bf16* __restrict__ tok, const float* __restrict__ va,
+                                    const float* __restrict__ vb, float ca, float cb, int64_t n,
+                                    const float* __restrict__ tsched, int step) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  const float dt = tsched[step + 1] - tsched[step];
+  float v = ca * va[i];
+  if (vb != nullptr) v = fmaf(cb, vb[i], v);
+  const float s = fmaf(dt, v, state[i]);
   state[i] = s;
   tok[i] = __float2bfloat16_rn(s);
 }

@@ -365,6 +365,15 @@ typedef struct {
   const dit_bf16* txt;               /* device bf16 [n_txt][txt_dim] */
   const int32_t* ids;                /* device int32 [n_txt + grid_h grid_w][3] */
   float* latent_out;                 /* device float [channels][2 grid_h][2 grid_w] */
+  /* Model-level step cache ([CG] §7: the loop decides per step whether to
+   * run the forward; skipped steps predict the velocity from history by a
+   * finite difference along t).  fresh: host array [steps], 1 = run the
+   * model at step i, 0 = predict; NULL = every step fresh.  Step 0 must be
+   * fresh.  cache_order 0 reuses the last model velocity; 1 extrapolates
+   * linearly from the last two, v(t) = v_a + (t - t_a)(v_a - v_b)/(t_a - t_b)
+   * (the last one alone until two exist).  Read at graph creation. */
+  const uint8_t* fresh;
+  int cache_order;
 } dit_loop_io;
 
 typedef struct dit_graph dit_graph;

@@ -354,16 +354,32 @@ def flux_velocity(img_tok, txt_raw, t, ids, model, n_heads, axes_dim=(16, 56, 56
 
 
 def euler_sample(latent, txt_raw, ids, model, n_heads, steps, axes_dim=(16, 56, 56),
-                 theta=10000.0, eps=1e-6):
+                 theta=10000.0, eps=1e-6, fresh=None, cache_order=1):
     """Flow-match Euler over the linear schedule t_i = 1 - i/steps:
     x <- x + (t_{i+1} - t_i) v(x, t_i).  Returns the final latent [C, H, W]
-    (reading s9: no resolution shift, no guidance)."""
+    (reading s9: no resolution shift, no guidance).
+
+    Model-level step cache ([CG] §7): fresh[i] = 1 runs the model at step i;
+    fresh[i] = 0 predicts the velocity from the model velocities of earlier
+    fresh steps.  cache_order 0 reuses the last one; 1 extrapolates linearly
+    in t from the last two (a finite-difference estimate of dv/dt), using the
+    last one alone while only one exists."""
     C, Hh, Ww = latent.shape
     x = patchify(np.asarray(latent, dtype=np.float64))
+    hist = []  # (t, v) of fresh steps, newest last
     for i in range(steps):
         t0 = 1.0 - i / steps
         t1 = 1.0 - (i + 1) / steps
-        v = flux_velocity(x, txt_raw, t0, ids, model, n_heads, axes_dim, theta, eps)
+        if fresh is None or fresh[i]:
+            v = flux_velocity(x, txt_raw, t0, ids, model, n_heads, axes_dim, theta, eps)
+            hist.append((t0, v))
+        else:
+            ta, va = hist[-1]
+            if cache_order == 1 and len(hist) >= 2:
+                tb, vb = hist[-2]
+                v = va + (t0 - ta) * (va - vb) / (ta - tb)
+            else:
+                v = va
         x = x + (t1 - t0) * v
     return unpatchify(x, C, Hh // 2, Ww // 2)
 

@@ -23,7 +23,7 @@ def cuda():
     torch.cuda.synchronize()
 
 
-def setup_loop(ls, seed=0):
+def setup_loop(ls, seed=0, fresh=None, cache_order=1):
     import torch
     b = ls.block
     mw = synth.model_weights(ls, seed=seed)
@@ -34,7 +34,8 @@ def setup_loop(ls, seed=0):
     txt = dev_bf16(inp["txt"])
     ids = torch.from_numpy(inp["ids"]).cuda()
     lat_out = torch.empty(inp["latent"].shape, dtype=torch.float32, device="cuda")
-    io = dit.loop_io(b.n_txt, b.grid_h, b.grid_w, ls.steps, lat_in, txt, ids, lat_out)
+    io = dit.loop_io(b.n_txt, b.grid_h, b.grid_w, ls.steps, lat_in, txt, ids, lat_out, fresh=fresh,
+                     cache_order=cache_order)
     ws = torch.empty(dit.dit_forward_workspace(model, io), dtype=torch.uint8, device="cuda")
     keep = (mdev, lat_in, txt, ids)
     return mw, inp, model, io, ws, lat_out, keep
@@ -98,3 +99,43 @@ def test_full_depth_velocity_at_tiny_dims():
     # (6e-2 RMS).
     parity(got - f["latent"], ref - f["latent"], "full-depth velocity", rel_l2=2e-2, max_abs_frac=6e-2)
     parity(got, ref, "full-depth latent")
+
+
+CACHED = synth.loop_shape(synth.BlockShape("loop_small", 16, 4, 6, 256, 2, 512), 2, 2, 6, channels=16, txt_in=64)
+
+
+def test_step_cache_all_fresh_is_bitwise_the_plain_loop():
+    import torch
+    _, _, model, io, ws, lat_out, keep = setup_loop(CACHED)
+    dit.dit_forward_eager(model, io, ws)
+    torch.cuda.synchronize()
+    plain = lat_out.clone()
+    _, _, model2, io2, ws2, lat_out2, keep2 = setup_loop(CACHED, fresh=[1] * CACHED.steps)
+    dit.dit_forward_eager(model2, io2, ws2)
+    torch.cuda.synchronize()
+    assert torch.equal(plain, lat_out2)
+
+
+@pytest.mark.parametrize("order", [0, 1])
+def test_step_cache_matches_oracle_and_graph_equals_eager(order):
+    """Model-level step cache: steps 2, 4, 5 predicted from kept velocities."""
+    import torch
+    fresh = [1, 1, 0, 1, 0, 0]
+    mw, inp, model, io, ws, lat_out, keep = setup_loop(CACHED, fresh=fresh, cache_order=order)
+    dit.dit_forward_eager(model, io, ws)
+    torch.cuda.synchronize()
+    eager = lat_out.clone()
+    g = dit.Graph(model, io, ws)
+    lat_out.zero_()
+    g.launch()
+    torch.cuda.synchronize()
+    assert torch.equal(lat_out, eager)
+    g.destroy()
+    f = synth.to_f64(inp)
+    ref = O.euler_sample(f["latent"], f["txt"], f["ids"], synth.to_f64(mw), CACHED.block.H, CACHED.steps,
+                         fresh=fresh, cache_order=order)
+    got = eager.cpu().double().numpy()
+    parity(got, ref, f"cached loop (order {order})")
+    parity(got - f["latent"], ref - f["latent"], f"cached loop displacement (order {order})")
+    st, code = dit.dit_get_device_error()
+    assert st == 0, f"device error word {code:#x}"

@@ -368,6 +368,43 @@ def test_euler_constant_velocity_closed_form():
     np.testing.assert_allclose(out, O.unpatchify(tok, 2, 2, 3), rtol=1e-12, atol=1e-12)
 
 
+def test_step_cache_all_fresh_and_constant_velocity():
+    ls = _tiny_loop()
+    m = synth.to_f64(synth.model_weights(ls))
+    inp = synth.to_f64(synth.loop_inputs(ls))
+    base = O.euler_sample(inp["latent"], inp["txt"], inp["ids"], m, ls.block.H, ls.steps)
+    all_fresh = O.euler_sample(inp["latent"], inp["txt"], inp["ids"], m, ls.block.H, ls.steps,
+                               fresh=[1] * ls.steps)
+    np.testing.assert_array_equal(base, all_fresh)
+    # a constant velocity is reproduced exactly by both cache rules
+    m["W_out"] = np.zeros_like(m["W_out"])
+    c = rng(33).standard_normal(m["b_out"].shape)
+    m["b_out"] = c
+    for order in (0, 1):
+        out = O.euler_sample(inp["latent"], inp["txt"], inp["ids"], m, ls.block.H, ls.steps,
+                             fresh=[1, 1, 0], cache_order=order)
+        tok = O.patchify(inp["latent"]) - c
+        np.testing.assert_allclose(out, O.unpatchify(tok, 2, 2, 3), rtol=1e-12, atol=1e-12)
+
+
+def test_step_cache_first_order_bookkeeping():
+    """3 steps over t = 1, 2/3, 1/3 with steps 0, 1 fresh and step 2 cached:
+    the prediction is v2 = v1 + (t2 - t1)(v1 - v0)/(t1 - t0) = 2 v1 - v0."""
+    ls = _tiny_loop()
+    m = synth.to_f64(synth.model_weights(ls))
+    inp = synth.to_f64(synth.loop_inputs(ls))
+    x0 = O.patchify(inp["latent"])
+    v0 = O.flux_velocity(x0, inp["txt"], 1.0, inp["ids"], m, ls.block.H)
+    x1 = x0 - v0 / 3
+    v1 = O.flux_velocity(x1, inp["txt"], 2.0 / 3.0, inp["ids"], m, ls.block.H)
+    x2 = x1 - v1 / 3
+    x3 = x2 - (2 * v1 - v0) / 3
+    got = O.euler_sample(inp["latent"], inp["txt"], inp["ids"], m, ls.block.H, 3, fresh=[1, 1, 0], cache_order=1)
+    np.testing.assert_allclose(got, O.unpatchify(x3, 2, 2, 3), rtol=1e-10, atol=1e-12)
+    got0 = O.euler_sample(inp["latent"], inp["txt"], inp["ids"], m, ls.block.H, 3, fresh=[1, 1, 0], cache_order=0)
+    np.testing.assert_allclose(got0, O.unpatchify(x2 - v1 / 3, 2, 2, 3), rtol=1e-10, atol=1e-12)
+
+
 def test_golden_flux_shapes():
     with open(os.path.join(GOLDEN, "flux_shapes.json")) as f:
         g = json.load(f)
