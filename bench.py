@@ -216,10 +216,15 @@ def run_ours(args, rank, world, local_rank):
         torch.distributed.barrier()
     torch.cuda.synchronize()
     wall0 = time.time()
+    # headline: K plain block forwards
     t_start.record(stream)
     for i in range(K):
-        step(evs[i])
+        step()
     t_end.record(stream)
+    torch.cuda.synchronize()
+    # breakdown: K more forwards with an event before and after every kernel
+    for i in range(K):
+        step(evs[i])
     torch.cuda.synchronize()
     wall1 = time.time()
     if world > 1:
@@ -271,12 +276,16 @@ def run_ours(args, rank, world, local_rank):
     e2e_value = whole_job_tflops(total_flops, Ke, world, e2e_ms)
 
     pk = peaks()
+    # a block timed inside a long run of blocks: the power-capped (sustained) tensor peak applies
+    # when the clock record shows the power cap, the burst peak otherwise
+    capped = "sw_power_cap" in clocks.get("reasons", [])
+    bf16_peak = pk["bf16_tflops_sustained"] if capped else pk["bf16_tflops"]
     dom = max(per_kernel, key=per_kernel.get)
     nbytes = block_bytes()
     if KERNEL_BOUND[dom] == "tensor":
         achieved = flops[dom] / (per_kernel[dom] * 1e-3) / 1e12
-        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": round(achieved / pk["bf16_tflops"], 4)}
+        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": bf16_peak, "unit": "TFLOP/s",
+                "frac": round(achieved / bf16_peak, 4)}
     else:
         achieved = nbytes[dom] / (per_kernel[dom] * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
@@ -284,18 +293,22 @@ def run_ours(args, rank, world, local_rank):
     roof["kernel"] = dom
     roof["traffic"] = traffic_for(dom)
     roof["traffic_unit"] = "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)"
-    roof["peak_source"] = pk["source"] + " burst (MEASURED_PEAKS.json)" if pk["source"] == "measured" else "fallback"
+    if pk["source"] == "measured":
+        roof["peak_source"] = ("measured sustained, power-capped" if capped and roof["bound"] == "tensor"
+                               else "measured burst") + " (MEASURED_PEAKS.json)"
+    else:
+        roof["peak_source"] = "fallback"
     kernels = {}
     for k in KERNELS:
         ent = {"ms": round(per_kernel[k], 4), "share": round(per_kernel[k] / sum(per_kernel.values()), 4)}
         if KERNEL_BOUND[k] == "tensor":
             a = flops[k] / (per_kernel[k] * 1e-3) / 1e12
-            ent.update({"tflops": round(a, 1), "frac_of_bf16_peak": round(a / pk["bf16_tflops"], 4)})
+            ent.update({"tflops": round(a, 1), "frac_of_bf16_peak": round(a / bf16_peak, 4)})
         else:
             a = nbytes[k] / (per_kernel[k] * 1e-3) / 1e9
             ent.update({"gbs": round(a, 1), "frac_of_hbm_peak": round(a / pk["hbm_gbs"], 4)})
         kernels[k] = ent
-    block_frac = (total_flops / (ms_per_step * 1e-3) / 1e12) / pk["bf16_tflops"]
+    block_frac = (total_flops / (ms_per_step * 1e-3) / 1e12) / bf16_peak
     res = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
@@ -316,11 +329,11 @@ def run_ours(args, rank, world, local_rank):
 # (profiles/*.ncu.md), with a hash of the kernel's sources at capture time.
 # A kernel whose sources changed since reports traffic null.
 NCU_TRAFFIC = {
-    "gemm_qkv_mlp_gelu_qknorm_rope": (336599808, ("gemm.cuh", "common.cuh"), "5894ad8931c28dfb"),
-    "gemm_out_gated_residual": (586020608, ("gemm.cuh", "common.cuh"), "5894ad8931c28dfb"),
-    "attention": (93017088, ("attention.cuh", "common.cuh"), "52e99483a88ee23f"),
-    "modulate_norm": (28450048, ("elementwise.cuh", "common.cuh"), "3bd8b97de326804d"),
-    "adaln_modulation": (56725504, ("elementwise.cuh", "common.cuh"), "3bd8b97de326804d"),
+    "gemm_qkv_mlp_gelu_qknorm_rope": (336449280, ("gemm.cuh", "common.cuh"), "fc2cefdbf8d48145"),
+    "gemm_out_gated_residual": (586581760, ("gemm.cuh", "common.cuh"), "fc2cefdbf8d48145"),
+    "attention": (95049984, ("attention.cuh", "common.cuh"), "703ad1ee60f1efde"),
+    "modulate_norm": (28416512, ("elementwise.cuh", "common.cuh"), "b21596d7241c9891"),
+    "adaln_modulation": (56665344, ("elementwise.cuh", "common.cuh"), "b21596d7241c9891"),
 }
 
 
@@ -631,19 +644,38 @@ def run_kernels(args):
         i = nxt()
         dit.dit_adaln_modulation(vec, Ws[i], None, mout)
 
-    K = max(20, args.steps)
+    def copy():  # yardstick, not part of the path: a library copy of the LayerNorm's bytes
+        i = nxt()
+        ys[i].copy_(xs[i])
+
+    # R launches per CUDA graph, so that host-side call overhead is not timed
+    R = 4 * NB
+    K = max(5, args.steps // R)
     stream = torch.cuda.current_stream()
     res = {}
     for name, fn, nbytes in (("modulate_norm", ln, 2 * S * D * 2),
                              ("qk_norm_rope", qk, 4 * S * D * 2 + S * 64 * 8),
-                             ("adaln_modulation", ada, 3 * D * D * 2)):
-        ms = _event_time(torch, fn, K, args.warmup, stream)
+                             ("adaln_modulation", ada, 3 * D * D * 2),
+                             ("torch_copy_same_bytes_as_modulate_norm", copy, 2 * S * D * 2)):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            for _ in range(R):
+                fn()
+        ms = _event_time(torch, graph.replay, K, 3, torch.cuda.current_stream()) / R
+        del graph
         gbs = nbytes / (ms * 1e-3) / 1e9
         res[name] = {"us": round(ms * 1e3, 2), "gbs": round(gbs, 1), "frac_of_hbm_peak": round(gbs / pk["hbm_gbs"], 4),
                      "bytes": nbytes}
+    st, code = dit.dit_get_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error word {code:#x}")
     return {"metric": "HBM-bound kernels alone, Flux single-block shape (S=4608, D=3072)", "unit": "GB/s",
-            "n_gpus": 1, "steps": K, "warmup": args.warmup, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": "hbm_kernels_S4608_D3072", "l2": "4 rotating buffer sets, > L2 in total"},
+            "n_gpus": 1, "steps": K * R, "warmup": args.warmup, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "hbm_kernels_S4608_D3072", "l2": "4 rotating buffer sets, > L2 in total",
+                       "timing": f"{R} launches per CUDA graph, {K} replays, CUDA events"},
             "hbm_peak_gbs": pk["hbm_gbs"], "kernels": res}
 
 

@@ -22,6 +22,7 @@ namespace {
 constexpr int kMaxDevices = 64;
 constexpr int kVecSmemMax = 200 * 1024;  // staged input vectors of dit_vec_linear (B * K fp32)
 constexpr int kRowSmemMax = 200 * 1024;  // bulk-staged row rings (8 warps x 2 rows) + vectors
+constexpr int kVecPipeSmemMax = 144 * 1024;  // adaLN: 4 warps x 4 weight rows of K <= 4096 bf16 + K fp32
 uint64_t g_wait_limit_ns = 2000000000ull;
 
 struct DeviceInfo {
@@ -102,6 +103,17 @@ dit_status device_setup(int* num_sms) {
                      : nb == 4 ? (void*)dit::vec_linear_bulk_kernel<4>
                                : (void*)dit::vec_linear_bulk_kernel<8>;
           DIT_CUDA_CHECK(cudaFuncSetAttribute(fb, cudaFuncAttributeMaxDynamicSharedMemorySize, kRowSmemMax));
+        }
+        const void* vec_pipe[8] = {
+            (const void*)dit::vec_linear_pipe_kernel<1>, (const void*)dit::vec_linear_pipe_kernel<2>,
+            (const void*)dit::vec_linear_pipe_kernel<3>, (const void*)dit::vec_linear_pipe_kernel<4>,
+            (const void*)dit::vec_linear_pipe_kernel<6>, (const void*)dit::vec_linear_pipe_kernel<8>,
+            (const void*)dit::vec_linear_pipe_kernel<12>, (const void*)dit::vec_linear_pipe_kernel<16>};
+        // the grid assumes every CTA the occupancy calculator allows is resident: ask for the
+        // largest shared-memory carveout so the launch does not pick a smaller one
+        for (const void* f : vec_pipe) {
+          DIT_CUDA_CHECK(cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, kVecPipeSmemMax));
+          DIT_CUDA_CHECK(cudaFuncSetAttribute(f, cudaFuncAttributePreferredSharedMemoryCarveout, 100));
         }
         if (g_encode == nullptr) {
           void* fn = nullptr;
@@ -261,11 +273,14 @@ dit_status dit_vec_linear(const dit_bf16* x, int64_t ldx, const dit_bf16* W, int
   const bf16* Wb = reinterpret_cast<const bf16*>(W);
   const bf16* bb = reinterpret_cast<const bf16*>(bias);
   if (B == 1 && (K % 256) == 0 && K <= 4096) {
-    int rgrid = (N + 3) / 4;
-    if (rgrid > sms * 2) rgrid = sms * 2;  // two 128-thread CTAs per SM (registers: input + two weight rows)
+    // weight rows in flight through warp-private shared-memory rings (cp.async, 3 rows ahead)
+    const size_t ring_smem = (size_t)dit::kVecPipeWarps * dit::kVecPipeSlots * K * 2 + (size_t)K * 4;
+    int rgrid = (N + dit::kVecPipeWarps - 1) / dit::kVecPipeWarps;
+    const int per_sm = (int)(220 * 1024 / (ring_smem + 1024));
+    if (rgrid > sms * per_sm) rgrid = sms * per_sm;
 #define DIT_VR_CASE(KC_)                                                                                   \
   case KC_:                                                                                                \
-    dit::vec_linear_reg_kernel<KC_><<<rgrid, 128, 0, st>>>(xb, Wb, ldw, bb, out, N, K, flags);             \
+    dit::vec_linear_pipe_kernel<KC_><<<rgrid, 128, ring_smem, st>>>(xb, Wb, ldw, bb, out, N, K, flags);     \
     return launch_status();
     switch (K / 256) {
       DIT_VR_CASE(1)
@@ -337,30 +352,35 @@ dit_status dit_modulate_norm(const dit_bf16* x, int64_t ldx, const float* shift,
   bf16* yb = reinterpret_cast<bf16*>(y);
   cudaStream_t st = (cudaStream_t)stream;
   {
-    // persistent row stream: D/8 threads per CTA, modulation held in registers
     int sms = 0;
     if ((s = device_setup(&sms)) != DIT_OK) return s;
-    // wide variant: E elements per thread with D/E threads a multiple of 32 (<= 256)
-    const int E = ((D % 1024) == 0 && D / 32 <= 256) ? 32 : ((D % 512) == 0 && D / 16 <= 256) ? 16 : 0;
-    if (E != 0) {
-      const int threads = D / E;
-      int per_sm = 0;
-      if (E == 32)
-        DIT_CUDA_CHECK(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, dit::modulate_norm_wide_kernel<32>,
-                                                                     threads, 0));
+    // one CTA per row: NC 16-byte chunks per thread, D / (8 NC) threads a multiple of 32 in [32, 256]
+    int NC = 0;
+    for (int c : {3, 4, 2, 1}) {
+      const int t = D / (8 * c);
+      if (D % (8 * c) == 0 && t % 32 == 0 && t >= 32 && t <= 256) {
+        NC = c;
+        break;
+      }
+    }
+    if (NC != 0 && B <= 65535) {
+      const dim3 grid((unsigned)S, (unsigned)B);
+      const int threads = D / (8 * NC);
+      if (NC == 1)
+        dit::modulate_norm_row_kernel<1><<<grid, threads, 0, st>>>(xb, ldx, shift, scale, mod_stride, yb, ldy, S, D,
+                                                                    eps);
+      else if (NC == 2)
+        dit::modulate_norm_row_kernel<2><<<grid, threads, 0, st>>>(xb, ldx, shift, scale, mod_stride, yb, ldy, S, D,
+                                                                    eps);
+      else if (NC == 3)
+        dit::modulate_norm_row_kernel<3><<<grid, threads, 0, st>>>(xb, ldx, shift, scale, mod_stride, yb, ldy, S, D,
+                                                                    eps);
       else
-        DIT_CUDA_CHECK(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, dit::modulate_norm_wide_kernel<16>,
-                                                                     threads, 0));
-      int64_t grid = (int64_t)sms * (per_sm > 0 ? per_sm : 1);  // every CTA resident: a persistent row stream
-      if (grid > rows) grid = rows;
-      if (E == 32)
-        dit::modulate_norm_wide_kernel<32><<<(unsigned)grid, threads, 0, st>>>(xb, ldx, shift, scale, mod_stride,
-                                                                              yb, ldy, rows, S, D, eps);
-      else
-        dit::modulate_norm_wide_kernel<16><<<(unsigned)grid, threads, 0, st>>>(xb, ldx, shift, scale, mod_stride,
-                                                                              yb, ldy, rows, S, D, eps);
+        dit::modulate_norm_row_kernel<4><<<grid, threads, 0, st>>>(xb, ldx, shift, scale, mod_stride, yb, ldy, S, D,
+                                                                    eps);
       return launch_status();
     }
+    // otherwise (D not a multiple of 256 or 768): persistent row stream, D/8 threads per CTA
     const int threads = ((D / 8 + 31) / 32) * 32;
     const int per_sm = 2048 / threads;
     int64_t grid = (int64_t)sms * (per_sm > 0 ? per_sm : 1);

@@ -105,199 +105,197 @@ __global__ void __launch_bounds__(1024) modulate_norm_stream_kernel(const bf16* 
 }
 
 // ---------------------------------------------------------------------------
-// LayerNorm + modulate, persistent row stream with E elements per thread
-// (E = 16 or 32; the CTA has D/E threads, a multiple of 32).  Thread t owns
-// the 16-byte chunks t, t + T, t + 2T, ... of every row (T = threads), keeps
-// (1 + scale) and shift for them in registers across rows, and prefetches the
-// next row's chunks before reducing the current one.  Statistics take one
-// reduction per row: each thread forms the exact mean and centred second
-// moment of its own E values, and the (mean, M2) pairs are merged across the
-// CTA with the parallel-variance update (Chan, Golub and LeVeque):
-//   M2 = M2a + M2b + (mean_b - mean_a)^2 * na nb / (na + nb).
-// Output math runs on packed fp32 pairs.
+// LayerNorm + modulate, one CTA per row (grid = tokens x batch, not
+// persistent): every thread issues its NC 16-byte loads on entry, so the
+// hardware keeps as many rows in flight as CTAs are resident and starts the
+// next row as soon as one retires.  D / (8 NC) threads, 8 NC values each.
+// Statistics: exact per-thread mean and M2, Chan merge across the lanes,
+// then the closed form for equal-count warps.  The modulation is read at the
+// output (L1-resident: every row of a batch row uses the same vectors).
 // ---------------------------------------------------------------------------
-template <int E>
-__global__ void __launch_bounds__(256) modulate_norm_wide_kernel(const bf16* __restrict__ x, int64_t ldx,
-                                                                 const float* __restrict__ shift,
-                                                                 const float* __restrict__ scale,
-                                                                 int64_t mod_stride, bf16* __restrict__ y,
-                                                                 int64_t ldy, int64_t rows, int S, int D,
-                                                                 float eps) {
-  constexpr int NC = E / 8;  // 16-byte chunks per thread
-  __shared__ float2 red[2][8];  // per warp (mean, M2); two buffers alternate by row
+template <int NC>
+__global__ void __launch_bounds__(256) modulate_norm_row_kernel(const bf16* __restrict__ x, int64_t ldx,
+                                                                const float* __restrict__ shift,
+                                                                const float* __restrict__ scale,
+                                                                int64_t mod_stride, bf16* __restrict__ y,
+                                                                int64_t ldy, int S, int D, float eps) {
+  constexpr int E = 8 * NC;
+  __shared__ float2 red[8];
   const int T = blockDim.x;
   const int w = threadIdx.x >> 5, l = threadIdx.x & 31, nw = T >> 5;
-  int64_t r = blockIdx.x;
-  uint4 cur[NC], nxt[NC];
+  const int b = blockIdx.y;
+  const int64_t r = (int64_t)b * S + blockIdx.x;
+  const uint4* xr = reinterpret_cast<const uint4*>(x + r * ldx);
+  uint4 u4[NC];
 #pragma unroll
-  for (int c = 0; c < NC; ++c)
-    cur[c] = (r < rows) ? __ldcs(reinterpret_cast<const uint4*>(x + r * ldx) + c * T + threadIdx.x)
-                        : make_uint4(0, 0, 0, 0);
-  int cur_b = -1;
-  uint64_t sc1[E / 2], sh[E / 2];  // packed pairs of (1 + scale) and shift
-  int par = 0;
-  for (; r < rows; r += gridDim.x) {
-    const int64_t rn = r + gridDim.x;
+  for (int c = 0; c < NC; ++c) u4[c] = __ldcs(xr + c * T + threadIdx.x);
+  uint64_t v[E / 2];
 #pragma unroll
-    for (int c = 0; c < NC; ++c)
-      nxt[c] = (rn < rows) ? __ldcs(reinterpret_cast<const uint4*>(x + rn * ldx) + c * T + threadIdx.x)
-                           : make_uint4(0, 0, 0, 0);
-    const int b = (int)(r / S);
-    if (b != cur_b) {
-      cur_b = b;
+  for (int c = 0; c < NC; ++c) {
+    const uint32_t u[4] = {u4[c].x, u4[c].y, u4[c].z, u4[c].w};
 #pragma unroll
-      for (int c = 0; c < NC; ++c) {
-        const int col = (c * T + threadIdx.x) * 8;
+    for (int q = 0; q < 4; ++q) v[c * 4 + q] = f2_pack(bf16_lo(u[q]), bf16_hi(u[q]));
+  }
+  uint64_t s2 = v[0];
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          float4 a = make_float4(0.f, 0.f, 0.f, 0.f), sc = a;
-          if (shift != nullptr) {
-            a = __ldg(reinterpret_cast<const float4*>(shift + b * mod_stride + col) + q);
-            sc = __ldg(reinterpret_cast<const float4*>(scale + b * mod_stride + col) + q);
-          }
-          sh[c * 4 + q * 2] = f2_pack(a.x, a.y);
-          sh[c * 4 + q * 2 + 1] = f2_pack(a.z, a.w);
-          sc1[c * 4 + q * 2] = f2_pack(1.f + sc.x, 1.f + sc.y);
-          sc1[c * 4 + q * 2 + 1] = f2_pack(1.f + sc.z, 1.f + sc.w);
-        }
+  for (int i = 1; i < E / 2; ++i) s2 = f2_add(s2, v[i]);
+  float mean = (f2_lo(s2) + f2_hi(s2)) * (1.0f / E);
+  const uint64_t negm = f2_pack(-mean, -mean);
+  uint64_t q2 = 0ull;
+#pragma unroll
+  for (int i = 0; i < E / 2; ++i) {
+    const uint64_t d = f2_add(v[i], negm);
+    q2 = f2_fma(d, d, q2);
+  }
+  float m2 = f2_lo(q2) + f2_hi(q2);
+  float n = (float)E;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const float mb = __shfl_xor_sync(0xffffffffu, mean, o);
+    const float qb = __shfl_xor_sync(0xffffffffu, m2, o);
+    const float dlt = mb - mean;
+    m2 = m2 + qb + dlt * dlt * (0.5f * n);
+    mean = 0.5f * (mean + mb);
+    n *= 2.0f;
+  }
+  if (l == 0) red[w] = make_float2(mean, m2);
+  __syncthreads();
+  // equal-count warps: mean = average of the warp means, M2 = sum of the warp
+  // M2 + (values per warp) * sum of squared deviations of the warp means
+  float msum = 0.0f;
+  for (int k = 0; k < nw; ++k) msum += red[k].x;
+  const float mu = msum / (float)nw;
+  float m2sum = 0.0f, dev = 0.0f;
+  for (int k = 0; k < nw; ++k) {
+    const float2 bq = red[k];
+    const float dlt = bq.x - mu;
+    m2sum += bq.y;
+    dev = fmaf(dlt, dlt, dev);
+  }
+  const float rstd = rsqrtf(fmaf(n, dev, m2sum) / (float)D + eps);
+  // y = ((x - mu) rstd) (1 + scale) + shift
+  const uint64_t rstd2 = f2_pack(rstd, rstd);
+  const uint64_t nmr2 = f2_pack(-mu * rstd, -mu * rstd);
+  uint4* yr = reinterpret_cast<uint4*>(y + r * ldy);
+#pragma unroll
+  for (int c = 0; c < NC; ++c) {
+    const int col = (c * T + threadIdx.x) * 8;
+    uint64_t sc1[4], sh[4];
+    if (shift != nullptr) {
+      const float4* ps = reinterpret_cast<const float4*>(shift + b * mod_stride + col);
+      const float4* pc = reinterpret_cast<const float4*>(scale + b * mod_stride + col);
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        const float4 a = __ldg(ps + q), sc = __ldg(pc + q);
+        sh[q * 2] = f2_pack(a.x, a.y);
+        sh[q * 2 + 1] = f2_pack(a.z, a.w);
+        sc1[q * 2] = f2_pack(1.f + sc.x, 1.f + sc.y);
+        sc1[q * 2 + 1] = f2_pack(1.f + sc.z, 1.f + sc.w);
       }
-    }
-    // packed (lo, hi) pairs of this thread's E values
-    uint64_t v[E / 2];
-#pragma unroll
-    for (int c = 0; c < NC; ++c) {
-      const uint32_t u[4] = {cur[c].x, cur[c].y, cur[c].z, cur[c].w};
-#pragma unroll
-      for (int q = 0; q < 4; ++q) v[c * 4 + q] = f2_pack(bf16_lo(u[q]), bf16_hi(u[q]));
-    }
-    // thread-local exact mean and M2
-    uint64_t s2 = v[0];
-#pragma unroll
-    for (int i = 1; i < E / 2; ++i) s2 = f2_add(s2, v[i]);
-    float mean = (f2_lo(s2) + f2_hi(s2)) * (1.0f / E);
-    const uint64_t negm = f2_pack(-mean, -mean);
-    uint64_t q2 = 0ull;
-#pragma unroll
-    for (int i = 0; i < E / 2; ++i) {
-      const uint64_t d = f2_add(v[i], negm);
-      q2 = f2_fma(d, d, q2);
-    }
-    float m2 = f2_lo(q2) + f2_hi(q2);
-    // merge across the warp: equal counts at every step
-    float n = (float)E;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const float mb = __shfl_xor_sync(0xffffffffu, mean, o);
-      const float qb = __shfl_xor_sync(0xffffffffu, m2, o);
-      const float dlt = mb - mean;
-      m2 = m2 + qb + dlt * dlt * (0.5f * n);
-      mean = 0.5f * (mean + mb);
-      n *= 2.0f;
-    }
-    if (l == 0) red[par][w] = make_float2(mean, m2);
-    __syncthreads();
-    // merge the warps (count 32E each), in order
-    float2 acc = red[par][0];
-    float na = n;
-    for (int k = 1; k < nw; ++k) {
-      const float2 bq = red[par][k];
-      const float dlt = bq.x - acc.x;
-      const float nt = na + n;
-      acc.y = acc.y + bq.y + dlt * dlt * (na * n / nt);
-      acc.x = acc.x + dlt * (n / nt);
-      na = nt;
-    }
-    par ^= 1;  // next row writes the other buffer; no thread still reads it
-    const float mu = acc.x;
-    const float rstd = rsqrtf(acc.y / (float)D + eps);
-    // y = (x - mu) * rstd * (1 + scale) + shift = x * a + (shift - mu * a), a = rstd (1 + scale)
-    const uint64_t rstd2 = f2_pack(rstd, rstd);
-    const uint64_t negmu2 = f2_pack(-mu, -mu);
-    bf16* yr = y + r * ldy;
-#pragma unroll
-    for (int c = 0; c < NC; ++c) {
-      uint32_t pk[4];
+    } else {
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        const int i = c * 4 + q;
-        const uint64_t a = f2_fma(sc1[i], rstd2, 0ull);              // rstd (1 + scale)
-        const uint64_t bb = f2_fma(negmu2, a, sh[i]);                // shift - mu a
-        const uint64_t o = f2_fma(v[i], a, bb);
-        pk[q] = pack_bf16x2(f2_lo(o), f2_hi(o));
+        sh[q] = 0ull;
+        sc1[q] = f2_pack(1.f, 1.f);
       }
-      *(reinterpret_cast<uint4*>(yr) + c * T + threadIdx.x) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
     }
+    uint32_t pk[4];
 #pragma unroll
-    for (int c = 0; c < NC; ++c) cur[c] = nxt[c];
+    for (int q = 0; q < 4; ++q) {
+      const uint64_t t = f2_fma(v[c * 4 + q], rstd2, nmr2);
+      const uint64_t o = f2_fma(t, sc1[q], sh[q]);
+      pk[q] = pack_bf16x2(f2_lo(o), f2_hi(o));
+    }
+    yr[c * T + threadIdx.x] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
   }
 }
 
 // ---------------------------------------------------------------------------
-// adaLN / vector x weight with the (mapped) input vector held in registers:
-// lane l of every warp owns input columns {8(l + 32j) .. +8}, j < KC, so each
-// weight row is read with KC 16-byte loads per lane and multiplied against
-// registers; no shared-memory traffic per row.  One warp per output feature,
-// features dealt round-robin over the grid.  B == 1 only (the block's
-// conditioning vector); other batch sizes use vec_linear_kernel.
+// adaLN / vector x weight, batch 1, with the weight rows in flight through a
+// warp-private shared-memory ring of P row slots.  Lane l copies its KC
+// 16-byte chunks (columns 8(l + 32j) .. +8) of the warp's next rows into the
+// ring with cp.async, P - 1 rows ahead, and reads back exactly what it copied
+// (no barrier); the input vector is held in registers in the same column
+// order.  One warp per output feature, features dealt round-robin; 4 warps
+// per CTA.
 // ---------------------------------------------------------------------------
+constexpr int kVecPipeWarps = 4;
+constexpr int kVecPipeSlots = 4;
+
 template <int KC>
-__global__ void __launch_bounds__(128, 2) vec_linear_reg_kernel(const bf16* __restrict__ x,
-                                                             const bf16* __restrict__ W, int64_t ldw,
-                                                             const bf16* __restrict__ bias, void* out, int N, int K,
-                                                             int flags) {
+__global__ void __launch_bounds__(128) vec_linear_pipe_kernel(const bf16* __restrict__ x,
+                                                              const bf16* __restrict__ W, int64_t ldw,
+                                                              const bf16* __restrict__ bias, void* out, int N,
+                                                              int K, int flags) {
+  constexpr int P = kVecPipeSlots;
+  extern __shared__ __align__(16) uint4 wring[];  // [warps][P][K / 8], then the mapped input (K fp32)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row_chunks = K / 8;
+  uint4* ring = wring + (size_t)warp * P * row_chunks;
+  float* xs = reinterpret_cast<float*>(wring + (size_t)kVecPipeWarps * P * row_chunks);
+  const int64_t nw = (int64_t)gridDim.x * kVecPipeWarps;
+  const int64_t n0 = (int64_t)blockIdx.x * kVecPipeWarps + warp;
+#pragma unroll
+  for (int k = 0; k < P - 1; ++k) {
+    const int64_t nn = n0 + k * nw;
+    if (nn < N) {
+#pragma unroll
+      for (int j = 0; j < KC; ++j)
+        cp_async16(&ring[k * row_chunks + lane + 32 * j],
+                   reinterpret_cast<const uint4*>(W + nn * ldw) + lane + 32 * j);
+    }
+    cp_async_commit();
+  }
+  // the mapped input is computed once per CTA, then each lane keeps its columns in registers
+  for (int k = threadIdx.x; k < K; k += blockDim.x) {
+    float z = __bfloat162float(x[k]);
+    if (flags & DIT_VEC_SILU_IN) z = silu(z);
+    xs[k] = z;
+  }
+  __syncthreads();
   float xv[KC * 8];
 #pragma unroll
   for (int j = 0; j < KC; ++j) {
-    const int k0 = (lane + 32 * j) * 8;
+    const float4* p = reinterpret_cast<const float4*>(xs + (lane + 32 * j) * 8);
+    const float4 a = p[0], c = p[1];
+    xv[j * 8 + 0] = a.x; xv[j * 8 + 1] = a.y; xv[j * 8 + 2] = a.z; xv[j * 8 + 3] = a.w;
+    xv[j * 8 + 4] = c.x; xv[j * 8 + 5] = c.y; xv[j * 8 + 6] = c.z; xv[j * 8 + 7] = c.w;
+  }
+  int slot = 0;
+  for (int64_t n = n0; n < N; n += nw) {
+    {  // the slot consumed one row ago gets the row P - 1 ahead
+      const int64_t nn = n + (int64_t)(P - 1) * nw;
+      const int si = (slot == 0 ? P : slot) - 1;
+      if (nn < N) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      float z = 0.0f;
-      if (k0 + i < K) {
-        z = __bfloat162float(x[k0 + i]);
-        if (flags & DIT_VEC_SILU_IN) z = silu(z);
+        for (int j = 0; j < KC; ++j)
+          cp_async16(&ring[si * row_chunks + lane + 32 * j],
+                     reinterpret_cast<const uint4*>(W + nn * ldw) + lane + 32 * j);
       }
-      xv[j * 8 + i] = z;
+      cp_async_commit();
     }
-  }
-  const int nw = gridDim.x * 4;
-  int n = blockIdx.x * 4 + warp;
-  // the next row's weights are loaded while the current row is multiplied
-  uint4 wn[KC];
-#pragma unroll
-  for (int j = 0; j < KC; ++j) {
-    const int k0 = (lane + 32 * j) * 8;
-    wn[j] = (n < N && k0 < K) ? __ldcs(reinterpret_cast<const uint4*>(W + (int64_t)n * ldw + k0))
-                              : make_uint4(0, 0, 0, 0);
-  }
-  for (; n < N; n += nw) {
-    uint4 wv[KC];
-#pragma unroll
-    for (int j = 0; j < KC; ++j) wv[j] = wn[j];
-    const int nn = n + nw;
-#pragma unroll
-    for (int j = 0; j < KC; ++j) {
-      const int k0 = (lane + 32 * j) * 8;
-      wn[j] = (nn < N && k0 < K) ? __ldcs(reinterpret_cast<const uint4*>(W + (int64_t)nn * ldw + k0))
-                                 : make_uint4(0, 0, 0, 0);
-    }
+    // the bias load is issued before the wait so that its latency overlaps the copies
+    const float bv = bias ? __bfloat162float(bias[n]) : 0.0f;
+    cp_async_wait<P - 1>();
     float a0 = 0.f, a1 = 0.f;
 #pragma unroll
     for (int j = 0; j < KC; ++j) {
-      const uint4 u = wv[j];
+      const uint4 u = ring[slot * row_chunks + lane + 32 * j];
       a0 = fmaf(bf16_lo(u.x), xv[j * 8 + 0], a0); a1 = fmaf(bf16_hi(u.x), xv[j * 8 + 1], a1);
       a0 = fmaf(bf16_lo(u.y), xv[j * 8 + 2], a0); a1 = fmaf(bf16_hi(u.y), xv[j * 8 + 3], a1);
       a0 = fmaf(bf16_lo(u.z), xv[j * 8 + 4], a0); a1 = fmaf(bf16_hi(u.z), xv[j * 8 + 5], a1);
       a0 = fmaf(bf16_lo(u.w), xv[j * 8 + 6], a0); a1 = fmaf(bf16_hi(u.w), xv[j * 8 + 7], a1);
     }
-    const float a = warp_sum(a0 + a1) + (bias ? __bfloat162float(bias[n]) : 0.0f);
+    const float a = warp_sum(a0 + a1) + bv;
     if (lane == 0) {
       if (flags & DIT_VEC_OUT_BF16)
         reinterpret_cast<bf16*>(out)[n] = __float2bfloat16_rn(a);
       else
         reinterpret_cast<float*>(out)[n] = a;
     }
+    if (++slot == P) slot = 0;
   }
+  cp_async_wait<0>();
 }
 
 // ---------------------------------------------------------------------------

@@ -53,7 +53,8 @@ def test_rope_table(pairs, axes, ids_fn):
 
 # ---------------------------------------------------------------- adaLN
 
-@pytest.mark.parametrize("B,N,K", [(1, 1152, 384), (2, 9216, 3072), (3, 200, 64)])
+@pytest.mark.parametrize("B,N,K", [(1, 1152, 384), (2, 9216, 3072), (3, 200, 64), (1, 9216, 3072), (1, 18432, 3072),
+                                   (1, 1001, 4096), (1, 37, 256), (1, 5, 1536)])
 def test_adaln_modulation(B, N, K):
     import torch
     vec = synth.normal_bf16(1, "vec", (B, K))
@@ -78,7 +79,8 @@ def test_vec_linear_bf16_out_no_silu():
 
 # ---------------------------------------------------------------- LayerNorm + modulate
 
-@pytest.mark.parametrize("B,S,D", [(2, 100, 384), (1, 37, 3072), (1, 5, 1536), (1, 3, 8)])
+@pytest.mark.parametrize("B,S,D", [(2, 100, 384), (1, 37, 3072), (1, 5, 1536), (1, 3, 8), (1, 4608, 3072),
+                                   (2, 1301, 1536), (1, 333, 8192), (3, 257, 512), (1, 1000, 6144)])
 def test_modulate_norm(B, S, D):
     import torch
     x = synth.normal_bf16(1, "x", (B * S, D), 2.0, 0.5)
