@@ -134,6 +134,10 @@ _SIGS = {
                                             ctypes.POINTER(c_void_p), i32, c_void_p]),
     "dit_single_block_fwd_noalloc": (i32, [ctypes.POINTER(dit_block_cfg), ctypes.POINTER(dit_single_weights),
                                            c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]),
+    "dit_single_block_host_workspace": (size_t, [ctypes.POINTER(dit_block_cfg)]),
+    "dit_single_block_fwd_host": (i32, [ctypes.POINTER(dit_block_cfg), ctypes.POINTER(dit_single_weights), i32,
+                                        ctypes.POINTER(c_void_p), ctypes.POINTER(c_void_p), ctypes.POINTER(c_void_p),
+                                        c_void_p, c_void_p, size_t, c_void_p]),
     "dit_double_block_fwd": (i32, [ctypes.POINTER(dit_block_cfg), ctypes.POINTER(dit_double_weights),
                                    c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                    size_t, c_void_p]),
@@ -343,6 +347,23 @@ def dit_single_block_fwd_noalloc(cfg, w: dit_single_weights, x, vec, rope, out, 
     array inside the library (shared by all calls; overlapping calls race)."""
     _call("dit_single_block_fwd_noalloc", ctypes.byref(cfg), ctypes.byref(w), _ptr(x), _ptr(vec), _ptr(rope),
           _ptr(out), _stream(stream))
+
+
+def dit_single_block_host_workspace(cfg: dit_block_cfg) -> int:
+    return lib().dit_single_block_host_workspace(ctypes.byref(cfg))
+
+
+def dit_single_block_fwd_host(cfg, w: dit_single_weights, xs, vecs, outs, rope, ws, stream=None):
+    """len(xs) independent single-stream block forwards whose inputs and
+    outputs are host tensors (page-locked for overlap); copies in, compute
+    and copies out are pipelined inside the library.  The outputs are in
+    `outs` once the stream has completed."""
+    n = len(xs)
+    if len(vecs) != n or len(outs) != n:
+        raise ValueError("xs, vecs and outs must have the same length")
+    arr = lambda ts: (c_void_p * n)(*[t.data_ptr() for t in ts])
+    _call("dit_single_block_fwd_host", ctypes.byref(cfg), ctypes.byref(w), n, arr(xs), arr(vecs), arr(outs),
+          _ptr(rope), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream))
 
 
 def dit_double_block_fwd(cfg, w: dit_double_weights, img, txt, vec, rope, img_out, txt_out, ws, stream=None):

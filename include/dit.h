@@ -315,6 +315,31 @@ dit_status dit_single_block_fwd_noalloc(const dit_block_cfg* cfg, const dit_sing
                                         const dit_bf16* x, const dit_bf16* vec, const float* rope,
                                         dit_bf16* out, void* stream);
 
+/* Host-buffer pipeline of independent single-stream block forwards, e.g. a
+ * server's queue of requests.  (The pages have no counterpart to this call;
+ * the block itself is the one of dit_single_block_fwd, five kernels.)
+ *   Request i reads x_host[i] (bf16 [B*S][D]) and vec_host[i] (bf16 [B][D])
+ *   from host memory and writes out_host[i] (bf16 [B*S][D]) back to host
+ *   memory; out_host[i] may equal x_host[i].
+ *   Request i+1's host-to-device copy and request i-1's device-to-host copy
+ *   run on two streams internal to the library while request i computes on
+ *   `stream`.  The device staging is double-buffered inside the workspace and
+ *   ordered by events.  One cudaMemcpyAsync per copy.
+ *   Host buffers should be page-locked (cudaHostAlloc / cudaHostRegister) for
+ *   the copies to overlap the compute; pageable buffers give the same results.
+ *   The call returns once everything is enqueued.  `stream` waits for the
+ *   last copy, so the outputs are in host memory once `stream` completes.
+ *   The internal streams and events are created on a device's first call and
+ *   kept; enqueues from several host threads are serialised inside the call.
+ *   Calls that share a workspace must not overlap.  Not for stream capture.
+ * rope: device float [S][64][2].  ws: device, 256-byte aligned, at least
+ * dit_single_block_host_workspace(cfg) bytes.  n >= 1; every pointer non-NULL. */
+size_t dit_single_block_host_workspace(const dit_block_cfg* cfg);
+dit_status dit_single_block_fwd_host(const dit_block_cfg* cfg, const dit_single_weights* w, int n,
+                                     const dit_bf16* const* x_host, const dit_bf16* const* vec_host,
+                                     dit_bf16* const* out_host, const float* rope, void* ws,
+                                     size_t ws_bytes, void* stream);
+
 /* Flux double-stream block: per stream s in (txt, img) its own adaLN (6
  * chunks), LN-modulate, QKV, QK RMSNorm; RoPE + joint attention over the
  * sequence txt | img (rope rows in that order); then

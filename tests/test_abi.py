@@ -67,3 +67,18 @@ def test_block_call_rejects_small_workspace(L):
     w = dit.dit_single_weights(*([16] * 8))
     st = L.dit_single_block_fwd(ctypes.byref(cfg), ctypes.byref(w), 16, 16, 16, 16, 256, 10, None)
     assert st == dit.DIT_ERR_WORKSPACE
+
+
+def test_host_pipeline_validation(L):
+    cfg = dit.block_cfg(1, 256, 384, 3, 1536)
+    w = dit.dit_single_weights(*([16] * 8))
+    one = (ctypes.c_void_p * 1)(16)
+    nul = (ctypes.c_void_p * 1)(None)
+    need = dit.dit_single_block_host_workspace(cfg)
+    # block workspace + two staging slots of x, vec and out
+    assert need >= dit.dit_single_block_workspace(cfg) + 2 * (2 * 256 * 384 * 2 + 384 * 2)
+    f = L.dit_single_block_fwd_host
+    assert f(ctypes.byref(cfg), ctypes.byref(w), 0, one, one, one, 16, 256, need, None) == dit.DIT_ERR_INVALID_ARG
+    assert f(ctypes.byref(cfg), ctypes.byref(w), 1, one, nul, one, 16, 256, need, None) == dit.DIT_ERR_INVALID_ARG
+    assert f(ctypes.byref(cfg), ctypes.byref(w), 1, one, one, one, 16, 256, need - 1, None) == dit.DIT_ERR_WORKSPACE
+    assert f(ctypes.byref(cfg), ctypes.byref(w), 1, one, one, one, 16, 264, need, None) == dit.DIT_ERR_ALIGNMENT
