@@ -177,6 +177,26 @@ def attention_lse(q, k, n_heads, scale=None):
     return res
 
 
+def attention_merge(outs, lses):
+    """Combine attention results over disjoint key sets ([CG] §5: sequence-
+    parallel ring attention merges each hop's partial result by its
+    log-sum-exp).  With key set j giving o_j (softmax over that set alone)
+    and lse_j, the attention over the union is
+        lse = log sum_j exp(lse_j),  o = sum_j exp(lse_j - lse) o_j.
+    outs: list of [Sq, H*d]; lses: list of [H, Sq] (natural log).
+    Returns (o [Sq, H*d], lse [H, Sq])."""
+    n_heads = lses[0].shape[0]
+    L = np.stack(lses)                      # [n, H, Sq]
+    m = L.max(axis=0)
+    lse = m + np.log(np.exp(L - m).sum(axis=0))
+    Sq = outs[0].shape[0]
+    d = outs[0].shape[1] // n_heads
+    o = np.zeros((Sq, n_heads, d))
+    for oj, lj in zip(outs, lses):
+        o += np.exp(lj - lse).T[:, :, None] * oj.reshape(Sq, n_heads, d)
+    return o.reshape(Sq, n_heads * d), lse
+
+
 # --------------------------------------------------------------------------
 # Blocks
 # --------------------------------------------------------------------------

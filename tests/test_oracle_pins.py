@@ -420,3 +420,25 @@ def test_golden_flux_shapes():
 def test_flops_model():
     f = O.single_block_flops(4608, 3072, 12288, 24)
     assert abs(f - 1.3047e12) / 1.3047e12 < 1e-3
+
+
+def test_attention_merge_over_key_splits_is_full_attention():
+    """Splitting the keys into disjoint sets and merging by log-sum-exp gives
+    the attention over all keys (up to rounding), for uneven splits and a
+    permuted order of the parts."""
+    r = rng(41)
+    H, d, Sq, Skv = 2, 8, 5, 23
+    q, k, v = (r.standard_normal((n, H * d)) for n in (Sq, Skv, Skv))
+    full = O.attention(q, k, v, H)
+    full_lse = O.attention_lse(q, k, H)
+    cuts = [0, 4, 5, 15, 23]
+    outs = [O.attention(q, k[a:b], v[a:b], H) for a, b in zip(cuts, cuts[1:])]
+    lses = [O.attention_lse(q, k[a:b], H) for a, b in zip(cuts, cuts[1:])]
+    o, lse = O.attention_merge(outs[::-1], lses[::-1])
+    np.testing.assert_allclose(o, full, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(lse, full_lse, rtol=1e-12, atol=1e-12)
+    # one part: unchanged; a part with lse far below the others gets no weight
+    o1, l1 = O.attention_merge(outs[:1], lses[:1])
+    np.testing.assert_array_equal(o1, outs[0])
+    o2, _ = O.attention_merge([outs[0], outs[1] + 1e6], [lses[0], lses[1] - 1e4])
+    np.testing.assert_allclose(o2, outs[0], rtol=1e-12, atol=1e-9)
