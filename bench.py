@@ -548,6 +548,57 @@ def run_video(args):
                        {"gpu_launches_per_step": 14})
 
 
+def run_ring8(args):
+    """One rank's compute in a CP=8 ring over the Flux sequence (4608 tokens
+    = 8 x 576 per rank, 24 heads x 128), on one GPU: attention of the 576 local
+    queries against each of the 8 key/value shards plus 7 in-place
+    log-sum-exp merges, captured as one CUDA graph (the transfers between
+    ranks are not part of this single-GPU measurement)."""
+    import torch
+    import diffusion_transformer_block_flux_b200 as dit
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device=dev)
+    g.manual_seed(13)
+    N, Sl = 8, S // 8
+    NB = 4  # buffer sets, rotated so K/V shards are not all L2-resident from the last replay
+    q = [_rand(torch, g, dev, Sl, D) for _ in range(NB)]
+    kv = [_rand(torch, g, dev, 2, S, D) for _ in range(NB)]
+    o = torch.empty((Sl, D), dtype=torch.bfloat16, device=dev)
+    part = torch.empty_like(o)
+    lse = torch.empty((1, H, Sl), dtype=torch.float32, device=dev)
+    lpart = torch.empty_like(lse)
+
+    def ring(i):
+        k, v = kv[i][0], kv[i][1]
+        for j in range(N):
+            ks, vs = k[j * Sl:(j + 1) * Sl], v[j * Sl:(j + 1) * Sl]
+            if j == 0:
+                dit.dit_attention(q[i], ks, vs, o, 1, Sl, Sl, H, lse=lse)
+            else:
+                dit.dit_attention(q[i], ks, vs, part, 1, Sl, Sl, H, lse=lpart)
+                dit.dit_attention_merge([o, part], [lse, lpart], o, lse, 1, Sl, H)
+
+    for i in range(NB):
+        ring(i)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for i in range(NB):
+            ring(i)
+    K = max(5, args.steps // 4)
+    ms = _event_time(torch, graph.replay, K, 3, torch.cuda.current_stream()) / NB
+    del graph
+    st, code = dit.dit_get_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error word {code:#x}")
+    flops = 4.0 * Sl * S * H * 128
+    return _extra_line("ring_cp8_rank_compute_S4608_576q_24x128", ms, flops, K * NB, 3,
+                       {"us_per_hop": round(ms * 1e3 / N, 2), "hops": N, "merges": N - 1,
+                        "gpu_launches_per_step": 2 * N - 1,
+                        "context": "the compile_graph page, section 5: one attention segment of the 8-card ring "
+                                   "took 0.073 ms on H20"})
+
+
 def run_loop(args):
     """Flux.1-dev-shaped denoising loop at 1024^2: 19 double + 38 single blocks,
     50 flow-match Euler steps, captured once as one CUDA graph and replayed."""
@@ -681,7 +732,7 @@ def run_kernels(args):
             "hbm_peak_gbs": pk["hbm_gbs"], "kernels": res}
 
 
-EXTRA = {"double": run_double, "video": run_video, "loop": run_loop, "kernels": run_kernels}
+EXTRA = {"double": run_double, "video": run_video, "loop": run_loop, "kernels": run_kernels, "ring8": run_ring8}
 
 
 def main():

@@ -124,6 +124,8 @@ _SIGS = {
     "dit_attention": (i32, [c_void_p, c_void_p, c_void_p, i64, i64, i64, c_void_p, i64, c_void_p, i32, i32,
                             i32, i32, i32, f32, c_void_p]),
     "dit_gemm_epilogue": (i32, [ctypes.POINTER(dit_gemm_args), c_void_p]),
+    "dit_attention_merge": (i32, [i32, ctypes.POINTER(c_void_p), ctypes.POINTER(c_void_p), i64, c_void_p, c_void_p,
+                                  i64, i32, i32, i32, c_void_p]),
     "dit_single_block_workspace": (size_t, [ctypes.POINTER(dit_block_cfg)]),
     "dit_double_block_workspace": (size_t, [ctypes.POINTER(dit_block_cfg)]),
     "dit_video_block_workspace": (size_t, [ctypes.POINTER(dit_block_cfg), i32]),
@@ -283,6 +285,21 @@ def dit_attention(q, k, v, o, B, Sq, Skv, H, softmax_scale=None, lse=None, strea
         softmax_scale = 128 ** -0.5
     _call("dit_attention", _ptr(q), _ptr(k), _ptr(v), q.stride(0), k.stride(0), v.stride(0), _ptr(o),
           o.stride(0), _ptr(lse), B, Sq, Skv, H, 128, float(softmax_scale), _stream(stream))
+
+
+def dit_attention_merge(o_parts, lse_parts, o, lse_out, B, Sq, H, stream=None):
+    """o = log-sum-exp weighted merge of attention results over disjoint key
+    sets; o_parts: bf16 [B*Sq, >= H*128] tensors (one row stride), lse_parts:
+    fp32 [B, H, Sq].  o may be one of o_parts, lse_out one of lse_parts."""
+    n = len(o_parts)
+    if len(lse_parts) != n:
+        raise ValueError("o_parts and lse_parts must have the same length")
+    ld = o_parts[0].stride(0)
+    if any(t.stride(0) != ld for t in o_parts):
+        raise ValueError("all parts must share one row stride")
+    op = (c_void_p * n)(*[t.data_ptr() for t in o_parts])
+    lp = (c_void_p * n)(*[t.data_ptr() for t in lse_parts])
+    _call("dit_attention_merge", n, op, lp, ld, _ptr(o), _ptr(lse_out), o.stride(0), B, Sq, H, _stream(stream))
 
 
 def dit_gemm_epilogue(A, W, C, epi=DIT_EPI_NONE, bias=None, C2=None, split_col=0, gelu_col_begin=0,

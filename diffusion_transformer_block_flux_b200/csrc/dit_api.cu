@@ -442,6 +442,38 @@ dit_status dit_attention(const dit_bf16* q, const dit_bf16* k, const dit_bf16* v
   return launch_status();
 }
 
+dit_status dit_attention_merge(int n, const dit_bf16* const* o_parts, const float* const* lse_parts, int64_t ld_in,
+                               dit_bf16* o, float* lse_out, int64_t ld_out, int B, int S, int H, void* stream) {
+  if (o_parts == nullptr || lse_parts == nullptr || o == nullptr) return DIT_ERR_INVALID_ARG;
+  if (n < 1 || n > dit::kMergeMaxParts) return DIT_ERR_INVALID_ARG;
+  if (B < 1 || S < 1 || H < 1) return DIT_ERR_SHAPE;
+  const int64_t D = (int64_t)H * 128;
+  if (ld_in < D || ld_out < D) return DIT_ERR_SHAPE;
+  if ((ld_in % 8) || (ld_out % 8) || !aligned16(o)) return DIT_ERR_ALIGNMENT;
+  dit::MergeParams p{};
+  for (int j = 0; j < n; ++j) {
+    if (o_parts[j] == nullptr || lse_parts[j] == nullptr) return DIT_ERR_INVALID_ARG;
+    if (!aligned16(o_parts[j])) return DIT_ERR_ALIGNMENT;
+    p.o[j] = reinterpret_cast<const bf16*>(o_parts[j]);
+    p.lse[j] = lse_parts[j];
+  }
+  p.out = reinterpret_cast<bf16*>(o);
+  p.lse_out = lse_out;
+  p.ld_in = ld_in;
+  p.ld_out = ld_out;
+  p.n = n;
+  p.B = B;
+  p.S = S;
+  p.H = H;
+  dit_status s = device_setup(nullptr);
+  if (s != DIT_OK) return s;
+  const int64_t threads = (int64_t)B * S * H * 16;
+  const int64_t blocks = (threads + 255) / 256;
+  if (blocks > INT32_MAX) return DIT_ERR_SHAPE;
+  dit::attention_merge_kernel<<<(unsigned)blocks, 256, 0, (cudaStream_t)stream>>>(p);
+  return launch_status();
+}
+
 dit_status dit_gemm_epilogue(const dit_gemm_args* a, void* stream) {
   if (a == nullptr || a->A == nullptr || a->W == nullptr || a->C == nullptr) return DIT_ERR_INVALID_ARG;
   if (a->M < 1 || a->N < 32 || a->K < 8 || (a->N % 32) != 0 || (a->K % 8) != 0) return DIT_ERR_SHAPE;

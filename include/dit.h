@@ -176,6 +176,21 @@ dit_status dit_attention(const dit_bf16* q, const dit_bf16* k, const dit_bf16* v
                          float* lse, int B, int Sq, int Skv, int H, int head_dim,
                          float softmax_scale, void* stream);
 
+/* Merge of attention results over disjoint key sets ([CG] §5: sequence-
+ * parallel ring attention merges each hop's partial result by its
+ * log-sum-exp):
+ *   lse[b,h,i] = log sum_j exp(lse_j[b,h,i])
+ *   o[b,i,h,:] = sum_j exp(lse_j[b,h,i] - lse[b,h,i]) o_j[b,i,h,:]
+ * n: 1..8 parts.  o_parts, lse_parts: host arrays of n device pointers; part
+ * j is bf16 [B][Sq][ld_in] (head h at column h*128, as dit_attention writes
+ * it) with its fp32 lse [B][H][Sq] from dit_attention.  o: bf16 [B][Sq][ld_out];
+ * lse_out: NULL or fp32 [B][H][Sq].  o may equal any o_parts[j] and lse_out
+ * any lse_parts[j] (so a ring can merge into its running result).  Weights
+ * and sums in fp32; o rounded to bf16 once. */
+dit_status dit_attention_merge(int n, const dit_bf16* const* o_parts, const float* const* lse_parts,
+                               int64_t ld_in, dit_bf16* o, float* lse_out, int64_t ld_out,
+                               int B, int Sq, int H, void* stream);
+
 /* ------------------------------------------------------------------------
  * GEMM with fused epilogue ([CG] §1.1 tail fused into the producing kernel;
  * the block's linears: QKV|MLP-in and the output projection)

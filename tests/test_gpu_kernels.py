@@ -288,6 +288,97 @@ def test_attention_strided_views_in_packed_buffer():
     assert torch.count_nonzero(cat[:, D:]) == 0
 
 
+# ---------------------------------------------------------------- sequence-parallel pieces
+
+@pytest.mark.parametrize("n,B,S,H", [(2, 1, 300, 3), (5, 2, 77, 2), (8, 1, 4608 // 8, 24)])
+def test_attention_merge_matches_oracle(n, B, S, H):
+    """Merge of n bf16 partial results with their fp32 lse against the fp64
+    merge of the same inputs; in place into the first part and its lse."""
+    import torch
+    D = H * 128
+    r = np.random.default_rng(n)
+    parts = [synth.normal_bf16(20 + j, f"o{j}", (B * S, D)) for j in range(n)]
+    lses = [(r.standard_normal((B, H, S)) * 3.0 + j).astype(np.float32) for j in range(n)]
+    dp = [dev_bf16(t) for t in parts]
+    dl = [torch.from_numpy(x).cuda() for x in lses]
+    o = torch.empty((B * S, D), dtype=torch.bfloat16, device="cuda")
+    lo = torch.empty((B, H, S), dtype=torch.float32, device="cuda")
+    dit.dit_attention_merge(dp, dl, o, lo, B, S, H)
+    pf = [synth.bf16_bits_to_f64(t).reshape(B, S, D) for t in parts]
+    got = host_f64(o).reshape(B, S, D)
+    for b in range(B):
+        ref, ref_lse = O.attention_merge([p[b] for p in pf], [x[b].astype(np.float64) for x in lses])
+        parity(got[b], ref, f"merge b={b}")
+        assert np.abs(lo[b].cpu().double().numpy() - ref_lse).max() < 1e-5 * max(1.0, np.abs(ref_lse).max())
+    # in place: the running result of a ring
+    dit.dit_attention_merge(dp, dl, dp[0], dl[0], B, S, H)
+    assert torch.equal(dp[0], o) and torch.equal(dl[0], lo)
+    assert_no_device_error()
+
+
+def test_ring_schedule_on_one_gpu_equals_full_attention():
+    """The arithmetic of one rank's ring hops on one GPU: attention of the
+    queries against each of 4 key/value shards (uneven tail), merged hop by
+    hop into the running result, equals attention over all keys."""
+    import torch
+    S, H = 640, 4
+    D = H * 128
+    q, k, v = (synth.normal_bf16(60 + i, n, (S, D)) for i, n in enumerate("qkv"))
+    dq, dk, dv = dev_bf16(q), dev_bf16(k), dev_bf16(v)
+    cuts = [0, 128, 300, 512, 640]
+    o = torch.empty((S, D), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((1, H, S), dtype=torch.float32, device="cuda")
+    part = torch.empty_like(o)
+    lpart = torch.empty_like(lse)
+    for j, (a, b) in enumerate(zip(cuts, cuts[1:])):
+        if j == 0:
+            dit.dit_attention(dq, dk[a:b], dv[a:b], o, 1, S, b - a, H, lse=lse)
+        else:
+            dit.dit_attention(dq, dk[a:b], dv[a:b], part, 1, S, b - a, H, lse=lpart)
+            dit.dit_attention_merge([o, part], [lse, lpart], o, lse, 1, S, H)
+    qf, kf, vf = (synth.bf16_bits_to_f64(t) for t in (q, k, v))
+    ref = O.attention(qf, kf, vf, H)
+    rms = np.sqrt(np.mean(ref ** 2))
+    # each hop's output and the merge round to bf16: four roundings of <= 2^-9
+    parity(host_f64(o), ref, "ring on one GPU", max_abs_frac=3e-2 + 4 * 2.0 ** -9 * np.abs(ref).max() / rms)
+    ref_lse = O.attention_lse(qf, kf, H)
+    assert np.abs(lse[0].cpu().double().numpy() - ref_lse).max() < 1e-3 * max(1.0, np.abs(ref_lse).max())
+    assert_no_device_error()
+
+
+def test_sequence_parallel_drivers_with_cuda_kernels_one_rank():
+    """ring_attention and ulysses_attention with their default CUDA local
+    operations in a one-rank NCCL group (no transfer; the multi-rank
+    schedules are checked on CPU ranks)."""
+    import datetime
+    import socket
+    import torch
+    import torch.distributed as dist
+    from diffusion_transformer_block_flux_b200 import sequence_parallel as sp
+    sock = socket.socket()
+    sock.bind(("127.0.0.1", 0))
+    port = sock.getsockname()[1]
+    sock.close()
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        S, H = 256, 2
+        D = H * 128
+        q, k, v = (synth.normal_bf16(70 + i, n, (S, D)) for i, n in enumerate("qkv"))
+        dq, dk, dv = dev_bf16(q), dev_bf16(k), dev_bf16(v)
+        ref = torch.empty((S, D), dtype=torch.bfloat16, device="cuda")
+        dit.dit_attention(dq, dk, dv, ref, 1, S, S, H)
+        o_ring = torch.empty_like(ref)
+        sp.ring_attention(dq, dk, dv, o_ring, H)
+        o_uly = torch.empty_like(ref)
+        sp.ulysses_attention(dq, dk, dv, o_uly, H)
+        torch.cuda.synchronize()
+        assert torch.equal(o_ring, ref) and torch.equal(o_uly, ref)
+    finally:
+        dist.destroy_process_group()
+    assert_no_device_error()
+
+
 # ---------------------------------------------------------------- failure detection
 
 def test_selftest_wait_times_out_and_reports():
