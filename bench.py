@@ -697,6 +697,13 @@ def run_kernels(args):
         i = nxt()
         dit.dit_adaln_modulation(vec, Ws[i], None, mout)
 
+    mo = [_rand(torch, g, dev, S, D) for _ in range(NB)]
+    ml = [torch.randn((1, H, S), generator=g, device=dev) for _ in range(2 * NB)]
+
+    def merge():  # one ring hop's merge: running result + new part, in place
+        i = nxt()
+        dit.dit_attention_merge([ys[i], mo[i]], [ml[2 * i], ml[2 * i + 1]], ys[i], ml[2 * i], 1, S, H)
+
     def copy():  # yardstick, not part of the path: a library copy of the LayerNorm's bytes
         i = nxt()
         ys[i].copy_(xs[i])
@@ -709,6 +716,7 @@ def run_kernels(args):
     for name, fn, nbytes in (("modulate_norm", ln, 2 * S * D * 2),
                              ("qk_norm_rope", qk, 4 * S * D * 2 + S * 64 * 8),
                              ("adaln_modulation", ada, 3 * D * D * 2),
+                             ("attention_merge_2parts", merge, 3 * S * D * 2 + 3 * H * S * 4),
                              ("torch_copy_same_bytes_as_modulate_norm", copy, 2 * S * D * 2)):
         for _ in range(args.warmup):
             fn()

@@ -446,7 +446,7 @@ dit_status dit_attention_merge(int n, const dit_bf16* const* o_parts, const floa
                                dit_bf16* o, float* lse_out, int64_t ld_out, int B, int S, int H, void* stream) {
   if (o_parts == nullptr || lse_parts == nullptr || o == nullptr) return DIT_ERR_INVALID_ARG;
   if (n < 1 || n > dit::kMergeMaxParts) return DIT_ERR_INVALID_ARG;
-  if (B < 1 || S < 1 || H < 1) return DIT_ERR_SHAPE;
+  if (B < 1 || S < 1 || H < 1 || B > 65535 || H > 65535) return DIT_ERR_SHAPE;
   const int64_t D = (int64_t)H * 128;
   if (ld_in < D || ld_out < D) return DIT_ERR_SHAPE;
   if ((ld_in % 8) || (ld_out % 8) || !aligned16(o)) return DIT_ERR_ALIGNMENT;
@@ -467,10 +467,13 @@ dit_status dit_attention_merge(int n, const dit_bf16* const* o_parts, const floa
   p.H = H;
   dit_status s = device_setup(nullptr);
   if (s != DIT_OK) return s;
-  const int64_t threads = (int64_t)B * S * H * 16;
-  const int64_t blocks = (threads + 255) / 256;
-  if (blocks > INT32_MAX) return DIT_ERR_SHAPE;
-  dit::attention_merge_kernel<<<(unsigned)blocks, 256, 0, (cudaStream_t)stream>>>(p);
+  const dim3 grid((unsigned)((S + 15) / 16), (unsigned)H, (unsigned)B);
+  if (n <= 2)
+    dit::attention_merge_kernel<2><<<grid, 256, 0, (cudaStream_t)stream>>>(p);
+  else if (n <= 4)
+    dit::attention_merge_kernel<4><<<grid, 256, 0, (cudaStream_t)stream>>>(p);
+  else
+    dit::attention_merge_kernel<8><<<grid, 256, 0, (cudaStream_t)stream>>>(p);
   return launch_status();
 }
 

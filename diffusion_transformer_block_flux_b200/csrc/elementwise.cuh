@@ -395,7 +395,7 @@ __global__ void __launch_bounds__(256) vec_linear_bulk_kernel(const bf16* __rest
 // Log-sum-exp merge of attention results over disjoint key sets (the ring
 // attention hop merge of "compile_graph" (chenyy20.com) §5):
 //   lse = log sum_j exp(lse_j),  o = sum_j exp(lse_j - lse) o_j.
-// 16 threads per (batch, token, head) row of 128, 8 values each; weights in
+// 16 threads per (batch, head, token) row of 128, 8 values each; weights in
 // fp32.  Each thread reads its columns of every part before writing them, so
 // the output may be one of the parts; the row's lse is written after the
 // half-warp has read every part's lse, so lse_out may be one of them too.
@@ -410,47 +410,45 @@ struct MergeParams {
   int n, B, S, H;
 };
 
+template <int NP>  // bound on the number of parts (2, 4 or 8): every load is issued before any is used
 __global__ void __launch_bounds__(256) attention_merge_kernel(const __grid_constant__ MergeParams p) {
-  const int64_t row = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 4;  // (b, s, h), h fastest
+  // grid (tokens / 16, H, B): 16 consecutive tokens of one (batch, head) per
+  // CTA, so the lse accesses are contiguous and no index needs a division
+  const int s = blockIdx.x * 16 + (threadIdx.x >> 4);
   const int sub = threadIdx.x & 15;
-  const int64_t rows = (int64_t)p.B * p.S * p.H;
-  const bool valid = row < rows;
-  const int h = valid ? (int)(row % p.H) : 0;
-  const int64_t bs = valid ? row / p.H : 0;  // b * S + s
-  const int s = (int)(bs % p.S);
-  const int b = (int)(bs / p.S);
-  const int64_t li = ((int64_t)b * p.H + h) * p.S + s;
-  float l[kMergeMaxParts];
-  float m = -INFINITY;
-#pragma unroll
-  for (int j = 0; j < kMergeMaxParts; ++j) {
-    l[j] = (j < p.n && valid) ? p.lse[j][li] : -INFINITY;
-    m = fmaxf(m, l[j]);
-  }
-  float den = 0.0f;
-#pragma unroll
-  for (int j = 0; j < kMergeMaxParts; ++j) {
-    l[j] = (j < p.n && valid) ? __expf(l[j] - m) : 0.0f;
-    den += l[j];
-  }
-  const float inv = valid ? 1.0f / den : 0.0f;
-  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  const int h = blockIdx.y, b = blockIdx.z;
+  const bool valid = s < p.S;
+  const int64_t li = ((int64_t)b * p.H + h) * p.S + (valid ? s : 0);
+  const int64_t bs = (int64_t)b * p.S + (valid ? s : 0);
   const int64_t col = (int64_t)h * 128 + sub * 8;
+  float l[NP];
+  uint4 u[NP];
 #pragma unroll
-  for (int j = 0; j < kMergeMaxParts; ++j) {
-    if (j < p.n && valid) {
-      const uint4 u = *reinterpret_cast<const uint4*>(p.o[j] + bs * p.ld_in + col);
-      const float wj = l[j] * inv;
-      acc[0] = fmaf(wj, bf16_lo(u.x), acc[0]); acc[1] = fmaf(wj, bf16_hi(u.x), acc[1]);
-      acc[2] = fmaf(wj, bf16_lo(u.y), acc[2]); acc[3] = fmaf(wj, bf16_hi(u.y), acc[3]);
-      acc[4] = fmaf(wj, bf16_lo(u.z), acc[4]); acc[5] = fmaf(wj, bf16_hi(u.z), acc[5]);
-      acc[6] = fmaf(wj, bf16_lo(u.w), acc[6]); acc[7] = fmaf(wj, bf16_hi(u.w), acc[7]);
-    }
+  for (int j = 0; j < NP; ++j) {
+    const bool on = valid && j < p.n;
+    l[j] = on ? p.lse[j][li] : -INFINITY;
+    u[j] = on ? *reinterpret_cast<const uint4*>(p.o[j] + bs * p.ld_in + col) : make_uint4(0, 0, 0, 0);
   }
-  if (valid)
+  float m = l[0];
+#pragma unroll
+  for (int j = 1; j < NP; ++j) m = fmaxf(m, l[j]);
+  float den = 0.0f;
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int j = 0; j < NP; ++j) {
+    const float wj = (j < p.n) ? __expf(l[j] - m) : 0.0f;
+    den += wj;
+    acc[0] = fmaf(wj, bf16_lo(u[j].x), acc[0]); acc[1] = fmaf(wj, bf16_hi(u[j].x), acc[1]);
+    acc[2] = fmaf(wj, bf16_lo(u[j].y), acc[2]); acc[3] = fmaf(wj, bf16_hi(u[j].y), acc[3]);
+    acc[4] = fmaf(wj, bf16_lo(u[j].z), acc[4]); acc[5] = fmaf(wj, bf16_hi(u[j].z), acc[5]);
+    acc[6] = fmaf(wj, bf16_lo(u[j].w), acc[6]); acc[7] = fmaf(wj, bf16_hi(u[j].w), acc[7]);
+  }
+  if (valid) {
+    const float inv = 1.0f / den;
     *reinterpret_cast<uint4*>(p.out + bs * p.ld_out + col) =
-        make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]), pack_bf16x2(acc[4], acc[5]),
-                   pack_bf16x2(acc[6], acc[7]));
+        make_uint4(pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv),
+                   pack_bf16x2(acc[4] * inv, acc[5] * inv), pack_bf16x2(acc[6] * inv, acc[7] * inv));
+  }
   __syncwarp();
   if (valid && sub == 0 && p.lse_out != nullptr) p.lse_out[li] = m + __logf(den);
 }

@@ -186,7 +186,7 @@ dit_status dit_attention(const dit_bf16* q, const dit_bf16* k, const dit_bf16* v
  * it) with its fp32 lse [B][H][Sq] from dit_attention.  o: bf16 [B][Sq][ld_out];
  * lse_out: NULL or fp32 [B][H][Sq].  o may equal any o_parts[j] and lse_out
  * any lse_parts[j] (so a ring can merge into its running result).  Weights
- * and sums in fp32; o rounded to bf16 once. */
+ * and sums in fp32; o rounded to bf16 once.  1 <= B, H <= 65535. */
 dit_status dit_attention_merge(int n, const dit_bf16* const* o_parts, const float* const* lse_parts,
                                int64_t ld_in, dit_bf16* o, float* lse_out, int64_t ld_out,
                                int B, int Sq, int H, void* stream);
