@@ -334,8 +334,8 @@ NCU_TRAFFIC = {
     "gemm_qkv_mlp_gelu_qknorm_rope": (336449280, ("gemm.cuh", "common.cuh"), "fc2cefdbf8d48145"),
     "gemm_out_gated_residual": (586581760, ("gemm.cuh", "common.cuh"), "fc2cefdbf8d48145"),
     "attention": (95049984, ("attention.cuh", "common.cuh"), "703ad1ee60f1efde"),
-    "modulate_norm": (28416512, ("elementwise.cuh", "common.cuh"), "b21596d7241c9891"),
-    "adaln_modulation": (56665344, ("elementwise.cuh", "common.cuh"), "b21596d7241c9891"),
+    "modulate_norm": (28414720, ("elementwise.cuh", "common.cuh"), "1a3bc3caf0ed9be5"),
+    "adaln_modulation": (56782336, ("elementwise.cuh", "common.cuh"), "1a3bc3caf0ed9be5"),
 }
 
 
