@@ -109,6 +109,15 @@ dit_status device_setup(int* num_sms) {
             (const void*)dit::vec_linear_pipe_kernel<3>, (const void*)dit::vec_linear_pipe_kernel<4>,
             (const void*)dit::vec_linear_pipe_kernel<6>, (const void*)dit::vec_linear_pipe_kernel<8>,
             (const void*)dit::vec_linear_pipe_kernel<12>, (const void*)dit::vec_linear_pipe_kernel<16>};
+        const void* vec_multi[8] = {
+            (const void*)dit::vec_linear_multi_kernel<1>, (const void*)dit::vec_linear_multi_kernel<2>,
+            (const void*)dit::vec_linear_multi_kernel<3>, (const void*)dit::vec_linear_multi_kernel<4>,
+            (const void*)dit::vec_linear_multi_kernel<6>, (const void*)dit::vec_linear_multi_kernel<8>,
+            (const void*)dit::vec_linear_multi_kernel<12>, (const void*)dit::vec_linear_multi_kernel<16>};
+        for (const void* f : vec_multi) {
+          DIT_CUDA_CHECK(cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, kVecPipeSmemMax));
+          DIT_CUDA_CHECK(cudaFuncSetAttribute(f, cudaFuncAttributePreferredSharedMemoryCarveout, 100));
+        }
         // the grid assumes every CTA the occupancy calculator allows is resident: ask for the
         // largest shared-memory carveout so the launch does not pick a smaller one
         for (const void* f : vec_pipe) {
@@ -326,6 +335,40 @@ dit_status dit_vec_linear(const dit_bf16* x, int64_t ldx, const dit_bf16* W, int
   else
     dit::vec_linear_kernel<8><<<blocks, threads, smem, st>>>(xb, ldx, Wb, ldw, bb, out, ldo, B, N, K, flags);
   return launch_status();
+}
+
+// One pass over every matrix of p (batch-1 input x shared by all): see
+// vec_linear_multi_kernel.  K % 256 == 0, K <= 4096; used by the loop.
+bool multi_linear_supported(int K) { return (K % 256) == 0 && K <= 4096; }
+
+dit_status multi_linear(const dit_bf16* x, const dit::MultiLinear& p, int flags, cudaStream_t st) {
+  if (!multi_linear_supported(p.K) || p.n_mats < 1 || p.n_mats > dit::kMultiMaxMats) return DIT_ERR_SHAPE;
+  int sms = 0;
+  dit_status s = device_setup(&sms);
+  if (s != DIT_OK) return s;
+  const int64_t N = p.row_begin[p.n_mats];
+  const size_t smem = (size_t)dit::kVecPipeWarps * dit::kVecPipeSlots * p.K * 2 + (size_t)p.K * 4;
+  int64_t grid = (N + dit::kVecPipeWarps - 1) / dit::kVecPipeWarps;
+  const int per_sm = (int)(220 * 1024 / (smem + 1024));
+  if (grid > (int64_t)sms * per_sm) grid = (int64_t)sms * per_sm;
+  const bf16* xb = reinterpret_cast<const bf16*>(x);
+  switch (p.K / 256) {
+#define DIT_VM_CASE(KC_)                                                                        \
+  case KC_:                                                                                     \
+    dit::vec_linear_multi_kernel<KC_><<<(unsigned)grid, 128, smem, st>>>(xb, p, flags);        \
+    return launch_status();
+    DIT_VM_CASE(1)
+    DIT_VM_CASE(2)
+    DIT_VM_CASE(3)
+    DIT_VM_CASE(4)
+    DIT_VM_CASE(6)
+    DIT_VM_CASE(8)
+    DIT_VM_CASE(12)
+    DIT_VM_CASE(16)
+#undef DIT_VM_CASE
+    default:
+      return DIT_ERR_SHAPE;
+  }
 }
 
 dit_status dit_adaln_modulation(const dit_bf16* vec, int64_t ldv, const dit_bf16* W, int64_t ldw,

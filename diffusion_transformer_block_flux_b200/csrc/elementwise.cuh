@@ -299,6 +299,108 @@ __global__ void __launch_bounds__(128) vec_linear_pipe_kernel(const bf16* __rest
 }
 
 // ---------------------------------------------------------------------------
+// The same contraction over a list of matrices that share one input vector:
+// every block's adaLN modulation of a denoising step depends only on that
+// step's conditioning vector, so all of them stream in one pass.  Global row
+// n belongs to matrix j with row_begin[j] <= n < row_begin[j+1] (binary
+// search); out[j][n - row_begin[j]] = W_j[row] . f(x) + bias_j[row], fp32.
+// Rows are dealt to warps and streamed exactly as in vec_linear_pipe_kernel
+// (same column order, same accumulation), so every output equals that
+// kernel's output for the same matrix.  Every matrix has K columns, ldw = K.
+// ---------------------------------------------------------------------------
+constexpr int kMultiMaxMats = 96;
+struct MultiLinear {
+  const bf16* W[kMultiMaxMats];
+  const bf16* bias[kMultiMaxMats];
+  float* out[kMultiMaxMats];
+  int row_begin[kMultiMaxMats + 1];
+  int n_mats;
+  int K;
+};
+
+__device__ __forceinline__ int multi_find(const MultiLinear& p, int64_t n) {
+  int lo = 0, hi = p.n_mats - 1;  // largest j with row_begin[j] <= n
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (p.row_begin[mid] <= n) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+template <int KC>
+__global__ void __launch_bounds__(128) vec_linear_multi_kernel(const bf16* __restrict__ x,
+                                                               const __grid_constant__ MultiLinear p, int flags) {
+  constexpr int P = kVecPipeSlots;
+  extern __shared__ __align__(16) uint4 wring[];  // [warps][P][K / 8], then the mapped input (K fp32)
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int K = p.K;
+  const int row_chunks = K / 8;
+  const int64_t N = p.row_begin[p.n_mats];
+  uint4* ring = wring + (size_t)warp * P * row_chunks;
+  float* xs = reinterpret_cast<float*>(wring + (size_t)kVecPipeWarps * P * row_chunks);
+  const int64_t nw = (int64_t)gridDim.x * kVecPipeWarps;
+  const int64_t n0 = (int64_t)blockIdx.x * kVecPipeWarps + warp;
+  auto row_ptr = [&](int64_t n) -> const uint4* {
+    const int j = multi_find(p, n);
+    return reinterpret_cast<const uint4*>(p.W[j] + (n - p.row_begin[j]) * K);
+  };
+#pragma unroll
+  for (int k = 0; k < P - 1; ++k) {
+    const int64_t nn = n0 + k * nw;
+    if (nn < N) {
+      const uint4* src = row_ptr(nn);
+#pragma unroll
+      for (int j = 0; j < KC; ++j) cp_async16(&ring[k * row_chunks + lane + 32 * j], src + lane + 32 * j);
+    }
+    cp_async_commit();
+  }
+  for (int k = threadIdx.x; k < K; k += blockDim.x) {
+    float z = __bfloat162float(x[k]);
+    if (flags & DIT_VEC_SILU_IN) z = silu(z);
+    xs[k] = z;
+  }
+  __syncthreads();
+  float xv[KC * 8];
+#pragma unroll
+  for (int j = 0; j < KC; ++j) {
+    const float4* q = reinterpret_cast<const float4*>(xs + (lane + 32 * j) * 8);
+    const float4 a = q[0], c = q[1];
+    xv[j * 8 + 0] = a.x; xv[j * 8 + 1] = a.y; xv[j * 8 + 2] = a.z; xv[j * 8 + 3] = a.w;
+    xv[j * 8 + 4] = c.x; xv[j * 8 + 5] = c.y; xv[j * 8 + 6] = c.z; xv[j * 8 + 7] = c.w;
+  }
+  int slot = 0;
+  for (int64_t n = n0; n < N; n += nw) {
+    {  // the slot consumed one row ago gets the row P - 1 ahead
+      const int64_t nn = n + (int64_t)(P - 1) * nw;
+      const int si = (slot == 0 ? P : slot) - 1;
+      if (nn < N) {
+        const uint4* src = row_ptr(nn);
+#pragma unroll
+        for (int j = 0; j < KC; ++j) cp_async16(&ring[si * row_chunks + lane + 32 * j], src + lane + 32 * j);
+      }
+      cp_async_commit();
+    }
+    const int jm = multi_find(p, n);
+    const int64_t local = n - p.row_begin[jm];
+    const float bv = p.bias[jm] ? __bfloat162float(p.bias[jm][local]) : 0.0f;
+    cp_async_wait<P - 1>();
+    float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+    for (int j = 0; j < KC; ++j) {
+      const uint4 u = ring[slot * row_chunks + lane + 32 * j];
+      a0 = fmaf(bf16_lo(u.x), xv[j * 8 + 0], a0); a1 = fmaf(bf16_hi(u.x), xv[j * 8 + 1], a1);
+      a0 = fmaf(bf16_lo(u.y), xv[j * 8 + 2], a0); a1 = fmaf(bf16_hi(u.y), xv[j * 8 + 3], a1);
+      a0 = fmaf(bf16_lo(u.z), xv[j * 8 + 4], a0); a1 = fmaf(bf16_hi(u.z), xv[j * 8 + 5], a1);
+      a0 = fmaf(bf16_lo(u.w), xv[j * 8 + 6], a0); a1 = fmaf(bf16_hi(u.w), xv[j * 8 + 7], a1);
+    }
+    const float a = warp_sum(a0 + a1) + bv;
+    if (lane == 0) p.out[jm][local] = a;
+    if (++slot == P) slot = 0;
+  }
+  cp_async_wait<0>();
+}
+
+// ---------------------------------------------------------------------------
 // Bulk-copy staging of rows: 8 warps per CTA, each warp owns a 2-deep ring of
 // row buffers in shared memory; lane 0 starts the copy of the warp's next row
 // before the warp works on the current one.
