@@ -175,12 +175,10 @@ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 dit_status launch_qk(const bf16* q, const bf16* k, int64_t ld_in, const bf16* qs, const bf16* ks, const float* rope,
                      bf16* qo, bf16* ko, int64_t ld_out, int B, int S, int H, float eps, int do_norm,
                      cudaStream_t st) {
-  const int64_t n_vecs = (int64_t)B * S * H * 2;
-  const int threads = 256;
-  const int64_t blocks = (n_vecs * 16 + threads - 1) / threads;
-  dit::qk_norm_rope_kernel<<<(unsigned)blocks, threads, 0, st>>>(q, k, ld_in, qs, ks,
-                                                                  reinterpret_cast<const float2*>(rope), qo, ko,
-                                                                  ld_out, S, H, n_vecs, eps, do_norm);
+  if (B > 65535) return DIT_ERR_SHAPE;
+  const dim3 grid((unsigned)S, (unsigned)B);  // one CTA per token row
+  dit::qk_norm_rope_kernel<3><<<grid, 128, 0, st>>>(q, k, ld_in, qs, ks, reinterpret_cast<const float2*>(rope), qo,
+                                                    ko, ld_out, S, H, eps, do_norm);
   return launch_status();
 }
 

@@ -556,69 +556,92 @@ __global__ void __launch_bounds__(256) attention_merge_kernel(const __grid_const
 }
 
 // ---------------------------------------------------------------------------
-// QK RMSNorm + RoPE: 16 threads per (token, head, q|k) vector of 128, each
-// thread 8 elements = 4 rotation pairs.  In place is safe: a group reads its
-// whole vector before any thread writes.
+// QK RMSNorm + RoPE: one CTA of 128 threads per token row (grid = tokens x
+// batch).  Thread t owns columns 8 (t & 15) .. +8 of every head vector, so its
+// RoPE angles and norm scales are loaded once and reused for all 2H vectors
+// (q heads, then k heads) that its group of 16 walks through, U at a time
+// with every load issued first.  The 16 threads of a vector reduce its sum of
+// squares with shuffles.  In place is safe: a vector is read in full before
+// any of its columns is written.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) qk_norm_rope_kernel(const bf16* q, const bf16* k, int64_t ld_in,
+template <int U>
+__global__ void __launch_bounds__(128) qk_norm_rope_kernel(const bf16* q, const bf16* k, int64_t ld_in,
                                                            const bf16* __restrict__ q_scale,
                                                            const bf16* __restrict__ k_scale,
                                                            const float2* __restrict__ rope, bf16* q_out,
-                                                           bf16* k_out, int64_t ld_out, int S, int H,
-                                                           int64_t n_vecs, float eps, int do_norm) {
-  const int64_t gid = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 4;
-  const int sub = threadIdx.x & 15;
-  const bool valid = gid < n_vecs;
-  const int which = (int)(gid & 1);  // 0: q, 1: k
-  const int64_t hv = gid >> 1;
-  const int h = (int)(hv % H);
-  const int64_t row = hv / H;
-  const int tok = (int)(row % S);
-  const bf16* src = (which ? k : q) + row * ld_in + h * 128 + sub * 8;
-  bf16* dst = (which ? k_out : q_out) + row * ld_out + h * 128 + sub * 8;
-  float v[8];
-  if (valid) {
-    uint4 u = *reinterpret_cast<const uint4*>(src);
-    v[0] = bf16_lo(u.x); v[1] = bf16_hi(u.x); v[2] = bf16_lo(u.y); v[3] = bf16_hi(u.y);
-    v[4] = bf16_lo(u.z); v[5] = bf16_hi(u.z); v[6] = bf16_lo(u.w); v[7] = bf16_hi(u.w);
-  } else {
+                                                           bf16* k_out, int64_t ld_out, int S, int H, float eps,
+                                                           int do_norm) {
+  const int sub = threadIdx.x & 15, grp = threadIdx.x >> 4;  // 8 groups of 16
+  const int tok = blockIdx.x;
+  const int64_t row = (int64_t)blockIdx.y * S + tok;
+  float scq[8], sck[8];  // two named arrays: a runtime index would put them in local memory
 #pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = 0.0f;
-  }
-  float ss = 0.0f;
+  for (int wq = 0; wq < 2; ++wq) {
+    const bf16* sp = wq ? k_scale : q_scale;
+    float* sc = wq ? sck : scq;
+    if (sp != nullptr) {
+      const uint4 u = __ldg(reinterpret_cast<const uint4*>(sp + sub * 8));
+      sc[0] = bf16_lo(u.x); sc[1] = bf16_hi(u.x); sc[2] = bf16_lo(u.y); sc[3] = bf16_hi(u.y);
+      sc[4] = bf16_lo(u.z); sc[5] = bf16_hi(u.z); sc[6] = bf16_lo(u.w); sc[7] = bf16_hi(u.w);
+    } else {
 #pragma unroll
-  for (int i = 0; i < 8; ++i) ss = fmaf(v[i], v[i], ss);
-#pragma unroll
-  for (int o = 8; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-  if (!valid) return;
-  const float r = do_norm ? rsqrtf(ss * (1.0f / 128.0f) + eps) : 1.0f;
-  const bf16* sp = which ? k_scale : q_scale;
-  float sc[8];
-  if (sp != nullptr) {
-    uint4 u = __ldg(reinterpret_cast<const uint4*>(sp + sub * 8));
-    sc[0] = bf16_lo(u.x); sc[1] = bf16_hi(u.x); sc[2] = bf16_lo(u.y); sc[3] = bf16_hi(u.y);
-    sc[4] = bf16_lo(u.z); sc[5] = bf16_hi(u.z); sc[6] = bf16_lo(u.w); sc[7] = bf16_hi(u.w);
-  } else {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) sc[i] = 1.0f;
-  }
-#pragma unroll
-  for (int i = 0; i < 8; ++i) v[i] = v[i] * r * sc[i];
-  if (rope != nullptr) {
-    const float4* rp = reinterpret_cast<const float4*>(rope + (int64_t)tok * 64 + sub * 4);
-    float4 t0 = __ldg(rp), t1 = __ldg(rp + 1);
-    float cs[4][2] = {{t0.x, t0.y}, {t0.z, t0.w}, {t1.x, t1.y}, {t1.z, t1.w}};
-#pragma unroll
-    for (int p = 0; p < 4; ++p) {
-      const float a = v[2 * p], bb = v[2 * p + 1], c = cs[p][0], s = cs[p][1];
-      v[2 * p] = a * c - bb * s;
-      v[2 * p + 1] = a * s + bb * c;
+      for (int i = 0; i < 8; ++i) sc[i] = 1.0f;
     }
   }
-  uint4 w;
-  w.x = pack_bf16x2(v[0], v[1]); w.y = pack_bf16x2(v[2], v[3]);
-  w.z = pack_bf16x2(v[4], v[5]); w.w = pack_bf16x2(v[6], v[7]);
-  *reinterpret_cast<uint4*>(dst) = w;
+  float cs[4][2];
+  if (rope != nullptr) {
+    const float4* rp = reinterpret_cast<const float4*>(rope + (int64_t)tok * 64 + sub * 4);
+    const float4 t0 = __ldg(rp), t1 = __ldg(rp + 1);
+    cs[0][0] = t0.x; cs[0][1] = t0.y; cs[1][0] = t0.z; cs[1][1] = t0.w;
+    cs[2][0] = t1.x; cs[2][1] = t1.y; cs[3][0] = t1.z; cs[3][1] = t1.w;
+  }
+  const int nv = 2 * H;
+  for (int v0 = grp; v0 < nv; v0 += 8 * U) {
+    uint4 u[U];
+#pragma unroll
+    for (int j = 0; j < U; ++j) {
+      const int v = v0 + 8 * j;
+      if (v < nv) {
+        const int w = v >= H, h = v - w * H;
+        u[j] = *reinterpret_cast<const uint4*>((w ? k : q) + row * ld_in + h * 128 + sub * 8);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < U; ++j) {
+      const int v = v0 + 8 * j;
+      const bool on = v < nv;  // uniform across the 16 threads of the vector
+      const int w = v >= H, h = v - w * H;
+      float x[8];
+      if (on) {
+        x[0] = bf16_lo(u[j].x); x[1] = bf16_hi(u[j].x); x[2] = bf16_lo(u[j].y); x[3] = bf16_hi(u[j].y);
+        x[4] = bf16_lo(u[j].z); x[5] = bf16_hi(u[j].z); x[6] = bf16_lo(u[j].w); x[7] = bf16_hi(u[j].w);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) x[i] = 0.0f;
+      }
+      float ss = 0.0f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) ss = fmaf(x[i], x[i], ss);
+#pragma unroll
+      for (int o = 8; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      if (!on) continue;
+      const float r = do_norm ? rsqrtf(ss * (1.0f / 128.0f) + eps) : 1.0f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) x[i] = x[i] * r * (w ? sck[i] : scq[i]);
+      if (rope != nullptr) {
+#pragma unroll
+        for (int pp = 0; pp < 4; ++pp) {
+          const float a = x[2 * pp], bb = x[2 * pp + 1], c = cs[pp][0], sn = cs[pp][1];
+          x[2 * pp] = a * c - bb * sn;
+          x[2 * pp + 1] = a * sn + bb * c;
+        }
+      }
+      uint4 o4;
+      o4.x = pack_bf16x2(x[0], x[1]); o4.y = pack_bf16x2(x[2], x[3]);
+      o4.z = pack_bf16x2(x[4], x[5]); o4.w = pack_bf16x2(x[6], x[7]);
+      *reinterpret_cast<uint4*>((w ? k_out : q_out) + row * ld_out + h * 128 + sub * 8) = o4;
+    }
+  }
 }
 
 // ---------------------------------------------------------------------------
