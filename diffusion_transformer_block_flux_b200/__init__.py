@@ -124,6 +124,7 @@ _SIGS = {
     "dit_attention": (i32, [c_void_p, c_void_p, c_void_p, i64, i64, i64, c_void_p, i64, c_void_p, i32, i32,
                             i32, i32, i32, f32, c_void_p]),
     "dit_gemm_epilogue": (i32, [ctypes.POINTER(dit_gemm_args), c_void_p]),
+    "dit_selftest_exp2_poly": (i32, [c_void_p, c_void_p, i64, c_void_p]),
     "dit_attention_merge": (i32, [i32, ctypes.POINTER(c_void_p), ctypes.POINTER(c_void_p), i64, c_void_p, c_void_p,
                                   i64, i32, i32, i32, c_void_p]),
     "dit_single_block_workspace": (size_t, [ctypes.POINTER(dit_block_cfg)]),
@@ -285,6 +286,11 @@ def dit_attention(q, k, v, o, B, Sq, Skv, H, softmax_scale=None, lse=None, strea
         softmax_scale = 128 ** -0.5
     _call("dit_attention", _ptr(q), _ptr(k), _ptr(v), q.stride(0), k.stride(0), v.stride(0), _ptr(o),
           o.stride(0), _ptr(lse), B, Sq, Skv, H, 128, float(softmax_scale), _stream(stream))
+
+
+def dit_selftest_exp2_poly(x, y, stream=None):
+    """y = the FMA-pipe 2^x approximation used inside the attention softmax (fp32 device tensors)."""
+    _call("dit_selftest_exp2_poly", _ptr(x), _ptr(y), x.numel(), _stream(stream))
 
 
 def dit_attention_merge(o_parts, lse_parts, o, lse_out, B, Sq, H, stream=None):

@@ -320,20 +320,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
       : "memory");
 }
 
-// 32 lanes x 16 consecutive columns (no wait; pair with tmem_wait_ld through
-// a register dependency, see tmem_ld16_wait).
-__device__ __forceinline__ void tmem_ld16_wait(uint32_t taddr, uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n\t"
-      "tcgen05.wait::ld.sync.aligned;"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
-        "=r"(r[15])
-      : "r"(taddr)
-      : "memory");
-}
-
 // 32 lanes x 32 columns without waiting: issue several, then tmem_wait_ld(),
 // then reg_fence32() on each destination so no use moves above the wait.
 __device__ __forceinline__ void tmem_ld32_nowait(uint32_t taddr, uint32_t (&r)[32]) {
@@ -411,21 +397,6 @@ __device__ __forceinline__ float gelu_tanh(float u) {
 
 __device__ __forceinline__ float silu(float z) { return z / (1.0f + __expf(-z)); }
 
-// 2^x on the FMA pipe (frees the MUFU unit): Cody-Waite split x = n + f with
-// n = rint(x) (by adding 1.5 * 2^23) and f in [-0.5, 0.5], 2^f from a cubic
-// fitted to relative error (Lawson-weighted least squares on Chebyshev nodes;
-// max relative error 7.5e-5, far below bf16's 2^-9), 2^n added to the
-// exponent field.  x is clamped at -126 so the result stays a normal or
-// denormal positive number (about 1e-38 at the clamp).
-__device__ __forceinline__ float exp2_poly(float x) {
-  x = fmaxf(x, -126.0f);
-  const float t = x + 12582912.0f;
-  const float f = x - (t - 12582912.0f);
-  const float p = fmaf(fmaf(fmaf(0.0551716648042202f, f, 0.2426111251115799f), f, 0.6932609677314758f), f,
-                       0.9999280571937561f);
-  return __int_as_float(__float_as_int(p) + ((__float_as_int(t) - 0x4B400000) << 23));
-}
-
 // Packed fp32 pairs (sm_100): one instruction updates two lanes of a 64-bit
 // register pair.
 __device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
@@ -449,9 +420,14 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
   return d;
 }
 
-// exp2_poly on a pair: the same Cody-Waite split and cubic, with packed fp32
-// arithmetic; 2^n is added to the exponent field as t_bits << 23 (the magic
-// constant 1.5 * 2^23 contributes nothing modulo 2^32 after the shift).
+// 2^x for a pair of floats on the FMA pipe (frees the MUFU unit), packed fp32
+// arithmetic: Cody-Waite split x = n + f with n = rint(x) (by adding
+// 1.5 * 2^23) and f in [-0.5, 0.5]; 2^f from a cubic fitted to relative error
+// (Lawson-weighted least squares on Chebyshev nodes; max relative error
+// 7.5e-5, far below bf16's 2^-9); 2^n added to the exponent field as
+// t_bits << 23 (the magic constant contributes nothing modulo 2^32 after the
+// shift).  x is clamped at -126 so the result stays a positive normal number
+// (about 1.2e-38 at the clamp).
 __device__ __forceinline__ uint64_t exp2_poly2(float x0, float x1) {
   const uint64_t x = f2_pack(fmaxf(x0, -126.0f), fmaxf(x1, -126.0f));
   const uint64_t magic = f2_pack(12582912.0f, 12582912.0f);

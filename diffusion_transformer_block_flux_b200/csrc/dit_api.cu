@@ -242,6 +242,17 @@ dit_status dit_selftest_wait_timeout(uint64_t limit_ns, void* stream) {
   return launch_status();
 }
 
+dit_status dit_selftest_exp2_poly(const float* x, float* y, int64_t n, void* stream) {
+  if (x == nullptr || y == nullptr || n < 1) return DIT_ERR_INVALID_ARG;
+  dit_status s = device_setup(nullptr);
+  if (s != DIT_OK) return s;
+  const int64_t pairs = (n + 1) / 2;
+  const int64_t blocks = (pairs + 255) / 256;
+  if (blocks > INT32_MAX) return DIT_ERR_SHAPE;
+  dit::selftest_exp2_poly_kernel<<<(unsigned)blocks, 256, 0, (cudaStream_t)stream>>>(x, y, n);
+  return launch_status();
+}
+
 dit_status dit_rope_table(const int32_t* ids, int S, int n_axes, const int* axes_pairs, double theta, float* rope,
                           void* stream) {
   if (ids == nullptr || rope == nullptr || axes_pairs == nullptr) return DIT_ERR_INVALID_ARG;

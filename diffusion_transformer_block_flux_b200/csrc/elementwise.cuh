@@ -555,6 +555,17 @@ __global__ void __launch_bounds__(256) attention_merge_kernel(const __grid_const
   if (valid && sub == 0 && p.lse_out != nullptr) p.lse_out[li] = m + __logf(den);
 }
 
+// Self test of the FMA-pipe 2^x that the attention softmax uses on a part of
+// its exponentials: y[i] = exp2_poly2 evaluated on the pair (x[2j], x[2j+1]).
+__global__ void selftest_exp2_poly_kernel(const float* __restrict__ x, float* __restrict__ y, int64_t n) {
+  const int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (2 * j >= n) return;
+  const float x0 = x[2 * j], x1 = (2 * j + 1 < n) ? x[2 * j + 1] : 0.0f;
+  const uint64_t r = exp2_poly2(x0, x1);
+  y[2 * j] = f2_lo(r);
+  if (2 * j + 1 < n) y[2 * j + 1] = f2_hi(r);
+}
+
 // ---------------------------------------------------------------------------
 // QK RMSNorm + RoPE: one CTA of 128 threads per token row (grid = tokens x
 // batch).  Thread t owns columns 8 (t & 15) .. +8 of every head vector, so its

@@ -94,6 +94,12 @@ dit_status dit_set_wait_limit_ns(uint64_t limit_ns);
  * stream; read the result with dit_get_device_error. */
 dit_status dit_selftest_wait_timeout(uint64_t limit_ns, void* stream);
 
+/* Self test of the 2^x approximation the attention softmax evaluates on the
+ * FMA pipe for a part of its exponentials (Cody-Waite split plus a fitted
+ * cubic; stated maximum relative error 7.5e-5; inputs below -126 are clamped
+ * to -126).  y[i] = that approximation of 2^x[i]; x, y device float [n]. */
+dit_status dit_selftest_exp2_poly(const float* x, float* y, int64_t n, void* stream);
+
 /* ------------------------------------------------------------------------
  * RoPE table ([CG] §3.1: positions from ids, rotation as complex product)
  * ------------------------------------------------------------------------ */
