@@ -331,11 +331,11 @@ def run_ours(args, rank, world, local_rank):
 # (profiles/*.ncu.md), with a hash of the kernel's sources at capture time.
 # A kernel whose sources changed since reports traffic null.
 NCU_TRAFFIC = {
-    "gemm_qkv_mlp_gelu_qknorm_rope": (336449280, ("gemm.cuh", "common.cuh"), "fc2cefdbf8d48145"),
-    "gemm_out_gated_residual": (586581760, ("gemm.cuh", "common.cuh"), "fc2cefdbf8d48145"),
-    "attention": (95049984, ("attention.cuh", "common.cuh"), "703ad1ee60f1efde"),
-    "modulate_norm": (28414720, ("elementwise.cuh", "common.cuh"), "1a3bc3caf0ed9be5"),
-    "adaln_modulation": (56782336, ("elementwise.cuh", "common.cuh"), "1a3bc3caf0ed9be5"),
+    "gemm_qkv_mlp_gelu_qknorm_rope": (335648256, ("gemm.cuh", "common.cuh"), "cf20cddbba096d1c"),
+    "gemm_out_gated_residual": (588929792, ("gemm.cuh", "common.cuh"), "cf20cddbba096d1c"),
+    "attention": (95100928, ("attention.cuh", "common.cuh"), "03b6fdd82910cea2"),
+    "modulate_norm": (28414720, ("elementwise.cuh", "common.cuh"), "97ff3e5e07faf2f4"),
+    "adaln_modulation": (56782336, ("elementwise.cuh", "common.cuh"), "97ff3e5e07faf2f4"),
 }
 
 

@@ -426,8 +426,10 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
 // (Lawson-weighted least squares on Chebyshev nodes; max relative error
 // 7.5e-5, far below bf16's 2^-9); 2^n added to the exponent field as
 // t_bits << 23 (the magic constant contributes nothing modulo 2^32 after the
-// shift).  x is clamped at -126 so the result stays a positive normal number
-// (about 1.2e-38 at the clamp).
+// shift).  x is clamped at -126, so the result is never zero or negative.
+// Within about 1e-4 of the clamp the cubic's value is just below 1 and the
+// exponent sum leaves the normal range.  There, results near 1.2e-38 carry up
+// to twice the stated relative error.
 __device__ __forceinline__ uint64_t exp2_poly2(float x0, float x1) {
   const uint64_t x = f2_pack(fmaxf(x0, -126.0f), fmaxf(x1, -126.0f));
   const uint64_t magic = f2_pack(12582912.0f, 12582912.0f);
