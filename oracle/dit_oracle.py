@@ -18,10 +18,15 @@ Sources (web pages, cited by title and section):
         the two block lists (double-stream "transformer_blocks" and
         single-stream "single_transformer_blocks").  §6.3 fixes the attention
         layout (B, S, H, D).  §2 and §8 give the flowmatch-euler 50-step loop.
+        §5 merges the partial results of ring attention by log-sum-exp; §7
+        skips model steps (MeanCache) with a finite-difference prediction.
   [WAN] Wan2.1 local-acceleration page (mhpq.cn), §1.1: video DiT blocks are
         dominated by self-attention over long (t, h, w) token sequences.
+  [SDXL] SDXL inference-optimisation guide (javey-q.github.io), §3.3:
+        classifier-free guidance, noise_u + scale (noise_c - noise_u) as batch 2,
+        switched off for the late steps.
 Where the pages leave a step open, the reading taken is stated at the function
-and collected in the design notes (readings s1-s13).
+and collected in the design notes (readings s1-s15).
 
 Parity status: every function below is pinned by tests in tests/test_oracle_*.py
 against invariants, closed forms or brute force; none is "parity unpinned".
@@ -374,16 +379,24 @@ def flux_velocity(img_tok, txt_raw, t, ids, model, n_heads, axes_dim=(16, 56, 56
 
 
 def euler_sample(latent, txt_raw, ids, model, n_heads, steps, axes_dim=(16, 56, 56),
-                 theta=10000.0, eps=1e-6, fresh=None, cache_order=1):
+                 theta=10000.0, eps=1e-6, fresh=None, cache_order=1, txt_uncond=None, guidance=1.0,
+                 cfg_steps=None):
     """Flow-match Euler over the linear schedule t_i = 1 - i/steps:
     x <- x + (t_{i+1} - t_i) v(x, t_i).  Returns the final latent [C, H, W]
-    (reading s9: no resolution shift, no guidance).
+    (reading s9: no resolution shift, no guidance embedding).
 
     Model-level step cache ([CG] §7): fresh[i] = 1 runs the model at step i;
     fresh[i] = 0 predicts the velocity from the model velocities of earlier
     fresh steps.  cache_order 0 reuses the last one; 1 extrapolates linearly
     in t from the last two (a finite-difference estimate of dv/dt), using the
-    last one alone while only one exists."""
+    last one alone while only one exists.
+
+    Classifier-free guidance (the SDXL inference-optimisation guide
+    (javey-q.github.io) §3.3, read for the flow-matching velocity): with
+    txt_uncond, a model step evaluates the velocity for both texts and uses
+    v = v_u + guidance (v_c - v_u).  cfg_steps limits guidance to the first
+    cfg_steps steps (the guide's late-step cut-off); later steps use v_c
+    alone.  Cached steps predict from the guided velocities."""
     C, Hh, Ww = latent.shape
     x = patchify(np.asarray(latent, dtype=np.float64))
     hist = []  # (t, v) of fresh steps, newest last
@@ -392,6 +405,9 @@ def euler_sample(latent, txt_raw, ids, model, n_heads, steps, axes_dim=(16, 56, 
         t1 = 1.0 - (i + 1) / steps
         if fresh is None or fresh[i]:
             v = flux_velocity(x, txt_raw, t0, ids, model, n_heads, axes_dim, theta, eps)
+            if txt_uncond is not None and (cfg_steps is None or i < cfg_steps):
+                vu = flux_velocity(x, txt_uncond, t0, ids, model, n_heads, axes_dim, theta, eps)
+                v = vu + guidance * (v - vu)
             hist.append((t0, v))
         else:
             ta, va = hist[-1]

@@ -442,3 +442,32 @@ def test_attention_merge_over_key_splits_is_full_attention():
     np.testing.assert_array_equal(o1, outs[0])
     o2, _ = O.attention_merge([outs[0], outs[1] + 1e6], [lses[0], lses[1] - 1e4])
     np.testing.assert_allclose(o2, outs[0], rtol=1e-12, atol=1e-9)
+
+
+def test_guidance_special_cases_and_bookkeeping():
+    """Classifier-free guidance in the sampler: guidance 1 gives the
+    conditional sampler, guidance 0 the unconditional one, equal texts make
+    the guidance irrelevant, cfg_steps = 0 switches it off; two guided steps
+    rebuilt by hand from four explicit model calls."""
+    ls = _tiny_loop()
+    m = synth.to_f64(synth.model_weights(ls))
+    inp = synth.to_f64(synth.loop_inputs(ls))
+    lat, txt, ids, H = inp["latent"], inp["txt"], inp["ids"], ls.block.H
+    unc = rng(77).standard_normal(txt.shape)
+    cond = O.euler_sample(lat, txt, ids, m, H, ls.steps)
+    unco = O.euler_sample(lat, unc, ids, m, H, ls.steps)
+    close = dict(rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(O.euler_sample(lat, txt, ids, m, H, ls.steps, txt_uncond=unc, guidance=1.0), cond, **close)
+    np.testing.assert_allclose(O.euler_sample(lat, txt, ids, m, H, ls.steps, txt_uncond=unc, guidance=0.0), unco, **close)
+    np.testing.assert_allclose(O.euler_sample(lat, txt, ids, m, H, ls.steps, txt_uncond=txt, guidance=4.0), cond, **close)
+    np.testing.assert_allclose(O.euler_sample(lat, txt, ids, m, H, ls.steps, txt_uncond=unc, guidance=4.0,
+                                              cfg_steps=0), cond, **close)
+    g = 3.5
+    x0 = O.patchify(lat)
+    v0 = O.flux_velocity(x0, unc, 1.0, ids, m, H)
+    v0 = v0 + g * (O.flux_velocity(x0, txt, 1.0, ids, m, H) - v0)
+    x1 = x0 - v0 / 2
+    v1 = O.flux_velocity(x1, txt, 0.5, ids, m, H)  # guidance only for the first step (cfg_steps = 1)
+    x2 = x1 - v1 / 2
+    got = O.euler_sample(lat, txt, ids, m, H, 2, txt_uncond=unc, guidance=g, cfg_steps=1)
+    np.testing.assert_allclose(got, O.unpatchify(x2, 2, 2, 3), **close)
