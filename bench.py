@@ -630,7 +630,11 @@ def run_loop(args):
     ids = torch.from_numpy(synth.flux_ids(S_TXT, GRID, GRID)).to(dev)
     out = torch.empty((ls.channels, 2 * GRID, 2 * GRID), dtype=torch.float32, device=dev)
     fresh = dit.cached_schedule(ls.steps) if args.cache else None
-    io = dit.loop_io(S_TXT, GRID, GRID, ls.steps, lat, txt, ids, out, fresh=fresh, cache_order=1)
+    # classifier-free guidance as the SDXL guide runs it: on for the first 75% of the steps
+    unc = _rand(torch, g, dev, S_TXT, ls.txt_in, std=1.0) if args.cfg else None
+    cfg_steps = (3 * ls.steps) // 4
+    io = dit.loop_io(S_TXT, GRID, GRID, ls.steps, lat, txt, ids, out, fresh=fresh, cache_order=1,
+                     txt_uncond=unc, guidance=3.5, cfg_steps=cfg_steps)
     ws = torch.empty(dit.dit_forward_workspace(model, io), dtype=torch.uint8, device=dev)
     t0 = time.time()
     graph = dit.Graph(model, io, ws)
@@ -646,11 +650,13 @@ def run_loop(args):
     dbl = 2.0 * S * D * (3 * D + D + 2 * M) + 4.0 * S * S * H * 128 + 2 * 2.0 * D * 6 * D
     emb = 2.0 * (S_TXT * ls.txt_in * D + (S - S_TXT) * F * D + ls.t_dim * D + D * D) + 2.0 * D * 2 * D \
         + 2.0 * (S - S_TXT) * D * F
-    n_fwd = sum(fresh) if fresh is not None else ls.steps
+    fresh_steps = [i for i in range(ls.steps) if fresh is None or fresh[i]]
+    n_fwd = len(fresh_steps) + (sum(1 for i in fresh_steps if i < cfg_steps) if args.cfg else 0)
     flops = n_fwd * (ls.n_double * dbl + ls.n_single * single + emb)
     n_nodes = graph.nodes()
     graph.destroy()
-    name = ls.name + ("_step_cache_%dfresh" % n_fwd if fresh is not None else "") + "_one_cuda_graph"
+    name = (ls.name + ("_step_cache" if fresh is not None else "") + ("_cfg%dof%d" % (cfg_steps, ls.steps) if args.cfg
+            else "") + "_%dforwards_one_cuda_graph" % n_fwd)
     return _extra_line(name, ms, flops, K, W,
                        {"s_per_image": round(ms / 1e3, 3), "graph_nodes": n_nodes, "model_forwards": n_fwd,
                         "graph_build_s": round(t_build, 2), "graph_launches_per_image": 1})
@@ -754,6 +760,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cache", action="store_true",
                     help="loop workload: model-level step cache (26 model forwards for 50 steps)")
+    ap.add_argument("--cfg", action="store_true",
+                    help="loop workload: classifier-free guidance on the first 75%% of the steps")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -97,7 +97,8 @@ class dit_model(ctypes.Structure):
 class dit_loop_io(ctypes.Structure):
     _fields_ = [("n_txt", i32), ("grid_h", i32), ("grid_w", i32), ("steps", i32),
                 ("latent_in", c_void_p), ("txt", c_void_p), ("ids", c_void_p), ("latent_out", c_void_p),
-                ("fresh", ctypes.POINTER(ctypes.c_uint8)), ("cache_order", i32)]
+                ("fresh", ctypes.POINTER(ctypes.c_uint8)), ("cache_order", i32),
+                ("txt_uncond", c_void_p), ("guidance", f32), ("cfg_steps", i32)]
 
 
 # ----------------------------------------------------------------------------
@@ -416,10 +417,13 @@ class Model:
 
 
 def loop_io(n_txt, grid_h, grid_w, steps, latent_in, txt, ids, latent_out, fresh=None,
-            cache_order=1) -> dit_loop_io:
-    """fresh: optional sequence of 0/1 per step (1 = run the model)."""
+            cache_order=1, txt_uncond=None, guidance=1.0, cfg_steps=-1) -> dit_loop_io:
+    """fresh: optional sequence of 0/1 per step (1 = run the model).
+    txt_uncond: optional unconditional text for classifier-free guidance with
+    scale `guidance` on the first cfg_steps steps (< 0: every step)."""
     io = dit_loop_io(n_txt=n_txt, grid_h=grid_h, grid_w=grid_w, steps=steps, latent_in=_ptr(latent_in),
-                     txt=_ptr(txt), ids=_ptr(ids), latent_out=_ptr(latent_out), cache_order=cache_order)
+                     txt=_ptr(txt), ids=_ptr(ids), latent_out=_ptr(latent_out), cache_order=cache_order,
+                     txt_uncond=_ptr(txt_uncond), guidance=float(guidance), cfg_steps=int(cfg_steps))
     if fresh is not None:
         arr = (ctypes.c_uint8 * steps)(*[1 if f else 0 for f in fresh])
         io._fresh_keep = arr

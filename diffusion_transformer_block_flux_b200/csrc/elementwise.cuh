@@ -809,12 +809,18 @@ __global__ void unpatchify_kernel(const float* __restrict__ state, int C, int Hg
 
 // x += (t_{i+1} - t_i) v, state fp32; also refresh the bf16 copy fed to img_in.
 // vhist (optional): keep the model velocity of this step for the step cache.
+// vu != null: classifier-free guidance, v = vu + g (v - vu) in fp32.
 __global__ void euler_kernel(float* __restrict__ state, bf16* __restrict__ tok, const bf16* __restrict__ v,
-                             int64_t n, const float* __restrict__ tsched, int step, float* __restrict__ vhist) {
+                             int64_t n, const float* __restrict__ tsched, int step, float* __restrict__ vhist,
+                             const bf16* __restrict__ vu = nullptr, float g = 1.0f) {
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= n) return;
   const float dt = tsched[step + 1] - tsched[step];
-  const float vi = __bfloat162float(v[i]);
+  float vi = __bfloat162float(v[i]);
+  if (vu != nullptr) {
+    const float u = __bfloat162float(vu[i]);
+    vi = fmaf(g, vi - u, u);
+  }
   if (vhist != nullptr) vhist[i] = vi;
   const float s = fmaf(dt, vi, state[i]);
   state[i] = s;

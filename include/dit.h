@@ -12,6 +12,8 @@
  *         buffers, fixed shapes and addresses, no host sync, no allocation.
  *   [WAN] Wan2.1 local-acceleration page (mhpq.cn), §1.1: video DiT blocks over
  *         long (t, h, w) token sequences, dominated by self-attention.
+ *   [SDXL] SDXL inference-optimisation guide (javey-q.github.io), §3.3:
+ *         classifier-free guidance and its late-step cut-off.
  *
  * Conventions shared by every call
  *   - dit_bf16 is the raw bit pattern of a bfloat16 value.
@@ -420,6 +422,16 @@ typedef struct {
    * (the last one alone until two exist).  Read at graph creation. */
   const uint8_t* fresh;
   int cache_order;
+  /* Classifier-free guidance ([SDXL] §3.3: v = v_u + g (v_c - v_u), read for
+   * the flow-matching velocity).  txt_uncond: NULL = no guidance; otherwise a
+   * device bf16 [n_txt][txt_dim] unconditional text.  A guided step runs the
+   * model once with txt and once with txt_uncond (same timestep embedding and
+   * modulation) and combines the two velocities in fp32.  cfg_steps: guidance
+   * on steps < cfg_steps only (the guide's late-step cut-off); < 0 = every
+   * step.  Cached steps predict from the guided velocities. */
+  const dit_bf16* txt_uncond;
+  float guidance;
+  int cfg_steps;
 } dit_loop_io;
 
 typedef struct dit_graph dit_graph;

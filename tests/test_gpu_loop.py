@@ -23,21 +23,43 @@ def cuda():
     torch.cuda.synchronize()
 
 
-def setup_loop(ls, seed=0, fresh=None, cache_order=1):
+def _scale_modulation(mw, k):
+    """Every block's adaLN weight times k (exact in bf16 for a power of two)."""
+    sc = lambda a: synth.f32_to_bf16_bits(synth.bf16_bits_to_f32(a) * np.float32(k))
+    for blk in mw["double"]:
+        for st in ("txt", "img"):
+            blk[st]["W_mod"] = sc(blk[st]["W_mod"])
+    for blk in mw["single"]:
+        blk["W_mod"] = sc(blk["W_mod"])
+    return mw
+
+
+def setup_loop(ls, seed=0, fresh=None, cache_order=1, guidance=None, cfg_steps=-1, mod_scale=1):
+    """guidance: None = no classifier-free guidance; otherwise the scale, with
+    a seeded unconditional text inp["txt_uncond"] of the text's shape.
+    mod_scale: multiplies every block's adaLN weight (larger gates give the
+    text a visible effect on the image velocity)."""
     import torch
     b = ls.block
     mw = synth.model_weights(ls, seed=seed)
+    if mod_scale != 1:
+        mw = _scale_modulation(mw, mod_scale)
     inp = synth.loop_inputs(ls, seed=seed + 1)
     mdev = dev_tree(mw)
     model = dit.Model(mdev, D=b.D, H=b.H, M=b.M, channels=ls.channels, txt_dim=ls.txt_in, t_dim=ls.t_dim)
     lat_in = dev_bf16(inp["latent"])
     txt = dev_bf16(inp["txt"])
+    unc = None
+    if guidance is not None:
+        inp["txt_uncond"] = synth.normal_bf16(seed + 2, "txt_uncond", inp["txt"].shape)
+        unc = dev_bf16(inp["txt_uncond"])
     ids = torch.from_numpy(inp["ids"]).cuda()
     lat_out = torch.empty(inp["latent"].shape, dtype=torch.float32, device="cuda")
     io = dit.loop_io(b.n_txt, b.grid_h, b.grid_w, ls.steps, lat_in, txt, ids, lat_out, fresh=fresh,
-                     cache_order=cache_order)
+                     cache_order=cache_order, txt_uncond=unc, guidance=1.0 if guidance is None else guidance,
+                     cfg_steps=cfg_steps)
     ws = torch.empty(dit.dit_forward_workspace(model, io), dtype=torch.uint8, device="cuda")
-    keep = (mdev, lat_in, txt, ids)
+    keep = (mdev, lat_in, txt, ids, unc)
     return mw, inp, model, io, ws, lat_out, keep
 
 
@@ -137,5 +159,40 @@ def test_step_cache_matches_oracle_and_graph_equals_eager(order):
     got = eager.cpu().double().numpy()
     parity(got, ref, f"cached loop (order {order})")
     parity(got - f["latent"], ref - f["latent"], f"cached loop displacement (order {order})")
+    st, code = dit.dit_get_device_error()
+    assert st == 0, f"device error word {code:#x}"
+
+
+@pytest.mark.parametrize("cfg_steps,fresh", [(-1, None), (4, None), (-1, [1, 1, 0, 1, 0, 0])])
+def test_guided_loop_matches_oracle_and_graph_equals_eager(cfg_steps, fresh):
+    """Classifier-free guidance (scale 1.5): every step, only the first four
+    steps, and with the step cache predicting from guided velocities.  The
+    adaLN weights are scaled by 32 so that the text moves the image velocity
+    by several percent; the test first checks that the guided and unguided
+    references differ by more than the tolerance, so it can tell them apart."""
+    import torch
+    g = 1.5
+    mw, inp, model, io, ws, lat_out, keep = setup_loop(CACHED, guidance=g, cfg_steps=cfg_steps, fresh=fresh,
+                                                       mod_scale=32)
+    dit.dit_forward_eager(model, io, ws)
+    torch.cuda.synchronize()
+    eager = lat_out.clone()
+    graph = dit.Graph(model, io, ws)
+    lat_out.zero_()
+    graph.launch()
+    torch.cuda.synchronize()
+    assert torch.equal(lat_out, eager)
+    graph.destroy()
+    f = synth.to_f64(inp)
+    ref = O.euler_sample(f["latent"], f["txt"], f["ids"], synth.to_f64(mw), CACHED.block.H, CACHED.steps,
+                         fresh=fresh, txt_uncond=f["txt_uncond"], guidance=g,
+                         cfg_steps=None if cfg_steps < 0 else cfg_steps)
+    unguided = O.euler_sample(f["latent"], f["txt"], f["ids"], synth.to_f64(mw), CACHED.block.H, CACHED.steps,
+                              fresh=fresh)
+    d = ref - f["latent"]
+    assert np.linalg.norm(unguided - ref) / np.linalg.norm(d) > 1.4e-2  # guidance is visible
+    got = eager.cpu().double().numpy()
+    parity(got, ref, f"guided loop (cfg_steps {cfg_steps})")
+    parity(got - f["latent"], ref - f["latent"], f"guided loop displacement (cfg_steps {cfg_steps})")
     st, code = dit.dit_get_device_error()
     assert st == 0, f"device error word {code:#x}"
