@@ -108,6 +108,7 @@ class dit_loop_io(ctypes.Structure):
 _SIGS = {
     "dit_status_string": (ctypes.c_char_p, [i32]),
     "dit_version": (i32, []),
+    "dit_abi_struct_size": (size_t, [i32]),
     "dit_last_cuda_error": (ctypes.c_char_p, []),
     "dit_get_device_error": (i32, [c_void_p, ctypes.POINTER(ctypes.c_uint32)]),
     "dit_clear_device_error": (i32, [c_void_p]),

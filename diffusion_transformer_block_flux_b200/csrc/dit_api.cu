@@ -228,6 +228,20 @@ dit_status dit_clear_device_error(void* stream) {
   return DIT_OK;
 }
 
+size_t dit_abi_struct_size(int which) {
+  switch (which) {
+    case 0: return sizeof(dit_gemm_args);
+    case 1: return sizeof(dit_block_cfg);
+    case 2: return sizeof(dit_single_weights);
+    case 3: return sizeof(dit_stream_weights);
+    case 4: return sizeof(dit_double_weights);
+    case 5: return sizeof(dit_video_weights);
+    case 6: return sizeof(dit_model);
+    case 7: return sizeof(dit_loop_io);
+    default: return 0;
+  }
+}
+
 dit_status dit_set_wait_limit_ns(uint64_t limit_ns) {
   if (limit_ns == 0) return DIT_ERR_INVALID_ARG;
   g_wait_limit_ns = limit_ns;

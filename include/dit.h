@@ -434,6 +434,13 @@ typedef struct {
   int cfg_steps;
 } dit_loop_io;
 
+/* Size in bytes of each struct of this header as the library was compiled,
+ * for a binding to check its own layout: which = 0 dit_gemm_args,
+ * 1 dit_block_cfg, 2 dit_single_weights, 3 dit_stream_weights,
+ * 4 dit_double_weights, 5 dit_video_weights, 6 dit_model, 7 dit_loop_io;
+ * 0 for any other value.  Host only: needs no GPU. */
+size_t dit_abi_struct_size(int which);
+
 typedef struct dit_graph dit_graph;
 
 size_t dit_forward_workspace(const dit_model* m, const dit_loop_io* io);

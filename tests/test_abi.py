@@ -82,3 +82,15 @@ def test_host_pipeline_validation(L):
     assert f(ctypes.byref(cfg), ctypes.byref(w), 1, one, nul, one, 16, 256, need, None) == dit.DIT_ERR_INVALID_ARG
     assert f(ctypes.byref(cfg), ctypes.byref(w), 1, one, one, one, 16, 256, need - 1, None) == dit.DIT_ERR_WORKSPACE
     assert f(ctypes.byref(cfg), ctypes.byref(w), 1, one, one, one, 16, 264, need, None) == dit.DIT_ERR_ALIGNMENT
+
+
+def test_binding_struct_layouts_match_the_library(L):
+    """Every ctypes struct of the binding has the size the library was
+    compiled with (a field added to the header but not to the binding, or
+    the other way round, fails here)."""
+    structs = [dit.dit_gemm_args, dit.dit_block_cfg, dit.dit_single_weights, dit.dit_stream_weights,
+               dit.dit_double_weights, dit.dit_video_weights, dit.dit_model, dit.dit_loop_io]
+    for i, st in enumerate(structs):
+        assert L.dit_abi_struct_size(i) == ctypes.sizeof(st), (st.__name__, L.dit_abi_struct_size(i),
+                                                               ctypes.sizeof(st))
+    assert L.dit_abi_struct_size(len(structs)) == 0
