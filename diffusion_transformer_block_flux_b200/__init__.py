@@ -109,6 +109,9 @@ _SIGS = {
     "dit_status_string": (ctypes.c_char_p, [i32]),
     "dit_version": (i32, []),
     "dit_abi_struct_size": (size_t, [i32]),
+    "dit_step_cache_plan": (i32, [i32, ctypes.POINTER(ctypes.c_uint8), i32, ctypes.POINTER(i32),
+                                  ctypes.POINTER(i32), ctypes.POINTER(i32), ctypes.POINTER(f32),
+                                  ctypes.POINTER(f32)]),
     "dit_last_cuda_error": (ctypes.c_char_p, []),
     "dit_get_device_error": (i32, [c_void_p, ctypes.POINTER(ctypes.c_uint32)]),
     "dit_clear_device_error": (i32, [c_void_p]),
@@ -430,6 +433,17 @@ def loop_io(n_txt, grid_h, grid_w, steps, latent_in, txt, ids, latent_out, fresh
         io._fresh_keep = arr
         io.fresh = ctypes.cast(arr, ctypes.POINTER(ctypes.c_uint8))
     return io
+
+
+def dit_step_cache_plan(steps: int, fresh, cache_order: int = 1) -> dict:
+    """The loop's step-cache plan (host only): per step the kept history slot,
+    or for a predicted step the slots and coefficients of v = ca v_a + cb v_b."""
+    fr = None if fresh is None else (ctypes.c_uint8 * steps)(*[1 if f else 0 for f in fresh])
+    arrs = {k: (i32 * steps)() for k in ("keep_slot", "slot_a", "slot_b")}
+    arrs.update({k: (f32 * steps)() for k in ("ca", "cb")})
+    _call("dit_step_cache_plan", steps, fr, cache_order, arrs["keep_slot"], arrs["slot_a"], arrs["slot_b"],
+          arrs["ca"], arrs["cb"])
+    return {k: list(v) for k, v in arrs.items()}
 
 
 def cached_schedule(steps: int) -> list:

@@ -441,6 +441,22 @@ typedef struct {
  * 0 for any other value.  Host only: needs no GPU. */
 size_t dit_abi_struct_size(int which);
 
+/* Host-side plan of the model-level step cache for `steps` Euler steps (the
+ * bookkeeping dit_forward_* follows, exposed so a caller can inspect it and so
+ * it can be checked without a GPU).  Per step i, arrays of length steps:
+ *   keep_slot[i] >= 0: the model runs and its velocity is kept in history
+ *     slot keep_slot[i] (0 or 1); -1 on a predicted step, and on every step
+ *     when fresh == NULL (no cache).
+ *   on a predicted step (fresh[i] == 0) the velocity is
+ *     ca[i] * v[slot_a[i]] + cb[i] * v[slot_b[i]]  (slot_b[i] = -1: one term);
+ *     ca, cb follow v = v_a + (t_i - t_a)(v_a - v_b)/(t_a - t_b) for order 1
+ *     with the two newest fresh steps a, b, and v = v_a otherwise.
+ *     slot_a, slot_b, ca, cb are -1, -1, 0, 0 on steps that run the model.
+ * Same validation as dit_forward_*: fresh[0] must be 1, cache_order 0 or 1.
+ * Host only: needs no GPU. */
+dit_status dit_step_cache_plan(int steps, const uint8_t* fresh, int cache_order, int* keep_slot, int* slot_a,
+                               int* slot_b, float* ca, float* cb);
+
 typedef struct dit_graph dit_graph;
 
 size_t dit_forward_workspace(const dit_model* m, const dit_loop_io* io);

@@ -94,3 +94,45 @@ def test_binding_struct_layouts_match_the_library(L):
         assert L.dit_abi_struct_size(i) == ctypes.sizeof(st), (st.__name__, L.dit_abi_struct_size(i),
                                                                ctypes.sizeof(st))
     assert L.dit_abi_struct_size(len(structs)) == 0
+
+
+@pytest.mark.parametrize("order", [0, 1])
+@pytest.mark.parametrize("fresh", [[1, 1, 0, 1, 0, 0], [1, 0, 0, 1, 0], [1] * 5, "cached50"])
+def test_step_cache_plan_follows_the_definition(L, order, fresh):
+    """The loop's host bookkeeping of the step cache: a predicted step reads the
+    kept velocities of the two newest fresh steps a (newest) and b, with
+    v = v_a + (t - t_a)(v_a - v_b)/(t_a - t_b) for order 1 (v_a alone for
+    order 0 or while only one exists); a fresh step keeps its velocity in the
+    slot not holding the newest one."""
+    if fresh == "cached50":
+        fresh = dit.cached_schedule(50)
+    n = len(fresh)
+    p = dit.dit_step_cache_plan(n, fresh, order)
+    t = [1.0 - i / n for i in range(n)]
+    done = []  # fresh steps so far
+    for i in range(n):
+        if fresh[i]:
+            assert p["keep_slot"][i] in (0, 1) and p["slot_a"][i] == -1 and p["slot_b"][i] == -1
+            if done:
+                assert p["keep_slot"][i] != p["keep_slot"][done[-1]]  # the newest stays readable
+            done.append(i)
+            continue
+        a = done[-1]
+        assert p["keep_slot"][i] == -1 and p["slot_a"][i] == p["keep_slot"][a]
+        if order == 1 and len(done) >= 2:
+            b = done[-2]
+            r = (t[i] - t[a]) / (t[a] - t[b])
+            assert p["slot_b"][i] == p["keep_slot"][b]
+            assert abs(p["ca"][i] - (1 + r)) <= 1e-6 * abs(1 + r) and abs(p["cb"][i] + r) <= 1e-6 * abs(r)
+        else:
+            assert p["slot_b"][i] == -1 and p["ca"][i] == 1.0 and p["cb"][i] == 0.0
+
+
+def test_step_cache_plan_without_cache_and_validation(L):
+    p = dit.dit_step_cache_plan(4, None, 1)
+    assert p["keep_slot"] == [-1] * 4 and p["slot_a"] == [-1] * 4
+    bad = (ctypes.c_uint8 * 3)(0, 1, 1)
+    i3 = (ctypes.c_int * 3)()
+    f3 = (ctypes.c_float * 3)()
+    assert L.dit_step_cache_plan(3, bad, 1, i3, i3, i3, f3, f3) == dit.DIT_ERR_INVALID_ARG
+    assert L.dit_step_cache_plan(3, None, 2, i3, i3, i3, f3, f3) == dit.DIT_ERR_INVALID_ARG
