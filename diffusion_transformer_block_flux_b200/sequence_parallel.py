@@ -57,7 +57,10 @@ def ring_attention(q, k, v, out, H, group=None, attn=None, merge=None):
     for hop in range(N):
         reqs = []
         if hop < N - 1:
-            reqs = [dist.isend(kv, nxt, group=group), dist.irecv(buf, prv, group=group)]
+            # one group for the send and the receive: with NCCL, separate calls
+            # would queue every rank's send ahead of its receive and wait in a cycle
+            reqs = dist.batch_isend_irecv([dist.P2POp(dist.isend, kv, nxt, group),
+                                           dist.P2POp(dist.irecv, buf, prv, group)])
         if hop == 0:
             attn(q, kv[0], kv[1], out, lse, H)
         else:
