@@ -136,3 +136,48 @@ def test_step_cache_plan_without_cache_and_validation(L):
     f3 = (ctypes.c_float * 3)()
     assert L.dit_step_cache_plan(3, bad, 1, i3, i3, i3, f3, f3) == dit.DIT_ERR_INVALID_ARG
     assert L.dit_step_cache_plan(3, None, 2, i3, i3, i3, f3, f3) == dit.DIT_ERR_INVALID_ARG
+
+
+def _fake_model(nd, ns, D=256, H=2, M=512):
+    """A dit_model of placeholder (never dereferenced) pointers: enough for the
+    host-side validation and workspace query."""
+    P = 256
+    dbl = (dit.dit_double_weights * max(nd, 1))(*[dit.dit_double_weights(
+        txt=dit.dit_stream_weights(*([P] * 12)), img=dit.dit_stream_weights(*([P] * 12))) for _ in range(nd)])
+    sgl = (dit.dit_single_weights * max(ns, 1))(*[dit.dit_single_weights(*([P] * 8)) for _ in range(ns)])
+    m = dit.dit_model(D=D, H=H, head_dim=128, M=M, channels=16, txt_dim=64, t_dim=256, n_double=nd, n_single=ns,
+                      double_blocks=ctypes.cast(dbl, ctypes.POINTER(dit.dit_double_weights)),
+                      single_blocks=ctypes.cast(sgl, ctypes.POINTER(dit.dit_single_weights)), eps=1e-6,
+                      **{k: P for k in ("W_img_in", "b_img_in", "W_txt_in", "b_txt_in", "W_t1", "b_t1", "W_t2",
+                                        "b_t2", "W_fmod", "b_fmod", "W_out", "b_out")})
+    m._keep = (dbl, sgl)
+    return m
+
+
+def _fake_io(steps=6, **kw):
+    io = dit.dit_loop_io(n_txt=16, grid_h=4, grid_w=6, steps=steps, latent_in=256, txt=256, ids=256, latent_out=256,
+                         cache_order=1, guidance=1.0, cfg_steps=-1)
+    for k, v in kw.items():
+        setattr(io, k, v)
+    return io
+
+
+def test_loop_workspace_query_validates_on_the_host(L):
+    m = _fake_model(2, 2)
+    ws = L.dit_forward_workspace(ctypes.byref(m), ctypes.byref(_fake_io()))
+    assert ws > 0
+    # the per-step modulation buffer (every block's vectors, fp32) is part of it
+    m0 = _fake_model(0, 0)
+    ws0 = L.dit_forward_workspace(ctypes.byref(m0), ctypes.byref(_fake_io()))
+    assert ws - ws0 >= 4 * 256 * (12 * 2 + 3 * 2)
+    # guidance: an unconditional text with a finite scale is fine, a NaN scale is not
+    assert L.dit_forward_workspace(ctypes.byref(m), ctypes.byref(_fake_io(txt_uncond=256, guidance=3.0))) == ws
+    assert L.dit_forward_workspace(ctypes.byref(m), ctypes.byref(_fake_io(txt_uncond=256,
+                                                                          guidance=float("nan")))) == 0
+    # step cache: the first step must run the model; orders 0 and 1 only
+    bad = (ctypes.c_uint8 * 6)(0, 1, 1, 1, 1, 1)
+    assert L.dit_forward_workspace(ctypes.byref(m), ctypes.byref(_fake_io(
+        fresh=ctypes.cast(bad, ctypes.POINTER(ctypes.c_uint8))))) == 0
+    assert L.dit_forward_workspace(ctypes.byref(m), ctypes.byref(_fake_io(cache_order=2))) == 0
+    assert L.dit_forward_workspace(ctypes.byref(m), ctypes.byref(_fake_io(steps=0))) == 0
+    assert L.dit_forward_workspace(ctypes.byref(m), ctypes.byref(_fake_io(txt=None))) == 0
