@@ -181,3 +181,20 @@ def test_loop_workspace_query_validates_on_the_host(L):
     assert L.dit_forward_workspace(ctypes.byref(m), ctypes.byref(_fake_io(cache_order=2))) == 0
     assert L.dit_forward_workspace(ctypes.byref(m), ctypes.byref(_fake_io(steps=0))) == 0
     assert L.dit_forward_workspace(ctypes.byref(m), ctypes.byref(_fake_io(txt=None))) == 0
+
+
+def test_new_entry_points_reject_bad_arguments_on_the_host(L):
+    p = ctypes.c_void_p(256)
+    one = (ctypes.c_void_p * 1)(256)
+    nine = (ctypes.c_void_p * 9)(*([256] * 9))
+    # merge: 1..8 parts, heads and batch in range, 16-byte aligned rows
+    assert L.dit_attention_merge(0, one, one, 128, p, None, 128, 1, 4, 1, None) == dit.DIT_ERR_INVALID_ARG
+    assert L.dit_attention_merge(9, nine, nine, 128, p, None, 128, 1, 4, 1, None) == dit.DIT_ERR_INVALID_ARG
+    assert L.dit_attention_merge(1, one, one, 64, p, None, 128, 1, 4, 1, None) == dit.DIT_ERR_SHAPE
+    assert L.dit_attention_merge(1, one, one, 130, p, None, 130, 1, 4, 1, None) == dit.DIT_ERR_ALIGNMENT
+    assert L.dit_attention_merge(1, one, one, 128, ctypes.c_void_p(258), None, 128, 1, 4, 1,
+                                 None) == dit.DIT_ERR_ALIGNMENT
+    assert L.dit_attention_merge(1, one, one, 128, p, None, 128, 70000, 4, 1, None) == dit.DIT_ERR_SHAPE
+    # exp2 self test
+    assert L.dit_selftest_exp2_poly(None, p, 4, None) == dit.DIT_ERR_INVALID_ARG
+    assert L.dit_selftest_exp2_poly(p, p, 0, None) == dit.DIT_ERR_INVALID_ARG
