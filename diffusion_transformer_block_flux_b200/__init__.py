@@ -389,6 +389,14 @@ def dit_single_block_fwd_host(cfg, w: dit_single_weights, xs, vecs, outs, rope, 
     n = len(xs)
     if len(vecs) != n or len(outs) != n:
         raise ValueError("xs, vecs and outs must have the same length")
+    # the copies read and write whole requests: check every host buffer first
+    need = {"x": cfg.B * cfg.S * cfg.D * 2, "vec": cfg.B * cfg.D * 2, "out": cfg.B * cfg.S * cfg.D * 2}
+    for kind, ts in (("x", xs), ("vec", vecs), ("out", outs)):
+        for i, t in enumerate(ts):
+            if t.device.type != "cpu" or not t.is_contiguous():
+                raise ValueError(f"{kind}[{i}] must be a contiguous host tensor")
+            if t.numel() * t.element_size() < need[kind]:
+                raise ValueError(f"{kind}[{i}] holds {t.numel() * t.element_size()} bytes, needs {need[kind]}")
     arr = lambda ts: (c_void_p * n)(*[t.data_ptr() for t in ts])
     _call("dit_single_block_fwd_host", ctypes.byref(cfg), ctypes.byref(w), n, arr(xs), arr(vecs), arr(outs),
           _ptr(rope), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream))

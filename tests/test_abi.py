@@ -198,3 +198,18 @@ def test_new_entry_points_reject_bad_arguments_on_the_host(L):
     # exp2 self test
     assert L.dit_selftest_exp2_poly(None, p, 4, None) == dit.DIT_ERR_INVALID_ARG
     assert L.dit_selftest_exp2_poly(p, p, 0, None) == dit.DIT_ERR_INVALID_ARG
+
+
+def test_host_pipeline_binding_checks_host_buffers(L):
+    import torch
+    cfg = dit.block_cfg(1, 8, 128, 1, 256)
+    w = dit.dit_single_weights(*([256] * 8))
+    ok = torch.empty((8, 128), dtype=torch.bfloat16)
+    v = torch.empty((1, 128), dtype=torch.bfloat16)
+    ws = torch.empty(16, dtype=torch.uint8)
+    with pytest.raises(ValueError, match="same length"):
+        dit.dit_single_block_fwd_host(cfg, w, [ok], [v, v], [ok], None, ws)
+    with pytest.raises(ValueError, match="needs"):
+        dit.dit_single_block_fwd_host(cfg, w, [ok[:4]], [v], [ok], None, ws)
+    with pytest.raises(ValueError, match="contiguous"):
+        dit.dit_single_block_fwd_host(cfg, w, [ok], [v], [torch.empty((128, 8), dtype=torch.bfloat16).t()], None, ws)
