@@ -22,6 +22,13 @@ namespace {
 constexpr int kMaxDevices = 64;
 constexpr int kVecSmemMax = 200 * 1024;  // staged input vectors of dit_vec_linear (B * K fp32)
 constexpr int kRowSmemMax = 200 * 1024;  // bulk-staged row rings (8 warps x 2 rows) + vectors
+// Per-CTA budgets of the tcgen05 kernels: 227 KB of shared memory (dynamic,
+// including the alignment slack each kernel adds) and the 512 TMEM columns.
+static_assert(dit::gemm::SMEM_BYTES <= 227 * 1024, "GEMM shared memory above the per-CTA limit");
+static_assert(dit::gemm::pair::SMEM_BYTES <= 227 * 1024, "pair GEMM shared memory above the per-CTA limit");
+static_assert(dit::attn::SMEM_BYTES <= 227 * 1024, "attention shared memory above the per-CTA limit");
+static_assert(dit::gemm::TMEM_COLS <= 512 && dit::gemm::pair::TMEM_COLS <= 512 && dit::attn::TMEM_COLS <= 512,
+              "TMEM allocation above 512 columns");
 constexpr int kVecPipeSmemMax = 144 * 1024;  // adaLN: 4 warps x 4 weight rows of K <= 4096 bf16 + K fp32
 uint64_t g_wait_limit_ns = 2000000000ull;
 
