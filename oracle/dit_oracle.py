@@ -189,16 +189,24 @@ def attention_merge(outs, lses):
     and lse_j, the attention over the union is
         lse = log sum_j exp(lse_j),  o = sum_j exp(lse_j - lse) o_j.
     outs: list of [Sq, H*d]; lses: list of [H, Sq] (natural log).
-    Returns (o [Sq, H*d], lse [H, Sq])."""
+    Returns (o [Sq, H*d], lse [H, Sq]).
+
+    A part over an empty key set has lse = log 0 = -inf and weight 0.  When
+    every part of a row is empty the union is empty too: lse = -inf and, by
+    the convention of the empty sum, o = 0."""
     n_heads = lses[0].shape[0]
     L = np.stack(lses)                      # [n, H, Sq]
     m = L.max(axis=0)
-    lse = m + np.log(np.exp(L - m).sum(axis=0))
+    empty = np.isneginf(m)
+    ms = np.where(empty, 0.0, m)            # any finite shift: every term is exp(-inf) = 0 there
+    tot = np.exp(L - ms).sum(axis=0)
+    lse = np.where(empty, -np.inf, ms + np.log(np.where(empty, 1.0, tot)))
     Sq = outs[0].shape[0]
     d = outs[0].shape[1] // n_heads
     o = np.zeros((Sq, n_heads, d))
     for oj, lj in zip(outs, lses):
-        o += np.exp(lj - lse).T[:, :, None] * oj.reshape(Sq, n_heads, d)
+        wj = np.where(empty, 0.0, np.exp(lj - np.where(empty, 0.0, lse)))
+        o += wj.T[:, :, None] * oj.reshape(Sq, n_heads, d)
     return o.reshape(Sq, n_heads * d), lse
 
 

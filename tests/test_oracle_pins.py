@@ -442,6 +442,22 @@ def test_attention_merge_over_key_splits_is_full_attention():
     np.testing.assert_array_equal(o1, outs[0])
     o2, _ = O.attention_merge([outs[0], outs[1] + 1e6], [lses[0], lses[1] - 1e4])
     np.testing.assert_allclose(o2, outs[0], rtol=1e-12, atol=1e-9)
+    # an empty key set (lse = log 0 = -inf) carries no weight: merging it changes nothing
+    empty_o, empty_l = np.full_like(outs[0], 5.0), np.full_like(lses[0], -np.inf)
+    o3, l3 = O.attention_merge([outs[0], empty_o, outs[1]], [lses[0], empty_l, lses[1]])
+    o4, l4 = O.attention_merge([outs[0], outs[1]], [lses[0], lses[1]])
+    np.testing.assert_array_equal(o3, o4)
+    np.testing.assert_array_equal(l3, l4)
+    # every part empty: the empty union, o = 0 and lse = -inf (no NaN)
+    o5, l5 = O.attention_merge([empty_o, empty_o], [empty_l, empty_l])
+    assert np.all(o5 == 0) and np.all(np.isneginf(l5))
+    # rows may differ: only the row whose parts are all empty gets the empty result
+    la, lb = lses[0].copy(), lses[1].copy()
+    la[:, 2] = -np.inf
+    lb[:, 2] = -np.inf
+    o6, l6 = O.attention_merge([outs[0], outs[1]], [la, lb])
+    assert np.all(o6[2] == 0) and np.all(np.isneginf(l6[:, 2]))
+    np.testing.assert_array_equal(o6[[0, 1, 3, 4]], o4[[0, 1, 3, 4]])
 
 
 def test_guidance_special_cases_and_bookkeeping():
@@ -471,3 +487,189 @@ def test_guidance_special_cases_and_bookkeeping():
     x2 = x1 - v1 / 2
     got = O.euler_sample(lat, txt, ids, m, H, 2, txt_uncond=unc, guidance=g, cfg_steps=1)
     np.testing.assert_allclose(got, O.unpatchify(x2, 2, 2, 3), **close)
+
+
+# ---------------------------------------------------------------- model forward (flux_velocity)
+
+def _sig(z):
+    """Logistic function written as (1 + tanh(z/2)) / 2: an expression
+    independent of the oracle's z / (1 + e^-z)."""
+    return 0.5 * (1.0 + math.tanh(0.5 * z))
+
+
+def _ln_row(r, eps=1e-6):
+    r = np.asarray(r, dtype=np.float64)
+    return (r - statistics.fmean(r)) / math.sqrt(statistics.pvariance(r) + eps)
+
+
+def _bare_model(D, cin, txt_in, t_dim=256):
+    z = lambda *s: np.zeros(s)
+    return {"W_img_in": z(D, cin), "b_img_in": z(D), "W_txt_in": z(D, txt_in), "b_txt_in": z(D),
+            "W_t1": z(D, t_dim), "b_t1": z(D), "W_t2": z(D, D), "b_t2": z(D),
+            "W_fmod": z(2 * D, D), "b_fmod": z(2 * D), "W_out": z(cin, D), "b_out": z(cin),
+            "double": [], "single": []}
+
+
+def test_flux_velocity_final_layer_order_time_mlp_and_img_in():
+    """One-hot weights route single values through the top level of the model
+    (the compile_graph page's eager forward, §3.1), with no blocks:
+      time path: h = W_t1 emb + b_t1 picks emb[0] = cos(1000 t) (cos half
+        first); vec = W_t2 silu(h) + b_t2 picks silu(h); the final adaLN adds
+        silu(vec) to shift j: two SiLUs in a row;
+      img_in: every image row is tok[t, 0] * u with u = (+1, -1, ...), whose
+        LayerNorm is tok0 u / sqrt(tok0^2 + eps) in closed form;
+      final layer: chunk 0 of W_fmod silu(vec) + b_fmod is the shift and chunk
+        1 the scale: v = ((1 + scale) LN + shift) W_out^T + b_out.
+    A swapped (shift, scale), a missing SiLU, or sin/cos in the other order
+    changes the value."""
+    D, H, C = 256, 2, 2
+    cin, n_txt, gh, gw, tdim = 4 * C, 4, 2, 3, 256
+    r = rng(61)
+    m = _bare_model(D, cin, 16, tdim)
+    u = np.array([1.0 if j % 2 == 0 else -1.0 for j in range(D)])
+    m["W_img_in"][:, 0] = u
+    i0, k, j, j1, f0, f1 = 5, 9, 17, 40, 3, 6
+    m["W_t1"][i0, 0] = 1.0
+    m["W_t2"][k, i0] = 1.0
+    m["W_fmod"][j, k] = 1.0
+    m["b_fmod"] = r.standard_normal(2 * D) * 0.5
+    m["W_out"][f0, j] = 1.0
+    m["W_out"][f1, j1] = 1.0
+    m["b_out"] = r.standard_normal(cin)
+    tok = r.standard_normal((gh * gw, cin))
+    txt = r.standard_normal((n_txt, 16))
+    ids = synth.flux_ids(n_txt, gh, gw)
+    t = 0.37
+    v = O.flux_velocity(tok, txt, t, ids, m, H)
+    assert v.shape == (gh * gw, cin)
+    c = math.cos(1000.0 * t)
+    vec_k = c * _sig(c)
+    s = vec_k * _sig(vec_k)  # silu(silu(cos(1000 t)))
+    sh, sc = m["b_fmod"][:D], m["b_fmod"][D:]
+    for ti in range(gh * gw):
+        a = tok[ti, 0]
+        ln = a * u / math.sqrt(a * a + 1e-6)
+        assert abs(v[ti, f0] - ((1 + sc[j]) * ln[j] + sh[j] + s + m["b_out"][f0])) < 1e-12
+        assert abs(v[ti, f1] - ((1 + sc[j1]) * ln[j1] + sh[j1] + m["b_out"][f1])) < 1e-12
+        for f in range(cin):
+            if f not in (f0, f1):
+                assert v[ti, f] == m["b_out"][f]
+
+
+def test_flux_velocity_text_joins_the_image_through_joint_attention():
+    """One single-stream block whose attention is uniform (q = k = 0) and whose
+    branch is o alone (v = LN(x), W2 = [I | 0], gate 1, scale = shift = 0):
+    every token becomes x_t + mean_s LN(x_s) over the joint sequence, so the
+    image velocity depends on txt_in(txt) through the mean.  Checked against
+    the text and image embeddings written out with their biases, the joint
+    mean over txt | img, and the final layer on the image rows only."""
+    D, H, C = 256, 2, 2
+    cin, n_txt, gh, gw, tin = 4 * C, 5, 2, 3, 16
+    r = rng(62)
+    m = _bare_model(D, cin, tin)
+    m["W_img_in"] = r.standard_normal((D, cin))
+    m["b_img_in"] = r.standard_normal(D)
+    m["W_txt_in"] = r.standard_normal((D, tin)) * 0.3
+    m["b_txt_in"] = r.standard_normal(D)
+    picks = [7, 100, 255, 31, 0, 64, 128, 200]
+    for f, jf in enumerate(picks):
+        m["W_out"][f, jf] = 1.0
+    Mh = 64
+    W1 = np.zeros((3 * D + Mh, D))
+    W1[2 * D:3 * D] = np.eye(D)  # v = y
+    W2 = np.zeros((D, D + Mh))
+    W2[:, :D] = np.eye(D)  # branch = o
+    b_mod = np.concatenate([np.zeros(2 * D), np.ones(D)])  # shift 0, scale 0, gate 1
+    m["single"] = [{"W_mod": np.zeros((3 * D, D)), "b_mod": b_mod, "W1": W1, "b1": np.zeros(3 * D + Mh),
+                    "q_scale": np.ones(128), "k_scale": np.ones(128), "W2": W2, "b2": np.zeros(D)}]
+    tok = r.standard_normal((gh * gw, cin))
+    txt = r.standard_normal((n_txt, tin))
+    ids = synth.flux_ids(n_txt, gh, gw)
+    v = O.flux_velocity(tok, txt, 0.5, ids, m, H)
+    te = [[sum(txt[s, i] * m["W_txt_in"][o, i] for i in range(tin)) + m["b_txt_in"][o] for o in range(D)]
+          for s in range(n_txt)]
+    ie = [[sum(tok[s, i] * m["W_img_in"][o, i] for i in range(cin)) + m["b_img_in"][o] for o in range(D)]
+          for s in range(gh * gw)]
+    lns = [_ln_row(row) for row in te + ie]
+    mean = np.sum(lns, axis=0) / len(lns)
+    for ti in range(gh * gw):
+        y = _ln_row(np.asarray(ie[ti]) + mean)
+        for f, jf in enumerate(picks):
+            assert abs(v[ti, f] - y[jf]) < 1e-10
+    # the text matters: another text gives another image velocity
+    v2 = O.flux_velocity(tok, txt * 2 + 1, 0.5, ids, m, H)
+    assert np.abs(v2 - v).max() > 1e-3
+
+
+def test_flux_velocity_identity_blocks_leave_the_embedding():
+    """Double and single blocks with zero modulation are the identity (gate 0),
+    so the velocity equals that of the same model with no blocks, bit for bit:
+    the double block's (img, txt) outputs go back to the right streams and the
+    image rows are split off the joint sequence after the single blocks."""
+    b = synth.BlockShape("vi", 5, 2, 3, 256, 2, 256)
+    ls = synth.loop_shape(b, 2, 2, 1, channels=2, txt_in=64)
+    m = synth.to_f64(synth.model_weights(ls, bias_std=0.1))
+    zd = synth.to_f64(synth.double_block_weights(b, zero_mod=True, bias_std=0.1))
+    zs = synth.to_f64(synth.single_block_weights(b, zero_mod=True, bias_std=0.1))
+    inp = synth.to_f64(synth.loop_inputs(ls))
+    tok = O.patchify(inp["latent"])
+    bare = dict(m, double=[], single=[])
+    ident = dict(m, double=[zd], single=[zs, zs])  # one double block: a swap of its outputs would stay
+    v0 = O.flux_velocity(tok, inp["txt"], 0.8, inp["ids"], bare, b.H)
+    v1 = O.flux_velocity(tok, inp["txt"], 0.8, inp["ids"], ident, b.H)
+    assert v0.shape == (6, 8)
+    np.testing.assert_array_equal(v0, v1)
+    # the real blocks do change it
+    v2 = O.flux_velocity(tok, inp["txt"], 0.8, inp["ids"], m, b.H)
+    assert np.abs(v2 - v0).max() > 1e-3
+
+
+def test_synth_bias_variant_changes_only_biases_and_scales():
+    s = synth.BlockShape("bv", 4, 2, 2, 256, 2, 256)
+    w0 = synth.single_block_weights(s)
+    w1 = synth.single_block_weights(s, bias_std=0.1, norm_scale_std=0.1)
+    for k in ("W_mod", "W1", "W2"):
+        np.testing.assert_array_equal(w0[k], w1[k])
+    for k in ("b_mod", "b1", "b2"):
+        b = synth.bf16_bits_to_f64(w1[k])
+        assert abs(b.std() - 0.1) < 0.03 and np.count_nonzero(b) > 0.9 * b.size
+    for k in ("q_scale", "k_scale"):
+        sc = synth.bf16_bits_to_f64(w1[k])
+        assert abs(sc.mean() - 1.0) < 0.05 and sc.std() > 0.05
+    zm = synth.single_block_weights(s, zero_mod=True, bias_std=0.1)
+    assert not synth.bf16_bits_to_f64(zm["b_mod"]).any()  # zero modulation stays the identity
+
+
+def test_flux_velocity_image_permutation_equivariance():
+    """Moving image tokens together with their position ids permutes the
+    velocity rows the same way (no mask; RoPE depends on the ids only), for a
+    model with real double and single blocks.  This fails if the blocks ever
+    see a token next to another token's ids (for example image rows placed
+    before the text in the joint sequence while the ids keep text first)."""
+    b = synth.BlockShape("vp", 5, 2, 3, 256, 2, 256)
+    ls = synth.loop_shape(b, 1, 1, 1, channels=2, txt_in=64)
+    m = synth.to_f64(synth.model_weights(ls, bias_std=0.1, norm_scale_std=0.1))
+    m = _scale_mod(m, 8.0)
+    inp = synth.to_f64(synth.loop_inputs(ls))
+    tok = O.patchify(inp["latent"])
+    ids = inp["ids"]
+    perm = np.array([4, 0, 5, 2, 1, 3])
+    ids_p = ids.copy()
+    ids_p[b.n_txt:] = ids[b.n_txt:][perm]
+    v = O.flux_velocity(tok, inp["txt"], 0.6, ids, m, b.H)
+    vp = O.flux_velocity(tok[perm], inp["txt"], 0.6, ids_p, m, b.H)
+    np.testing.assert_allclose(vp, v[perm], rtol=1e-10, atol=1e-12)
+    # and the ids matter: the same permutation of the tokens alone changes the result
+    vq = O.flux_velocity(tok[perm], inp["txt"], 0.6, ids, m, b.H)
+    assert np.abs(vq - v[perm]).max() > 1e-4
+
+
+def _scale_mod(m, k):
+    """Every block's adaLN weight times k: larger gates, so that each block's
+    branch moves its residual stream visibly."""
+    for blk in m["double"]:
+        for st in ("txt", "img"):
+            blk[st]["W_mod"] = blk[st]["W_mod"] * k
+    for blk in m["single"]:
+        blk["W_mod"] = blk["W_mod"] * k
+    return m
