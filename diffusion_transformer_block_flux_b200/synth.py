@@ -5,19 +5,27 @@ It holds none of the block's arithmetic, so both the CUDA path and the CPU
 oracle may consume what it produces.
 
 Distributions follow the workload descriptions: linear weights ~ N(0, 0.02),
-biases 0, RMSNorm scales 1, tokens and conditioning ~ N(0, 1).  Every tensor
+biases 0, RMSNorm scales 1, tokens and conditioning ~ N(0, 1).  A test-only
+variant (bias_std > 0, norm_scale_std > 0) draws every bias from N(0, bias_std)
+and the q/k RMSNorm scales from N(1, norm_scale_std), so that the bias and
+scale wiring of every kernel and block is exercised too.  Every tensor
 gets its own generator seeded from (seed, crc32(name)), so a tensor's values do
 not depend on which other tensors were drawn.  Values are rounded to bf16
 (round-to-nearest-even) and returned as raw uint16 bit patterns.
 """
 from __future__ import annotations
 
+import os
 import zlib
+from concurrent.futures import ThreadPoolExecutor
 from dataclasses import dataclass
 
 import numpy as np
 
 WEIGHT_STD = 0.02
+# the test-only variant: nonzero biases and non-unit q/k norm scales
+TEST_BIAS_STD = 0.1
+TEST_NORM_SCALE_STD = 0.1
 
 
 # --------------------------------------------------------------------------
@@ -26,11 +34,19 @@ WEIGHT_STD = 0.02
 
 
 def f32_to_bf16_bits(a) -> np.ndarray:
-    """Round float32 values to bf16 (nearest-even); return uint16 bits."""
+    """Round float32 values to bf16 (nearest-even); return uint16 bits.
+    In 32-bit integer arithmetic: for every finite value (and +-inf) the sum
+    below stays under 2^32; NaNs map to the canonical quiet NaN."""
     a = np.ascontiguousarray(a, dtype=np.float32)
-    u = a.view(np.uint32).astype(np.uint64)
-    u = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
-    return u.astype(np.uint16)
+    u = a.view(np.uint32)
+    r = u + np.uint32(0x7FFF)
+    r += (u >> np.uint32(16)) & np.uint32(1)
+    r >>= np.uint32(16)
+    out = r.astype(np.uint16)
+    nan = np.isnan(a)
+    if nan.any():
+        out[nan] = 0x7FC0
+    return out
 
 
 def bf16_bits_to_f64(b) -> np.ndarray:
@@ -137,49 +153,57 @@ def _w(seed, name, shape, std=WEIGHT_STD):
     return normal_bf16(seed, name, shape, std)
 
 
+def _b(seed, name, n, bias_std):
+    """A bias: zero in the workload recipe, N(0, bias_std) in the test variant."""
+    return normal_bf16(seed, name, (n,), bias_std) if bias_std > 0 else const_bf16((n,), 0.0)
+
+
+def _s(seed, name, d, norm_scale_std):
+    """An RMSNorm scale: one in the workload recipe, N(1, std) in the test variant."""
+    return normal_bf16(seed, name, (d,), norm_scale_std, 1.0) if norm_scale_std > 0 else const_bf16((d,), 1.0)
+
+
 def single_block_weights(shape: BlockShape, seed: int = 0, prefix: str = "single",
-                         norm_scale_std: float = 0.0, zero_mod: bool = False) -> dict:
+                         norm_scale_std: float = 0.0, zero_mod: bool = False, bias_std: float = 0.0) -> dict:
+    """zero_mod: W_mod and b_mod zero (shift = scale = gate = 0: the block is the identity)."""
     D, M, d = shape.D, shape.M, shape.d
     w = {
         "W_mod": const_bf16((3 * D, D), 0.0) if zero_mod else _w(seed, f"{prefix}.W_mod", (3 * D, D)),
-        "b_mod": const_bf16((3 * D,), 0.0),
+        "b_mod": _b(seed, f"{prefix}.b_mod", 3 * D, 0.0 if zero_mod else bias_std),
         "W1": _w(seed, f"{prefix}.W1", (3 * D + M, D)),
-        "b1": const_bf16((3 * D + M,), 0.0),
+        "b1": _b(seed, f"{prefix}.b1", 3 * D + M, bias_std),
         "W2": _w(seed, f"{prefix}.W2", (D, D + M)),
-        "b2": const_bf16((D,), 0.0),
+        "b2": _b(seed, f"{prefix}.b2", D, bias_std),
     }
     for nm in ("q_scale", "k_scale"):
-        if norm_scale_std > 0:
-            w[nm] = normal_bf16(seed, f"{prefix}.{nm}", (d,), norm_scale_std, 1.0)
-        else:
-            w[nm] = const_bf16((d,), 1.0)
+        w[nm] = _s(seed, f"{prefix}.{nm}", d, norm_scale_std)
     return w
 
 
 def double_block_weights(shape: BlockShape, seed: int = 0, prefix: str = "double",
-                         zero_mod: bool = False) -> dict:
+                         zero_mod: bool = False, bias_std: float = 0.0, norm_scale_std: float = 0.0) -> dict:
     D, M, d = shape.D, shape.M, shape.d
     out = {}
     for s in ("txt", "img"):
         p = f"{prefix}.{s}"
         out[s] = {
             "W_mod": const_bf16((6 * D, D), 0.0) if zero_mod else _w(seed, p + ".W_mod", (6 * D, D)),
-            "b_mod": const_bf16((6 * D,), 0.0),
+            "b_mod": _b(seed, p + ".b_mod", 6 * D, 0.0 if zero_mod else bias_std),
             "W_qkv": _w(seed, p + ".W_qkv", (3 * D, D)),
-            "b_qkv": const_bf16((3 * D,), 0.0),
-            "q_scale": const_bf16((d,), 1.0),
-            "k_scale": const_bf16((d,), 1.0),
+            "b_qkv": _b(seed, p + ".b_qkv", 3 * D, bias_std),
+            "q_scale": _s(seed, p + ".q_scale", d, norm_scale_std),
+            "k_scale": _s(seed, p + ".k_scale", d, norm_scale_std),
             "W_proj": _w(seed, p + ".W_proj", (D, D)),
-            "b_proj": const_bf16((D,), 0.0),
+            "b_proj": _b(seed, p + ".b_proj", D, bias_std),
             "W_mlp1": _w(seed, p + ".W_mlp1", (M, D)),
-            "b_mlp1": const_bf16((M,), 0.0),
+            "b_mlp1": _b(seed, p + ".b_mlp1", M, bias_std),
             "W_mlp2": _w(seed, p + ".W_mlp2", (D, M)),
-            "b_mlp2": const_bf16((D,), 0.0),
+            "b_mlp2": _b(seed, p + ".b_mlp2", D, bias_std),
         }
     return out
 
 
-def video_block_weights(shape: VideoShape, seed: int = 0, prefix: str = "video") -> dict:
+def video_block_weights(shape: VideoShape, seed: int = 0, prefix: str = "video", bias_std: float = 0.0) -> dict:
     D, M = shape.D, shape.M
     names = {
         "W_mod": (6 * D, D), "W_qkv": (3 * D, D), "W_o": (D, D), "W_cq": (D, D),
@@ -188,7 +212,7 @@ def video_block_weights(shape: VideoShape, seed: int = 0, prefix: str = "video")
     w = {}
     for nm, shp in names.items():
         w[nm] = _w(seed, f"{prefix}.{nm}", shp)
-        w["b" + nm[1:]] = const_bf16((shp[0],), 0.0)
+        w["b" + nm[1:]] = _b(seed, f"{prefix}.b{nm[1:]}", shp[0], bias_std)
     return w
 
 
@@ -240,20 +264,26 @@ def loop_shape(block: BlockShape, n_double: int, n_single: int, steps: int,
                      channels, n_double, n_single, steps, txt_in)
 
 
-def model_weights(ls: LoopShape, seed: int = 0) -> dict:
+def model_weights(ls: LoopShape, seed: int = 0, bias_std: float = 0.0, norm_scale_std: float = 0.0) -> dict:
     b = ls.block
     D = b.D
     cin = ls.channels * 4
     m = {
-        "W_img_in": _w(seed, "img_in.W", (D, cin)), "b_img_in": const_bf16((D,), 0.0),
-        "W_txt_in": _w(seed, "txt_in.W", (D, ls.txt_in)), "b_txt_in": const_bf16((D,), 0.0),
-        "W_t1": _w(seed, "time_in.W1", (D, ls.t_dim)), "b_t1": const_bf16((D,), 0.0),
-        "W_t2": _w(seed, "time_in.W2", (D, D)), "b_t2": const_bf16((D,), 0.0),
-        "W_fmod": _w(seed, "final.W_mod", (2 * D, D)), "b_fmod": const_bf16((2 * D,), 0.0),
-        "W_out": _w(seed, "final.W_out", (cin, D)), "b_out": const_bf16((cin,), 0.0),
+        "W_img_in": _w(seed, "img_in.W", (D, cin)), "b_img_in": _b(seed, "img_in.b", D, bias_std),
+        "W_txt_in": _w(seed, "txt_in.W", (D, ls.txt_in)), "b_txt_in": _b(seed, "txt_in.b", D, bias_std),
+        "W_t1": _w(seed, "time_in.W1", (D, ls.t_dim)), "b_t1": _b(seed, "time_in.b1", D, bias_std),
+        "W_t2": _w(seed, "time_in.W2", (D, D)), "b_t2": _b(seed, "time_in.b2", D, bias_std),
+        "W_fmod": _w(seed, "final.W_mod", (2 * D, D)), "b_fmod": _b(seed, "final.b_mod", 2 * D, bias_std),
+        "W_out": _w(seed, "final.W_out", (cin, D)), "b_out": _b(seed, "final.b_out", cin, bias_std),
     }
-    m["double"] = [double_block_weights(b, seed, prefix=f"double{i}") for i in range(ls.n_double)]
-    m["single"] = [single_block_weights(b, seed, prefix=f"single{i}") for i in range(ls.n_single)]
+    # every tensor has its own stream, so the blocks can be drawn concurrently
+    # (numpy releases the GIL while filling and converting large arrays)
+    with ThreadPoolExecutor(max(1, min(16, os.cpu_count() or 1))) as ex:
+        dbl = ex.map(lambda i: double_block_weights(b, seed, prefix=f"double{i}", bias_std=bias_std,
+                                                    norm_scale_std=norm_scale_std), range(ls.n_double))
+        sgl = ex.map(lambda i: single_block_weights(b, seed, prefix=f"single{i}", bias_std=bias_std,
+                                                    norm_scale_std=norm_scale_std), range(ls.n_single))
+        m["double"], m["single"] = list(dbl), list(sgl)
     return m
 
 

@@ -59,6 +59,11 @@ def check_out(got, ref, what, small_x):
     parity(got, ref, what, max_abs_frac=BRANCH_MAX_ABS if small_x else 3e-2)
 
 
+# The test-only weight variant: every bias N(0, 0.1), q/k norm scales N(1, 0.1).
+BIAS = dict(bias_std=synth.TEST_BIAS_STD)
+BIAS_NORM = dict(bias_std=synth.TEST_BIAS_STD, norm_scale_std=synth.TEST_NORM_SCALE_STD)
+
+
 def sample_rows(S, n_txt, k, seed=0):
     r = np.random.default_rng(seed)
     fixed = [0, n_txt - 1, n_txt, S - 1] if n_txt > 0 else [0, S - 1]
@@ -82,10 +87,11 @@ def run_single(shape, w_bits, a_bits):
     return x, out
 
 
-@pytest.mark.parametrize("norm_std,small_x", [(0.0, False), (0.1, False), (0.0, True)])
-def test_single_block_tiny(norm_std, small_x):
+@pytest.mark.parametrize("norm_std,small_x,bias", [(0.0, False, 0.0), (0.1, False, 0.0), (0.0, True, 0.0),
+                                                  (0.1, False, 0.1), (0.1, True, 0.1)])
+def test_single_block_tiny(norm_std, small_x, bias):
     s = synth.TINY
-    wb = synth.single_block_weights(s, norm_scale_std=norm_std)
+    wb = synth.single_block_weights(s, norm_scale_std=norm_std, bias_std=bias)
     ab = synth.block_activations(s)
     if small_x:
         ab["x"] = shrink(ab["x"])
@@ -154,12 +160,13 @@ def test_single_block_host_pipeline_equals_device_calls_bitwise(n):
     no_device_error()
 
 
-def test_single_block_batch2_matches_per_sample_oracle():
+@pytest.mark.parametrize("biased", [False, True])
+def test_single_block_batch2_matches_per_sample_oracle(biased):
     """B = 2 (e.g. the two halves of classifier-free guidance): two samples with
     their own tokens and conditioning vectors in one call."""
     import torch
     s = synth.TINY
-    wb = synth.single_block_weights(s)
+    wb = synth.single_block_weights(s, **(BIAS_NORM if biased else {}))
     a0, a1 = synth.block_activations(s, seed=1), synth.block_activations(s, seed=2)
     w = dev_tree(wb)
     x = dev_bf16(np.concatenate([a0["x"], a1["x"]]))
@@ -179,10 +186,11 @@ def test_single_block_batch2_matches_per_sample_oracle():
     no_device_error()
 
 
-def test_double_block_batch2_matches_per_sample_oracle():
+@pytest.mark.parametrize("biased", [False, True])
+def test_double_block_batch2_matches_per_sample_oracle(biased):
     import torch
     s = synth.BlockShape("small_double", 40, 6, 9, 256, 2, 512)
-    wb = synth.double_block_weights(s)
+    wb = synth.double_block_weights(s, **(BIAS_NORM if biased else {}))
     a0, a1 = synth.double_block_activations(s, seed=1), synth.double_block_activations(s, seed=2)
     w = dev_tree(wb)
     img = dev_bf16(np.concatenate([a0["img"], a1["img"]]))
@@ -205,10 +213,10 @@ def test_double_block_batch2_matches_per_sample_oracle():
     no_device_error()
 
 
-@pytest.mark.parametrize("small_x", [False, True])
-def test_single_block_full_shape_sampled_rows(small_x):
+@pytest.mark.parametrize("small_x,biased", [(False, False), (True, False), (False, True), (True, True)])
+def test_single_block_full_shape_sampled_rows(small_x, biased):
     s = synth.FLUX
-    wb = synth.single_block_weights(s)
+    wb = synth.single_block_weights(s, **(BIAS_NORM if biased else {}))
     ab = synth.block_activations(s)
     if small_x:
         ab["x"] = shrink(ab["x"])
@@ -237,10 +245,10 @@ def run_double(shape, w_bits, a_bits):
     return img_o, txt_o
 
 
-@pytest.mark.parametrize("small_x", [False, True])
-def test_double_block_small(small_x):
+@pytest.mark.parametrize("small_x,biased", [(False, False), (True, False), (False, True), (True, True)])
+def test_double_block_small(small_x, biased):
     s = synth.BlockShape("small_double", 40, 6, 9, 256, 2, 512)
-    wb = synth.double_block_weights(s)
+    wb = synth.double_block_weights(s, **(BIAS_NORM if biased else {}))
     ab = synth.double_block_activations(s)
     if small_x:
         ab["img"], ab["txt"] = shrink(ab["img"]), shrink(ab["txt"])
@@ -261,10 +269,10 @@ def test_double_block_zero_modulation_identity_bitwise():
     assert torch.equal(img_o, dev_bf16(ab["img"])) and torch.equal(txt_o, dev_bf16(ab["txt"]))
 
 
-@pytest.mark.parametrize("small_x", [False, True])
-def test_double_block_full_shape_sampled_rows(small_x):
+@pytest.mark.parametrize("small_x,biased", [(False, False), (True, False), (False, True), (True, True)])
+def test_double_block_full_shape_sampled_rows(small_x, biased):
     s = synth.FLUX_DOUBLE
-    wb = synth.double_block_weights(s)
+    wb = synth.double_block_weights(s, **(BIAS_NORM if biased else {}))
     ab = synth.double_block_activations(s)
     if small_x:
         ab["img"], ab["txt"] = shrink(ab["img"]), shrink(ab["txt"])
@@ -296,10 +304,10 @@ def run_video(vs, w_bits, a_bits):
     return out
 
 
-@pytest.mark.parametrize("small_x", [False, True])
-def test_video_block_small_ragged(small_x):
+@pytest.mark.parametrize("small_x,biased", [(False, False), (True, False), (False, True), (True, True)])
+def test_video_block_small_ragged(small_x, biased):
     vs = synth.VideoShape("small_video", 3, 7, 9, 256, 2, 384, 40)  # S = 189: ragged tiles
-    wb = synth.video_block_weights(vs)
+    wb = synth.video_block_weights(vs, **(BIAS if biased else {}))
     ab = synth.video_activations(vs)
     if small_x:
         ab["x"] = shrink(ab["x"])
@@ -311,10 +319,10 @@ def test_video_block_small_ragged(small_x):
     no_device_error()
 
 
-@pytest.mark.parametrize("small_x", [False, True])
-def test_video_block_full_shape_sampled_rows(small_x):
+@pytest.mark.parametrize("small_x,biased", [(False, False), (True, False), (False, True)])
+def test_video_block_full_shape_sampled_rows(small_x, biased):
     vs = synth.VIDEO
-    wb = synth.video_block_weights(vs)
+    wb = synth.video_block_weights(vs, **(BIAS if biased else {}))
     ab = synth.video_activations(vs)
     if small_x:
         ab["x"] = shrink(ab["x"])

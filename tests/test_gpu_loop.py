@@ -34,14 +34,18 @@ def _scale_modulation(mw, k):
     return mw
 
 
-def setup_loop(ls, seed=0, fresh=None, cache_order=1, guidance=None, cfg_steps=-1, mod_scale=1):
+BIAS_NORM = dict(bias_std=synth.TEST_BIAS_STD, norm_scale_std=synth.TEST_NORM_SCALE_STD)
+
+
+def setup_loop(ls, seed=0, fresh=None, cache_order=1, guidance=None, cfg_steps=-1, mod_scale=1, biased=False):
     """guidance: None = no classifier-free guidance; otherwise the scale, with
     a seeded unconditional text inp["txt_uncond"] of the text's shape.
     mod_scale: multiplies every block's adaLN weight (larger gates give the
-    text a visible effect on the image velocity)."""
+    text a visible effect on the image velocity).  biased: the test-only
+    weight variant (every bias N(0, 0.1), q/k norm scales N(1, 0.1))."""
     import torch
     b = ls.block
-    mw = synth.model_weights(ls, seed=seed)
+    mw = synth.model_weights(ls, seed=seed, **(BIAS_NORM if biased else {}))
     if mod_scale != 1:
         mw = _scale_modulation(mw, mod_scale)
     inp = synth.loop_inputs(ls, seed=seed + 1)
@@ -87,9 +91,10 @@ def test_graph_replay_equals_eager_bitwise():
     assert st == 0, f"device error word {code:#x}"
 
 
-def test_loop_matches_oracle_small():
+@pytest.mark.parametrize("biased", [False, True])
+def test_loop_matches_oracle_small(biased):
     import torch
-    mw, inp, model, io, ws, lat_out, keep = setup_loop(SMALL)
+    mw, inp, model, io, ws, lat_out, keep = setup_loop(SMALL, biased=biased)
     g = dit.Graph(model, io, ws)
     g.launch()
     torch.cuda.synchronize()
@@ -102,12 +107,13 @@ def test_loop_matches_oracle_small():
     g.destroy()
 
 
-def test_full_depth_velocity_at_tiny_dims():
+@pytest.mark.parametrize("biased", [False, True])
+def test_full_depth_velocity_at_tiny_dims(biased):
     """19 double + 38 single blocks at dim 384 (S = 64 + 192): one Euler step
     from t=1 to 0 moves the latent by exactly -v(x0, 1), the model forward."""
     import torch
     ls = synth.loop_shape(synth.TINY, 19, 38, 1, channels=16, txt_in=4096)
-    mw, inp, model, io, ws, lat_out, keep = setup_loop(ls)
+    mw, inp, model, io, ws, lat_out, keep = setup_loop(ls, biased=biased)
     dit.dit_forward_eager(model, io, ws)
     torch.cuda.synchronize()
     got = lat_out.cpu().double().numpy()
@@ -138,12 +144,12 @@ def test_step_cache_all_fresh_is_bitwise_the_plain_loop():
     assert torch.equal(plain, lat_out2)
 
 
-@pytest.mark.parametrize("order", [0, 1])
-def test_step_cache_matches_oracle_and_graph_equals_eager(order):
+@pytest.mark.parametrize("order,biased", [(0, False), (1, False), (1, True)])
+def test_step_cache_matches_oracle_and_graph_equals_eager(order, biased):
     """Model-level step cache: steps 2, 4, 5 predicted from kept velocities."""
     import torch
     fresh = [1, 1, 0, 1, 0, 0]
-    mw, inp, model, io, ws, lat_out, keep = setup_loop(CACHED, fresh=fresh, cache_order=order)
+    mw, inp, model, io, ws, lat_out, keep = setup_loop(CACHED, fresh=fresh, cache_order=order, biased=biased)
     dit.dit_forward_eager(model, io, ws)
     torch.cuda.synchronize()
     eager = lat_out.clone()
@@ -163,8 +169,9 @@ def test_step_cache_matches_oracle_and_graph_equals_eager(order):
     assert st == 0, f"device error word {code:#x}"
 
 
-@pytest.mark.parametrize("cfg_steps,fresh", [(-1, None), (4, None), (-1, [1, 1, 0, 1, 0, 0])])
-def test_guided_loop_matches_oracle_and_graph_equals_eager(cfg_steps, fresh):
+@pytest.mark.parametrize("cfg_steps,fresh,biased", [(-1, None, False), (4, None, False),
+                                                    (-1, [1, 1, 0, 1, 0, 0], False), (4, None, True)])
+def test_guided_loop_matches_oracle_and_graph_equals_eager(cfg_steps, fresh, biased):
     """Classifier-free guidance (scale 1.5): every step, only the first four
     steps, and with the step cache predicting from guided velocities.  The
     adaLN weights are scaled by 32 so that the text moves the image velocity
@@ -173,7 +180,7 @@ def test_guided_loop_matches_oracle_and_graph_equals_eager(cfg_steps, fresh):
     import torch
     g = 1.5
     mw, inp, model, io, ws, lat_out, keep = setup_loop(CACHED, guidance=g, cfg_steps=cfg_steps, fresh=fresh,
-                                                       mod_scale=32)
+                                                       mod_scale=32, biased=biased)
     dit.dit_forward_eager(model, io, ws)
     torch.cuda.synchronize()
     eager = lat_out.clone()
@@ -196,3 +203,48 @@ def test_guided_loop_matches_oracle_and_graph_equals_eager(cfg_steps, fresh):
     parity(got - f["latent"], ref - f["latent"], f"guided loop displacement (cfg_steps {cfg_steps})")
     st, code = dit.dit_get_device_error()
     assert st == 0, f"device error word {code:#x}"
+
+
+class _LazyF64Blocks:
+    """A model's block list converted to float64 one block at a time, as the
+    oracle walks it (the float64 copy of every block at once would not fit)."""
+
+    def __init__(self, blocks):
+        self.blocks = blocks
+
+    def __len__(self):
+        return len(self.blocks)
+
+    def __iter__(self):
+        for blk in self.blocks:
+            yield synth.to_f64(blk)
+
+
+def test_full_dim_loop_velocity_matches_oracle():
+    """The loop at the Flux model's width and depth: dim 3072, 24 heads,
+    19 double + 38 single blocks, on a short sequence (64 text + 8 x 8 image
+    tokens, MLP hidden 256 to keep the weights at 12 GB) with the biased weight
+    variant, one Euler step captured as a graph.  Every block's modulation of
+    the step comes from one batched pass over all 77 modulation matrices
+    (K = 3072), the path the full-size loop runs."""
+    import torch
+    b = synth.BlockShape("loop_dim3072", 64, 8, 8, 3072, 24, 256)
+    ls = synth.loop_shape(b, 19, 38, 1, channels=16, txt_in=4096)
+    mw, inp, model, io, ws, lat_out, keep = setup_loop(ls, biased=True)
+    g = dit.Graph(model, io, ws)
+    g.launch()
+    torch.cuda.synchronize()
+    g.destroy()
+    st, code = dit.dit_get_device_error()
+    assert st == 0, f"device error word {code:#x}"
+    got = lat_out.cpu().double().numpy()
+    del model, io, ws, keep
+    torch.cuda.empty_cache()
+    f = synth.to_f64(inp)
+    m64 = {k: synth.to_f64(v) for k, v in mw.items() if k not in ("double", "single")}
+    m64["double"] = _LazyF64Blocks(mw["double"])
+    m64["single"] = _LazyF64Blocks(mw["single"])
+    ref = O.euler_sample(f["latent"], f["txt"], f["ids"], m64, b.H, 1)
+    # the 57-block chain tolerance of test_full_depth_velocity_at_tiny_dims
+    parity(got - f["latent"], ref - f["latent"], "dim-3072 full-depth velocity", rel_l2=2e-2, max_abs_frac=6e-2)
+    parity(got, ref, "dim-3072 full-depth latent")
