@@ -8,6 +8,7 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "attention.cuh"
@@ -32,8 +33,11 @@ static_assert(dit::gemm::TMEM_COLS <= 512 && dit::gemm::pair::TMEM_COLS <= 512 &
 constexpr int kVecPipeSmemMax = 144 * 1024;  // adaLN: 4 warps x 4 weight rows of K <= 4096 bf16 + K fp32
 uint64_t g_wait_limit_ns = 2000000000ull;
 
+// Per-device state, filled once under g_mu.  `init` is published with a
+// release store after every other field is written and read with an acquire
+// load, so a thread that sees it set also sees the fields.
 struct DeviceInfo {
-  bool init = false;
+  std::atomic<bool> init{false};
   bool supported = false;
   int num_sms = 0;
   bool attrs_set = false;
@@ -72,9 +76,9 @@ dit_status device_setup(int* num_sms) {
   DIT_CUDA_CHECK(cudaGetDevice(&dev));
   if (dev < 0 || dev >= kMaxDevices) return DIT_ERR_UNSUPPORTED;
   DeviceInfo& d = g_dev[dev];
-  if (!d.init) {
+  if (!d.init.load(std::memory_order_acquire)) {
     std::lock_guard<std::mutex> lk(g_mu);
-    if (!d.init) {
+    if (!d.init.load(std::memory_order_relaxed)) {
       int major = 0, sms = 0;
       DIT_CUDA_CHECK(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev));
       DIT_CUDA_CHECK(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
@@ -139,7 +143,7 @@ dit_status device_setup(int* num_sms) {
           g_encode = reinterpret_cast<EncodeTiledFn>(fn);
         }
       }
-      d.init = true;
+      d.init.store(true, std::memory_order_release);
     }
   }
   if (!d.supported) return DIT_ERR_UNSUPPORTED;

@@ -58,7 +58,10 @@ dit_status dit_single_block_fwd_noalloc(const dit_block_cfg* cfg, const dit_sing
                                         const dit_bf16* vec, const float* rope, dit_bf16* out, void* stream) {
   if (cfg == nullptr) return DIT_ERR_INVALID_ARG;
   const size_t need = dit_single_block_workspace(cfg);
-  if (need == 0) return DIT_ERR_SHAPE;
+  // An invalid configuration: let the workspace entry point report it, so that
+  // both calls give the same status for the same bad input (its checks come
+  // before any use of the workspace, and it enqueues nothing when they fail).
+  if (need == 0) return dit_single_block_fwd(cfg, w, x, vec, rope, out, nullptr, 0, stream);
   if (need > kScratchBytes) return DIT_ERR_WORKSPACE;  // the block's intermediates do not fit in 16 MiB
   void* scratch = nullptr;
   dit_status s = scratch_address(&scratch);

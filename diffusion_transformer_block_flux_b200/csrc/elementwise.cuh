@@ -534,11 +534,14 @@ __global__ void __launch_bounds__(256) attention_merge_kernel(const __grid_const
   float m = l[0];
 #pragma unroll
   for (int j = 1; j < NP; ++j) m = fmaxf(m, l[j]);
+  // every part of the row over an empty key set (lse = -inf): the union is
+  // empty too, so o = 0 and lse = -inf instead of exp(-inf - -inf) = NaN
+  const bool empty = m == -INFINITY;
   float den = 0.0f;
   float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
   for (int j = 0; j < NP; ++j) {
-    const float wj = (j < p.n) ? __expf(l[j] - m) : 0.0f;
+    const float wj = (j < p.n && !empty) ? __expf(l[j] - m) : 0.0f;
     den += wj;
     acc[0] = fmaf(wj, bf16_lo(u[j].x), acc[0]); acc[1] = fmaf(wj, bf16_hi(u[j].x), acc[1]);
     acc[2] = fmaf(wj, bf16_lo(u[j].y), acc[2]); acc[3] = fmaf(wj, bf16_hi(u[j].y), acc[3]);
@@ -546,13 +549,13 @@ __global__ void __launch_bounds__(256) attention_merge_kernel(const __grid_const
     acc[6] = fmaf(wj, bf16_lo(u[j].w), acc[6]); acc[7] = fmaf(wj, bf16_hi(u[j].w), acc[7]);
   }
   if (valid) {
-    const float inv = 1.0f / den;
+    const float inv = empty ? 0.0f : 1.0f / den;
     *reinterpret_cast<uint4*>(p.out + bs * p.ld_out + col) =
         make_uint4(pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv),
                    pack_bf16x2(acc[4] * inv, acc[5] * inv), pack_bf16x2(acc[6] * inv, acc[7] * inv));
   }
   __syncwarp();
-  if (valid && sub == 0 && p.lse_out != nullptr) p.lse_out[li] = m + __logf(den);
+  if (valid && sub == 0 && p.lse_out != nullptr) p.lse_out[li] = empty ? -INFINITY : m + __logf(den);
 }
 
 // Self test of the FMA-pipe 2^x that the attention softmax uses on a part of

@@ -33,6 +33,12 @@
  *     is enqueued.  A kernel that waits longer than the wait limit (default 2 s)
  *     on an internal barrier records DIT_ERR_TIMEOUT in the device error word,
  *     releases its resources and exits; dit_get_device_error reports it.
+ *   - Per-device state is set up by the first call on each device and kept
+ *     until the process exits: kernel attributes, the driver's tensor-map
+ *     encoder, the host-buffer pipeline's streams and events, and the address
+ *     of the allocation-free call's scratch array.  A device reset
+ *     (cudaDeviceReset) while the library is loaded invalidates that state and
+ *     is not supported.
  */
 #ifndef DIT_H_
 #define DIT_H_
@@ -194,7 +200,10 @@ dit_status dit_attention(const dit_bf16* q, const dit_bf16* k, const dit_bf16* v
  * it) with its fp32 lse [B][H][Sq] from dit_attention.  o: bf16 [B][Sq][ld_out];
  * lse_out: NULL or fp32 [B][H][Sq].  o may equal any o_parts[j] and lse_out
  * any lse_parts[j] (so a ring can merge into its running result).  Weights
- * and sums in fp32; o rounded to bf16 once.  1 <= B, H <= 65535. */
+ * and sums in fp32; o rounded to bf16 once.  1 <= B, H <= 65535.
+ * A part over an empty key set has lse = -inf and weight 0 (its o values must
+ * be finite: they are multiplied by that zero weight).  A row whose every
+ * part is empty gets o = 0 and lse = -inf. */
 dit_status dit_attention_merge(int n, const dit_bf16* const* o_parts, const float* const* lse_parts,
                                int64_t ld_in, dit_bf16* o, float* lse_out, int64_t ld_out,
                                int B, int Sq, int H, void* stream);
@@ -324,9 +333,10 @@ dit_status dit_single_block_fwd_profiled(const dit_block_cfg* cfg, const dit_sin
  * cudaMalloc/cudaFree once running (those calls can synchronise the device).
  * Same inputs and outputs as dit_single_block_fwd, but the intermediates live
  * in a 16 MiB array inside the library that each device keeps until exit.
- *   - Configurations whose workspace (dit_single_block_workspace) exceeds
- *     16 MiB are rejected with DIT_ERR_WORKSPACE (e.g. S=256, D=384 fits;
- *     S=4608, D=3072 does not).
+ *   - A configuration that dit_single_block_fwd rejects gets the same status
+ *     here.  Valid configurations whose workspace (dit_single_block_workspace)
+ *     exceeds 16 MiB are rejected with DIT_ERR_WORKSPACE (e.g. S=256, D=384
+ *     fits; S=4608, D=3072 does not).
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress with that device current); make that first call
  *     before capturing any stream into a graph.

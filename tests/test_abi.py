@@ -213,3 +213,25 @@ def test_host_pipeline_binding_checks_host_buffers(L):
         dit.dit_single_block_fwd_host(cfg, w, [ok[:4]], [v], [ok], None, ws)
     with pytest.raises(ValueError, match="contiguous"):
         dit.dit_single_block_fwd_host(cfg, w, [ok], [v], [torch.empty((128, 8), dtype=torch.bfloat16).t()], None, ws)
+
+
+def test_noalloc_reports_the_same_status_as_the_workspace_call(L):
+    """For a configuration the block rejects, the allocation-free call returns
+    the status the workspace call returns (both checks run on the host before
+    anything is enqueued); a valid but too large configuration is a workspace
+    error."""
+    w = dit.dit_single_block_workspace
+    weights = dit.dit_single_weights()
+    for cfg in (dit.block_cfg(1, 256, 384, 2, 1536),            # D != H * 128
+                dit.block_cfg(1, 256, 384, 3, 1536, eps=float("nan")),
+                dit.block_cfg(0, 256, 384, 3, 1536),
+                dit.block_cfg(1, 256, 384, 3, 100)):              # M not a multiple of 32
+        assert w(cfg) == 0
+        ref = L.dit_single_block_fwd(ctypes.byref(cfg), ctypes.byref(weights), None, None, None, None, None, 0, None)
+        got = L.dit_single_block_fwd_noalloc(ctypes.byref(cfg), ctypes.byref(weights), None, None, None, None, None)
+        assert ref != dit.DIT_OK and got == ref
+    assert L.dit_single_block_fwd_noalloc(None, ctypes.byref(weights), None, None, None, None, None) == \
+        dit.DIT_ERR_INVALID_ARG
+    big = dit.block_cfg(1, 4608, 3072, 24, 12288)
+    assert L.dit_single_block_fwd_noalloc(ctypes.byref(big), ctypes.byref(weights), None, None, None, None,
+                                          None) == dit.DIT_ERR_WORKSPACE

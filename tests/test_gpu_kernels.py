@@ -316,6 +316,39 @@ def test_attention_merge_matches_oracle(n, B, S, H):
     assert_no_device_error()
 
 
+def test_attention_merge_empty_parts():
+    """Parts over empty key sets (lse = -inf): a fully empty part carries no
+    weight, and rows whose every part is empty give o = 0 and lse = -inf
+    rather than NaN, as in the oracle's merge."""
+    import torch
+    B, S, H = 1, 50, 3
+    D = H * 128
+    r = np.random.default_rng(11)
+    parts = [synth.normal_bf16(40 + j, f"e{j}", (S, D)) for j in range(3)]
+    lses = [(r.standard_normal((B, H, S)) * 2.0).astype(np.float32) for _ in range(3)]
+    lses[1][:] = -np.inf  # part 1 covers no keys at all
+    for j in (0, 2):  # rows 7 and 31 of head 1 have no keys in any part
+        lses[j][0, 1, [7, 31]] = -np.inf
+    dp = [dev_bf16(t) for t in parts]
+    dl = [torch.from_numpy(x).cuda() for x in lses]
+    o = torch.empty((S, D), dtype=torch.bfloat16, device="cuda")
+    lo = torch.empty((B, H, S), dtype=torch.float32, device="cuda")
+    dit.dit_attention_merge(dp, dl, o, lo, B, S, H)
+    torch.cuda.synchronize()
+    pf = [synth.bf16_bits_to_f64(t) for t in parts]
+    ref, ref_lse = O.attention_merge(pf, [x[0].astype(np.float64) for x in lses])
+    got = host_f64(o)
+    assert np.all(np.isfinite(got))
+    gl = lo[0].cpu().double().numpy()
+    assert np.array_equal(np.isneginf(gl), np.isneginf(ref_lse))
+    fin = np.isfinite(ref_lse)
+    assert np.abs(gl[fin] - ref_lse[fin]).max() < 1e-5 * max(1.0, np.abs(ref_lse[fin]).max())
+    empty_cols = got[[7, 31]][:, 128:256]
+    assert np.all(empty_cols == 0)
+    parity(got, ref, "merge with empty parts")
+    assert_no_device_error()
+
+
 def test_ring_schedule_on_one_gpu_equals_full_attention():
     """The arithmetic of one rank's ring hops on one GPU: attention of the
     queries against each of 4 key/value shards (uneven tail), merged hop by
