@@ -81,14 +81,53 @@ def peaks():
 REASON_COLS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
 
+def _nvml_handle(torch, dev_index):
+    """NVML handle of the CUDA device, matched by UUID (NVML numbers every GPU
+    of the machine; CUDA only the visible ones)."""
+    import pynvml
+    pynvml.nvmlInit()
+    props = torch.cuda.get_device_properties(dev_index)
+    uuid = str(getattr(props, "uuid", ""))
+    if uuid:
+        try:
+            return pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+        except pynvml.NVMLError:
+            pass
+    return pynvml.nvmlDeviceGetHandleByIndex(dev_index)
+
+
 class ClockSampler:
+    """Read-only sampling of the SM clock (every ~1 ms), power and clock-event
+    reasons (every ~5 ms) through NVML on a background thread, so that even a
+    20 ms timed region holds tens of samples.  Falls back to nvidia-smi at
+    100 ms when NVML is not available.  Changes no GPU setting."""
+
     def __init__(self, index: int):
         self.index = index
-        self.samples = []
-        self.proc = None
+        self.samples = []   # (time, sm_mhz)
+        self.slow = []      # (time, power_w, reason bits)
+        self.max_mhz = None
+        self.mode = None
+        self._stop = threading.Event()
         self.t = None
+        self.proc = None
 
     def start(self):
+        try:
+            import pynvml
+            import torch
+            self.h = _nvml_handle(torch, self.index)
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM))
+            self.bits = {"hw_slowdown": pynvml.nvmlClocksEventReasonHwSlowdown,
+                         "hw_thermal_slowdown": pynvml.nvmlClocksEventReasonHwThermalSlowdown,
+                         "sw_thermal_slowdown": pynvml.nvmlClocksEventReasonSwThermalSlowdown,
+                         "sw_power_cap": pynvml.nvmlClocksEventReasonSwPowerCap}
+            self.mode = "nvml"
+            self.t = threading.Thread(target=self._nvml_loop, daemon=True)
+            self.t.start()
+            return
+        except Exception:
+            self.mode = None
         q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
              "clocks_event_reasons.sw_power_cap")
@@ -99,38 +138,74 @@ class ClockSampler:
         except OSError:
             self.proc = None
             return
-        self.t = threading.Thread(target=self._read, daemon=True)
+        self.mode = "nvidia-smi"
+        self.t = threading.Thread(target=self._smi_loop, daemon=True)
         self.t.start()
 
-    def _read(self):
+    def _nvml_loop(self):
+        import pynvml
+        n = 0
+        while not self._stop.is_set():
+            t = time.time()
+            try:
+                self.samples.append((t, float(pynvml.nvmlDeviceGetClockInfo(self.h, pynvml.NVML_CLOCK_SM))))
+                if n % 5 == 0:
+                    pw = pynvml.nvmlDeviceGetPowerUsage(self.h) / 1000.0
+                    rb = pynvml.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                    self.slow.append((t, pw, rb))
+            except pynvml.NVMLError:
+                pass
+            n += 1
+            time.sleep(0.001)
+
+    def _smi_loop(self):
         for line in self.proc.stdout:
             parts = [p.strip() for p in line.split(",")]
             if len(parts) >= 7:
-                self.samples.append((time.time(), parts))
+                t = time.time()
+                try:
+                    self.samples.append((t, float(parts[0])))
+                    self.max_mhz = float(parts[1])
+                except ValueError:
+                    continue
+                rb = sum(1 << i for i in range(4) if parts[3 + i].lower().startswith("active"))
+                try:
+                    pw = float(parts[2])
+                except ValueError:
+                    pw = None
+                self.slow.append((t, pw, rb))
 
     def stop(self):
+        self._stop.set()
         if self.proc is not None:
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
+        if self.t is not None:
+            self.t.join(timeout=5)
 
     def summary(self, t0, t1):
-        rows = [p for (t, p) in self.samples if t0 - 0.05 <= t <= t1 + 0.05] or [p for (_, p) in self.samples]
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-
-        def num(x):
-            try:
-                return float(x)
-            except ValueError:
-                return None
-        sm = [num(r[0]) for r in rows if num(r[0]) is not None]
+        """Median SM clock over the samples taken in [t0, t1] while the GPU
+        was busy (above 500 MHz), the clock-event reasons seen there, and the
+        largest power drawn."""
+        win = [(t, v) for (t, v) in self.samples if t0 <= t <= t1]
+        slow = [x for x in self.slow if t0 - 0.005 <= x[0] <= t1 + 0.005]
+        if not win:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0, "source": self.mode}
+        sm = [v for (_, v) in win]
         busy = [v for v in sm if v > 500] or sm
-        reasons = sorted({REASON_COLS[i] for r in rows for i in range(4) if r[3 + i].lower().startswith("active")})
-        return {"sm_mhz": statistics.median(busy) if busy else None,
-                "sm_max_mhz": num(rows[0][1]), "reasons": reasons, "samples": len(rows)}
+        reasons = set()
+        for (_, _, rb) in slow:
+            for i, name in enumerate(REASON_COLS):
+                bit = self.bits[name] if self.mode == "nvml" else (1 << i)
+                if rb & bit:
+                    reasons.add(name)
+        pw = [p for (_, p, _) in slow if p is not None]
+        return {"sm_mhz": statistics.median(busy), "sm_min_mhz": min(busy), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(reasons), "samples": len(win), "power_w_max": max(pw) if pw else None,
+                "source": self.mode + (" 1 ms" if self.mode == "nvml" else " 100 ms")}
 
 
 # ----------------------------------------------------------------------------
@@ -222,6 +297,7 @@ def run_ours(args, rank, world, local_rank):
         step()
     t_end.record(stream)
     torch.cuda.synchronize()
+    wallh = time.time()
     # breakdown: K more forwards with an event before and after every kernel
     for i in range(K):
         step(evs[i])
@@ -229,9 +305,10 @@ def run_ours(args, rank, world, local_rank):
     wall1 = time.time()
     if world > 1:
         torch.distributed.barrier()
-    time.sleep(0.2)
+    time.sleep(0.05)
     sampler.stop()
-    clocks = sampler.summary(wall0, wall1)
+    clocks = sampler.summary(wall0, wallh)
+    clocks_breakdown = sampler.summary(wallh, wall1)
     elapsed_ms = t_start.elapsed_time(t_end)
     per_kernel = {k: statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(K))
                   for j, k in enumerate(KERNELS)}
@@ -300,8 +377,11 @@ def run_ours(args, rank, world, local_rank):
     else:
         roof["peak_source"] = "fallback"
     kernels = {}
+    mhz = clocks_breakdown.get("sm_mhz")
     for k in KERNELS:
         ent = {"ms": round(per_kernel[k], 4), "share": round(per_kernel[k] / sum(per_kernel.values()), 4)}
+        if mhz:  # time x median SM clock of the breakdown pass: clock-independent work in cycles
+            ent["mcycles"] = round(per_kernel[k] * 1e-3 * mhz, 4)
         if KERNEL_BOUND[k] == "tensor":
             a = flops[k] / (per_kernel[k] * 1e-3) / 1e12
             ent.update({"tflops": round(a, 1), "frac_of_bf16_peak": round(a / bf16_peak, 4)})
@@ -322,7 +402,7 @@ def run_ours(args, rank, world, local_rank):
         "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "api": "dit_single_block_fwd_host, pinned host buffers",
                 "h2d_bytes_per_step": S * D * 2 + D * 2,
                 "d2h_bytes_per_step": S * D * 2, "steps": Ke},
-        "roofline": roof, "kernels": kernels, "clocks": clocks,
+        "roofline": roof, "kernels": kernels, "clocks": clocks, "clocks_breakdown_pass": clocks_breakdown,
     }
     return res
 
@@ -453,17 +533,30 @@ def run_reference(args):
 # ----------------------------------------------------------------------------
 
 
+_LAST_CLOCKS = {}
+
+
 def _event_time(torch, fn, K, W, stream):
+    """Mean CUDA-event time of fn over K calls after W warm-up calls; the clock
+    record of the timed calls is kept in _LAST_CLOCKS for the JSON line."""
     for _ in range(W):
         fn()
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(torch.cuda.current_device())
+    sampler.start()
+    time.sleep(0.05)
+    t0 = time.time()
     e0.record(stream)
     for _ in range(K):
         fn()
     e1.record(stream)
     torch.cuda.synchronize()
+    t1 = time.time()
+    sampler.stop()
+    _LAST_CLOCKS.clear()
+    _LAST_CLOCKS.update(sampler.summary(t0, t1))
     return e0.elapsed_time(e1) / K
 
 
@@ -477,7 +570,8 @@ def _extra_line(workload, ms, flops, K, W, extra=None):
     res = {"metric": f"{workload} ms & TFLOP/s (bf16)", "value": round(tf, 2), "unit": "TFLOP/s", "n_gpus": 1,
            "steps": K, "warmup": W, "ms_per_step": round(ms, 4), "higher_is_better": True, "dtype": "bf16",
            "data": "synthetic", "config": {"workload": workload},
-           "frac_of_bf16_peak": round(tf / pk["bf16_tflops"], 4), "algorithmic_flops": flops}
+           "frac_of_bf16_peak": round(tf / pk["bf16_tflops"], 4), "algorithmic_flops": flops,
+           "clocks": dict(_LAST_CLOCKS)}
     if extra:
         res.update(extra)
     return res
