@@ -55,8 +55,16 @@ def shrink(bits, e=-6):
 BRANCH_MAX_ABS = 6e-2
 
 
-def check_out(got, ref, what, small_x):
-    parity(got, ref, what, max_abs_frac=BRANCH_MAX_ABS if small_x else 3e-2)
+def check_out(got, ref, what, small_x, resid_roundings=0):
+    parity(got, ref, what, max_abs_frac=BRANCH_MAX_ABS if small_x else 3e-2, resid_roundings=resid_roundings)
+
+
+# The double-stream block stores each stream's residual in bf16 after its
+# attention branch, then adds the MLP branch: one rounding of the residual
+# stream beyond the output's own.  The video block stores it after self and
+# after cross attention: two.
+DOUBLE_RESID = 1
+VIDEO_RESID = 2
 
 
 # The test-only weight variant: every bias N(0, 0.1), q/k norm scales N(1, 0.1).
@@ -208,8 +216,8 @@ def test_double_block_batch2_matches_per_sample_oracle(biased):
     for b, ab in enumerate((a0, a1)):
         f = synth.to_f64(ab)
         ri, rt = O.double_block(f["img"], f["txt"], f["vec"], f["ids"], wf, s.H)
-        parity(gi[b * ni:(b + 1) * ni], ri, f"batch-2 double img, sample {b}")
-        parity(gt[b * s.n_txt:(b + 1) * s.n_txt], rt, f"batch-2 double txt, sample {b}")
+        parity(gi[b * ni:(b + 1) * ni], ri, f"batch-2 double img, sample {b}", resid_roundings=DOUBLE_RESID)
+        parity(gt[b * s.n_txt:(b + 1) * s.n_txt], rt, f"batch-2 double txt, sample {b}", resid_roundings=DOUBLE_RESID)
     no_device_error()
 
 
@@ -255,8 +263,8 @@ def test_double_block_small(small_x, biased):
     img_o, txt_o = run_double(s, wb, ab)
     f = synth.to_f64(ab)
     ref_img, ref_txt = O.double_block(f["img"], f["txt"], f["vec"], f["ids"], synth.to_f64(wb), s.H)
-    check_out(host_f64(img_o), ref_img, "double img", small_x)
-    check_out(host_f64(txt_o), ref_txt, "double txt", small_x)
+    check_out(host_f64(img_o), ref_img, "double img", small_x, DOUBLE_RESID)
+    check_out(host_f64(txt_o), ref_txt, "double txt", small_x, DOUBLE_RESID)
     no_device_error()
 
 
@@ -283,8 +291,8 @@ def test_double_block_full_shape_sampled_rows(small_x, biased):
     f = synth.to_f64(ab)
     ref_img, ref_txt = O.double_block(f["img"], f["txt"], f["vec"], f["ids"], synth.to_f64(wb), s.H,
                                       rows_img=ri, rows_txt=rt)
-    check_out(host_f64(img_o)[ri], ref_img, "full double img", small_x)
-    check_out(host_f64(txt_o)[rt], ref_txt, "full double txt", small_x)
+    check_out(host_f64(img_o)[ri], ref_img, "full double img", small_x, DOUBLE_RESID)
+    check_out(host_f64(txt_o)[rt], ref_txt, "full double txt", small_x, DOUBLE_RESID)
     no_device_error()
 
 
@@ -315,7 +323,7 @@ def test_video_block_small_ragged(small_x, biased):
     f = synth.to_f64(ab)
     ref = O.video_block(f["x"], f["ctx"], f["vec"], f["ids"], synth.to_f64(wb), vs.H)
     got = host_f64(out)
-    check_out(got, ref, "video out", small_x)
+    check_out(got, ref, "video out", small_x, VIDEO_RESID)
     no_device_error()
 
 
@@ -331,5 +339,5 @@ def test_video_block_full_shape_sampled_rows(small_x, biased):
     f = synth.to_f64(ab)
     ref = O.video_block(f["x"], f["ctx"], f["vec"], f["ids"], synth.to_f64(wb), vs.H, rows=rows)
     got = host_f64(out)[rows]
-    check_out(got, ref, "full video out", small_x)
+    check_out(got, ref, "full video out", small_x, VIDEO_RESID)
     no_device_error()

@@ -126,7 +126,7 @@ def test_full_depth_velocity_at_tiny_dims(biased):
     # 2.5e-3 * sqrt(57), about 1.9e-2, on rel L2; max abs scales the same way
     # (6e-2 RMS).
     parity(got - f["latent"], ref - f["latent"], "full-depth velocity", rel_l2=2e-2, max_abs_frac=6e-2)
-    parity(got, ref, "full-depth latent")
+    parity(got, ref, "full-depth latent", max_abs_frac=6e-2)
 
 
 CACHED = synth.loop_shape(synth.BlockShape("loop_small", 16, 4, 6, 256, 2, 512), 2, 2, 6, channels=16, txt_in=64)
@@ -245,6 +245,8 @@ def test_full_dim_loop_velocity_matches_oracle():
     m64["double"] = _LazyF64Blocks(mw["double"])
     m64["single"] = _LazyF64Blocks(mw["single"])
     ref = O.euler_sample(f["latent"], f["txt"], f["ids"], m64, b.H, 1)
-    # the 57-block chain tolerance of test_full_depth_velocity_at_tiny_dims
+    # the 57-block chain tolerance of test_full_depth_velocity_at_tiny_dims;
+    # one step from t = 1 to 0 moves the latent by -v exactly, so the latent's
+    # error is the velocity's, whose max is bounded by the chain's 6e-2 RMS(v)
     parity(got - f["latent"], ref - f["latent"], "dim-3072 full-depth velocity", rel_l2=2e-2, max_abs_frac=6e-2)
-    parity(got, ref, "dim-3072 full-depth latent")
+    parity(got, ref, "dim-3072 full-depth latent", max_abs_frac=6e-2)
