@@ -1,21 +1,25 @@
-"""Sequence-parallel attention over the ranks of a torch.distributed group.
+"""Sequence-parallel attention and the sequence-parallel single-stream block
+over the ranks of a torch.distributed group.
 
-Page: "compile_graph" (chenyy20.com) §5.  The sequence is split evenly over
-the GPUs and every per-token step stays local; only attention needs the
+Page: "compile_graph" (chenyy20.com) §5 and §6.  The sequence is split evenly
+over the GPUs and every per-token step stays local; only attention needs the
 whole sequence.  Two ways to assemble it:
   - Ring: K and V travel around the ranks by point-to-point transfers, one hop
     per rank; every hop computes attention of the local queries against the
     shard in hand and merges it into the running result by log-sum-exp.
   - Ulysses: an all-to-all trades tokens for heads, so each rank holds the
     whole sequence for H/N heads; local attention; an all-to-all trades back.
+§6 captures the whole step, transfers included, as one CUDA graph: that needs
+fixed buffers and no allocation inside the step, so every plan below owns its
+buffers, allocated once, and a call only launches work on the current stream.
 
 Each rank holds a contiguous shard of S/N tokens: rank r owns tokens
-[r S/N, (r+1) S/N).  Tensors are [S/N, H*128] row-major (head h at columns
-h*128), as the block entry points lay them out.  The local operations default
-to this library's CUDA kernels (dit_attention with its log-sum-exp,
-dit_attention_merge); `attn` and `merge` can be replaced by callables with
-the same contracts, which the multi-process CPU tests use to check the
-schedules themselves.
+[r S/N, (r+1) S/N).  Tensors are [S/N, H*128] row views (head h at columns
+h*128, any row stride), as the block entry points lay them out.  The local
+operations default to this library's CUDA kernels (dit_attention with its
+log-sum-exp, dit_attention_merge, and the block's kernels); `ops` (or
+`attn` / `merge`) can be replaced by objects with the same contracts, which
+the multi-process CPU tests use to check the schedules themselves.
 """
 from __future__ import annotations
 
@@ -35,70 +39,179 @@ def _peer(group, r):
     return r if group is None else dist.get_global_rank(group, r)
 
 
+class RingAttention:
+    """One rank's ring attention with buffers owned by the plan.
+
+    Call: out = attention(q, K, V) where K and V are the concatenation of every
+    rank's k and v shards.  The local k and v are copied into slot 0 of a
+    two-slot ring; for N - 1 hops the shard in hand is sent to rank r+1 while
+    the next one is received from rank r-1, and the local attention of the
+    shard in hand runs meanwhile.  Hop 0 writes the running result, later hops
+    a partial result merged into it by log-sum-exp; the last merge writes
+    `out`.  Returns the fp32 log-sum-exp [1, H, S/N] of the local queries over
+    all keys (a buffer of the plan)."""
+
+    def __init__(self, S_loc, H, device, dtype=None, group=None, attn=None, merge=None):
+        import torch
+        import torch.distributed as dist
+        dtype = dtype or torch.bfloat16
+        self.H, self.S_loc, self.group = H, S_loc, group
+        self.N = dist.get_world_size(group)
+        self.r = dist.get_rank(group)
+        self.attn = attn or _cuda_attn
+        self.merge = merge or _cuda_merge
+        D = H * 128
+        self.kv = torch.empty((2, 2, S_loc, D), dtype=dtype, device=device)  # slot, (k, v)
+        self.o_acc = torch.empty((S_loc, D), dtype=dtype, device=device)
+        self.part = torch.empty_like(self.o_acc)
+        self.lse = torch.empty((1, H, S_loc), dtype=torch.float32, device=device)
+        self.lse_part = torch.empty_like(self.lse)
+        self.nxt = _peer(group, (self.r + 1) % self.N)
+        self.prv = _peer(group, (self.r - 1) % self.N)
+
+    def __call__(self, q, k, v, out):
+        import torch.distributed as dist
+        D, N, H = self.H * 128, self.N, self.H
+        self.kv[0, 0].copy_(k[:, :D])
+        self.kv[0, 1].copy_(v[:, :D])
+        for hop in range(N):
+            cur, nxt = hop & 1, (hop + 1) & 1
+            reqs = []
+            if hop < N - 1:
+                # one group for the send and the receive: with NCCL, separate calls
+                # would queue every rank's send ahead of its receive and wait in a cycle
+                reqs = dist.batch_isend_irecv([dist.P2POp(dist.isend, self.kv[cur], self.nxt, self.group),
+                                               dist.P2POp(dist.irecv, self.kv[nxt], self.prv, self.group)])
+            kk, vv = self.kv[cur, 0], self.kv[cur, 1]
+            if hop == 0:
+                self.attn(q, kk, vv, out if N == 1 else self.o_acc, self.lse, H)
+            else:
+                self.attn(q, kk, vv, self.part, self.lse_part, H)
+                self.merge([self.o_acc, self.part], [self.lse, self.lse_part],
+                           out if hop == N - 1 else self.o_acc, self.lse, H)
+            for req in reqs:
+                req.wait()
+        return self.lse
+
+
+class UlyssesAttention:
+    """One rank's Ulysses attention with buffers owned by the plan.
+
+    Call: out = attention(q, K, V) over the whole sequence with heads split
+    across ranks: an all-to-all gives rank r all tokens of heads
+    [r H/N, (r+1) H/N), attention runs there, and a second all-to-all returns
+    every rank its own tokens.  H must be a multiple of the group size."""
+
+    def __init__(self, S_loc, H, device, dtype=None, group=None, attn=None):
+        import torch
+        import torch.distributed as dist
+        dtype = dtype or torch.bfloat16
+        self.N = dist.get_world_size(group)
+        if H % self.N:
+            raise ValueError(f"{H} heads do not split over {self.N} ranks")
+        self.H, self.S_loc, self.group = H, S_loc, group
+        self.attn = attn or _cuda_attn
+        self.Hl = H // self.N
+        w = self.Hl * 128
+        # q, k, v; chunk i of the token shard goes to rank i / comes from rank i
+        self.send = torch.empty((3, self.N, S_loc, w), dtype=dtype, device=device)
+        self.recv = torch.empty_like(self.send)
+        self.o_heads = torch.empty((self.N * S_loc, w), dtype=dtype, device=device)
+        self.o_back = torch.empty((self.N, S_loc, w), dtype=dtype, device=device)
+
+    def __call__(self, q, k, v, out):
+        import torch.distributed as dist
+        N, S_loc, Hl = self.N, self.S_loc, self.Hl
+        w = Hl * 128
+        for i, t in enumerate((q, k, v)):  # [S_loc, H*128] -> [N, S_loc, w]: head group i -> rank i
+            self.send[i].copy_(t[:, :N * w].reshape(S_loc, N, w).transpose(0, 1))
+        for i in range(3):
+            dist.all_to_all_single(self.recv[i], self.send[i], group=self.group)
+        # rank i's tokens in rank order: the whole sequence for this rank's heads
+        qh, kh, vh = (self.recv[i].view(N * S_loc, w) for i in range(3))
+        self.attn(qh, kh, vh, self.o_heads, None, Hl)
+        dist.all_to_all_single(self.o_back, self.o_heads.view(N, S_loc, w), group=self.group)
+        out[:, :N * w].copy_(self.o_back.transpose(0, 1).reshape(S_loc, N * w))  # head group i came from rank i
+        return out
+
+
 def ring_attention(q, k, v, out, H, group=None, attn=None, merge=None):
-    """out = attention(q, K, V) where K and V are the concatenation of every
-    rank's k and v shards.  N - 1 hops: the shard in hand is sent to rank r+1
-    and the next one received from rank r-1 while the local attention of the
-    shard in hand runs; each hop's result is merged into `out` by log-sum-exp.
-    Returns the fp32 log-sum-exp [H, S/N] of the local queries over all keys."""
-    import torch
-    import torch.distributed as dist
-    attn = attn or _cuda_attn
-    merge = merge or _cuda_merge
-    N = dist.get_world_size(group)
-    r = dist.get_rank(group)
-    S_loc = q.shape[0]
-    kv = torch.stack([k, v])
-    buf = torch.empty_like(kv)
-    lse = torch.empty((H, S_loc), dtype=torch.float32, device=q.device)
-    part = torch.empty_like(out)
-    lse_part = torch.empty_like(lse)
-    nxt, prv = _peer(group, (r + 1) % N), _peer(group, (r - 1) % N)
-    for hop in range(N):
-        reqs = []
-        if hop < N - 1:
-            # one group for the send and the receive: with NCCL, separate calls
-            # would queue every rank's send ahead of its receive and wait in a cycle
-            reqs = dist.batch_isend_irecv([dist.P2POp(dist.isend, kv, nxt, group),
-                                           dist.P2POp(dist.irecv, buf, prv, group)])
-        if hop == 0:
-            attn(q, kv[0], kv[1], out, lse, H)
-        else:
-            attn(q, kv[0], kv[1], part, lse_part, H)
-            merge([out, part], [lse, lse_part], out, lse, H)
-        for req in reqs:
-            req.wait()
-        if hop < N - 1:
-            kv, buf = buf, kv
-    return lse
+    """One-off ring attention (a plan built for this call); see RingAttention."""
+    plan = RingAttention(q.shape[0], H, q.device, q.dtype, group, attn, merge)
+    lse = plan(q, k, v, out)
+    return lse[0]
 
 
 def ulysses_attention(q, k, v, out, H, group=None, attn=None):
-    """out = attention(q, K, V) over the whole sequence with heads split across
-    ranks: an all-to-all gives rank r all tokens of heads [r H/N, (r+1) H/N),
-    attention runs there, and a second all-to-all returns every rank its own
-    tokens.  H must be a multiple of the group size."""
-    import torch
-    import torch.distributed as dist
-    attn = attn or _cuda_attn
-    N = dist.get_world_size(group)
-    if H % N:
-        raise ValueError(f"{H} heads do not split over {N} ranks")
-    S_loc = q.shape[0]
-    Hl = H // N
-    w = Hl * 128
+    """One-off Ulysses attention (a plan built for this call); see UlyssesAttention."""
+    return UlyssesAttention(q.shape[0], H, q.device, q.dtype, group, attn)(q, k, v, out)
 
-    def to_heads(t):  # [S_loc, H*128] -> [S, Hl*128]: this rank's heads, every rank's tokens
-        send = t.reshape(S_loc, N, w).transpose(0, 1).contiguous()  # [N, S_loc, w], chunk i -> rank i
-        recv = torch.empty_like(send)
-        dist.all_to_all_single(recv, send, group=group)
-        return recv.reshape(N * S_loc, w)  # rank i's tokens in rank order
 
-    qh, kh, vh = to_heads(q), to_heads(k), to_heads(v)
-    oh = torch.empty_like(qh)
-    attn(qh, kh, vh, oh, None, Hl)
-    send = oh.reshape(N, S_loc, w).contiguous()  # token chunk i -> rank i
-    recv = torch.empty_like(send)
-    dist.all_to_all_single(recv, send, group=group)
-    out.copy_(recv.transpose(0, 1).reshape(S_loc, N * w))  # head group i came from rank i
-    return out
+class CudaBlockOps:
+    """The per-token steps of the single-stream block as this library's
+    kernels (the same calls dit_single_block_fwd makes)."""
+
+    def __init__(self, D, H, M, eps=1e-6):
+        self.D, self.H, self.M, self.eps = D, H, M, eps
+
+    def adaln(self, w, vec, mod):
+        from . import dit_adaln_modulation
+        dit_adaln_modulation(vec, w["W_mod"], w["b_mod"], mod)
+
+    def modulate_norm(self, x, mod, y):
+        from . import dit_modulate_norm
+        D = self.D
+        dit_modulate_norm(x, mod[0, :D], mod[0, D:2 * D], y, 1, x.shape[0], self.eps)
+
+    def qkv_mlp(self, w, y, rope, qkv, cat):
+        from . import dit_gemm_epilogue, DIT_EPI_BIAS_GELU_COLS
+        D = self.D
+        dit_gemm_epilogue(y, w["W1"], qkv, epi=DIT_EPI_BIAS_GELU_COLS, bias=w["b1"], C2=cat[:, D:],
+                          split_col=3 * D, gelu_col_begin=3 * D, qk_cols=2 * D, qk_norm=1, qk_eps=self.eps,
+                          q_scale=w["q_scale"], k_scale=w["k_scale"], rope=rope, rope_rows=y.shape[0])
+
+    def out_proj(self, w, cat, x, mod, out):
+        from . import dit_gemm_epilogue, DIT_EPI_BIAS_GATED_RESIDUAL
+        D = self.D
+        dit_gemm_epilogue(cat, w["W2"], out, epi=DIT_EPI_BIAS_GATED_RESIDUAL, bias=w["b2"],
+                          gate=mod[0, 2 * D:], gate_stride=0, resid=x, rows_per_batch=x.shape[0])
+
+
+class SequenceParallelSingleBlock:
+    """Flux single-stream block over a sequence sharded across the ranks of a
+    group ("compile_graph" §5-§6): adaLN, LayerNorm + modulate, the fused
+    QKV|MLP-in GEMM (QK RMSNorm + RoPE with this shard's rows of the RoPE
+    table, GELU on the MLP columns) and the output GEMM with the gated residual
+    run on the local S/N tokens; attention assembles the whole sequence by the
+    ring or by Ulysses.  Every buffer is allocated here, once, so a forward
+    launches work only and can be captured, transfers included, into a CUDA
+    graph.
+
+    forward(w, x, vec, rope, out): x, out [S/N, D] bf16 (out may be x); vec
+    [1, D] bf16; rope: this shard's rows of the RoPE table [S/N, 64, 2] fp32."""
+
+    def __init__(self, S_loc, D, H, M, device, group=None, mode="ring", ops=None, attn=None, merge=None,
+                 dtype=None, eps=1e-6):
+        import torch
+        dtype = dtype or torch.bfloat16
+        if mode not in ("ring", "ulysses"):
+            raise ValueError(f"mode {mode!r}")
+        self.D, self.M, self.S_loc = D, M, S_loc
+        self.ops = ops or CudaBlockOps(D, H, M, eps)
+        self.mod = torch.empty((1, 3 * D), dtype=torch.float32 if dtype == torch.bfloat16 else dtype, device=device)
+        self.y = torch.empty((S_loc, D), dtype=dtype, device=device)
+        self.qkv = torch.empty((S_loc, 3 * D), dtype=dtype, device=device)
+        self.cat = torch.empty((S_loc, D + M), dtype=dtype, device=device)
+        if mode == "ring":
+            self.attention = RingAttention(S_loc, H, device, dtype, group, attn, merge)
+        else:
+            self.attention = UlyssesAttention(S_loc, H, device, dtype, group, attn)
+
+    def forward(self, w, x, vec, rope, out):
+        D = self.D
+        self.ops.adaln(w, vec, self.mod)
+        self.ops.modulate_norm(x, self.mod, self.y)
+        self.ops.qkv_mlp(w, self.y, rope, self.qkv, self.cat)
+        self.attention(self.qkv[:, :D], self.qkv[:, D:2 * D], self.qkv[:, 2 * D:], self.cat[:, :D])
+        self.ops.out_proj(w, self.cat, x, self.mod, out)
+        return out

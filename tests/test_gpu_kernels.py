@@ -412,6 +412,61 @@ def test_sequence_parallel_drivers_with_cuda_kernels_one_rank():
     assert_no_device_error()
 
 
+@pytest.mark.parametrize("mode", ["ring", "ulysses"])
+def test_sequence_parallel_block_one_rank_equals_block_and_graph_replays_it(mode):
+    """The sequence-parallel single-stream block (static buffers, CUDA
+    kernels) in a one-rank NCCL group runs the block's five kernels on the
+    same inputs, so it equals dit_single_block_fwd bit for bit; captured into a
+    CUDA graph (the Ulysses all-to-alls included), a replay gives the same bits
+    again.  The multi-rank schedules are checked on CPU ranks."""
+    import datetime
+    import socket
+    import torch
+    import torch.distributed as dist
+    from diffusion_transformer_block_flux_b200 import sequence_parallel as sp
+    sock = socket.socket()
+    sock.bind(("127.0.0.1", 0))
+    port = sock.getsockname()[1]
+    sock.close()
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1,
+                            timeout=datetime.timedelta(seconds=60), device_id=torch.device("cuda", 0))
+    graph = None
+    try:
+        s = synth.TINY
+        wb = synth.single_block_weights(s, bias_std=synth.TEST_BIAS_STD, norm_scale_std=synth.TEST_NORM_SCALE_STD)
+        ab = synth.block_activations(s)
+        w = dev_tree(wb)
+        x = dev_bf16(ab["x"])
+        vec = dev_bf16(ab["vec"]).reshape(1, -1)
+        rope = torch.empty((s.S, 64, 2), dtype=torch.float32, device="cuda")
+        dit.dit_rope_table(torch.from_numpy(ab["ids"]).cuda(), (8, 28, 28), 10000.0, rope)
+        cfg = dit.block_cfg(1, s.S, s.D, s.H, s.M)
+        ws = torch.empty(dit.dit_single_block_workspace(cfg), dtype=torch.uint8, device="cuda")
+        ref = torch.empty_like(x)
+        dit.dit_single_block_fwd(cfg, dit.single_weights(w), x, vec, rope, ref, ws)
+        blk = sp.SequenceParallelSingleBlock(s.S, s.D, s.H, s.M, "cuda", mode=mode)
+        out = torch.empty_like(x)
+        blk.forward(w, x, vec, rope, out)
+        torch.cuda.synchronize()
+        assert torch.equal(out, ref)
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            blk.forward(w, x, vec, rope, out)  # warm-up on the capture stream
+        torch.cuda.current_stream().wait_stream(side)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            blk.forward(w, x, vec, rope, out)
+        out.zero_()
+        graph.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(out, ref)
+    finally:
+        del graph  # a graph holding NCCL work is released before the group
+        dist.destroy_process_group()
+    assert_no_device_error()
+
+
 # ---------------------------------------------------------------- failure detection
 
 def test_selftest_wait_times_out_and_reports():
