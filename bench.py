@@ -700,6 +700,11 @@ def run_loop(args):
     import diffusion_transformer_block_flux_b200 as dit
     from diffusion_transformer_block_flux_b200 import synth
     ls = synth.FLUX_LOOP
+    if args.loop_blocks or args.loop_steps:
+        # a shorter or shallower loop of the same width (profiling captures on a few GB)
+        nd, ns = (int(v) for v in args.loop_blocks.split(",")) if args.loop_blocks else (ls.n_double, ls.n_single)
+        ls = synth.loop_shape(synth.FLUX, nd, ns, args.loop_steps or ls.steps, channels=ls.channels,
+                              txt_in=ls.txt_in)
     dev = torch.device("cuda", 0)
     g = torch.Generator(device=dev)
     g.manual_seed(11)
@@ -840,7 +845,47 @@ def run_kernels(args):
             "hbm_peak_gbs": pk["hbm_gbs"], "kernels": res}
 
 
-EXTRA = {"double": run_double, "video": run_video, "loop": run_loop, "kernels": run_kernels, "ring8": run_ring8}
+def run_cfg_batch(args):
+    """Classifier-free guidance as one batch-2 pass or as two batch-1 passes:
+    the single-stream block (S=4608) and the double-stream block (512 + 4096)
+    at B = 2 against two B = 1 calls on the same two samples (the SDXL guide,
+    section 3.3, runs the conditional and unconditional halves as one batch)."""
+    import torch
+    import diffusion_transformer_block_flux_b200 as dit
+    from diffusion_transformer_block_flux_b200 import synth
+    dev = torch.device("cuda", 0)
+    w, x, vec = make_block(torch, dev, seed=21)
+    x2 = torch.cat([x, torch.roll(x, 1, 0)])
+    vec2 = torch.cat([vec, vec])
+    ids = torch.from_numpy(synth.flux_ids(S_TXT, GRID, GRID)).to(dev)
+    rope = torch.empty((S, 64, 2), dtype=torch.float32, device=dev)
+    dit.dit_rope_table(ids, (8, 28, 28), 10000.0, rope)
+    cw = dit.single_weights(w)
+    c1, c2 = dit.block_cfg(1, S, D, H, M), dit.block_cfg(2, S, D, H, M)
+    ws = torch.empty(dit.dit_single_block_workspace(c2), dtype=torch.uint8, device=dev)
+    o2 = torch.empty_like(x2)
+    K, W = args.steps, args.warmup
+    st = torch.cuda.current_stream()
+    t2 = _event_time(torch, lambda: dit.dit_single_block_fwd(c2, cw, x2, vec2, rope, o2, ws), K, W, st)
+    clk2 = dict(_LAST_CLOCKS)
+
+    def two():
+        dit.dit_single_block_fwd(c1, cw, x2[:S], vec2[:1], rope, o2[:S], ws)
+        dit.dit_single_block_fwd(c1, cw, x2[S:], vec2[1:], rope, o2[S:], ws)
+    t1 = _event_time(torch, two, K, W, st)
+    flops = 2 * block_flops_total()
+    res = _extra_line("cfg_single_block_batch2_vs_2x_batch1_S4608_D3072", t2, flops, K, W,
+                      {"ms_batch2": round(t2, 4), "ms_two_batch1": round(t1, 4),
+                       "batch2_speedup": round(t1 / t2, 4), "clocks_batch2": clk2})
+    return res
+
+
+def block_flops_total(S_=S):
+    return sum(block_flops(S_).values())
+
+
+EXTRA = {"double": run_double, "video": run_video, "loop": run_loop, "kernels": run_kernels, "ring8": run_ring8,
+         "cfg_batch": run_cfg_batch}
 
 
 def main():
@@ -856,6 +901,10 @@ def main():
                     help="loop workload: model-level step cache (26 model forwards for 50 steps)")
     ap.add_argument("--cfg", action="store_true",
                     help="loop workload: classifier-free guidance on the first 75%% of the steps")
+    ap.add_argument("--loop-blocks", default="",
+                    help="loop workload: 'double,single' block counts instead of 19,38 (same width)")
+    ap.add_argument("--loop-steps", type=int, default=0,
+                    help="loop workload: Euler steps instead of 50")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -81,7 +81,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(&v_full[s], 1);
       mbar_init(&v_empty[s], 1);
       mbar_init(&s_full[s], 1);
-      mbar_init(&p_full[s], 128);
+      mbar_init(&p_full[s], 4);  // one arrival per softmax warp of the tile
       mbar_init(&o_full[s], 1);
     }
     mbar_init(drain, 1);
@@ -297,7 +297,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       m_run = m_new;
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&p_full[t]);
+      __syncwarp();  // every lane's P (and O) stores are complete before the warp's one arrival
+      if (lane == 0) mbar_arrive(&p_full[t]);
     }
     if (ok) {
       ok = mbar_wait(&o_full[t], 0, wait_limit, abort_flag, SITE_ATTN_SOFTMAX);

@@ -106,6 +106,27 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64
   return mbar_wait_slow(bar, parity, limit_ns, abort, site);
 }
 
+// The same bounded wait with the slow path inlined, for kernels that give
+// their warpgroups different register counts (setmaxnreg): ptxas cannot
+// allocate a called function that is reached under two register limits.
+__device__ __forceinline__ bool mbar_wait_inl(uint64_t* bar, uint32_t parity, uint64_t limit_ns,
+                                              volatile int* abort, uint32_t site) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  uint32_t n = 0;
+  while (!mbar_try_wait(bar, parity)) {
+    if ((++n & 255u) == 0) {
+      if (abort != nullptr && *abort) return false;
+      if (globaltimer_ns() - t0 > limit_ns) {
+        atomicCAS(&g_dit_error, 0u, (uint32_t)DIT_ERR_TIMEOUT | (site << 8));
+        if (abort != nullptr) *abort = 1;
+        return false;
+      }
+    }
+  }
+  return true;
+}
+
 // ---------------------------------------------------------------------------
 // TMA (cp.async.bulk.tensor), no multicast
 // ---------------------------------------------------------------------------
@@ -195,6 +216,26 @@ __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* m
       " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(m)), "r"(bar_cluster), "r"(c0), "r"(c1)
       : "memory");
+}
+
+// The same load with an L2 cache-eviction hint (a policy from createpolicy).
+__device__ __forceinline__ void tma_load_2d_pair_hint(void* dst, const CUtensorMap* m, uint32_t bar_cluster, int c0,
+                                                      int c1, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(bar_cluster), "r"(c0), "r"(c1), "l"(policy)
+      : "memory");
+}
+
+// L2 policy for data read once per kernel phase: its lines are the first
+// candidates for eviction, which keeps the lines of data that is read again
+// (a GEMM's re-used operand) in the cache.  Applies to the hinted accesses
+// only; nothing stays pinned after the kernel.
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
 }
 
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {

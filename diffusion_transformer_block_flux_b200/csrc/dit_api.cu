@@ -30,7 +30,8 @@ static_assert(dit::gemm::pair::SMEM_BYTES <= 227 * 1024, "pair GEMM shared memor
 static_assert(dit::attn::SMEM_BYTES <= 227 * 1024, "attention shared memory above the per-CTA limit");
 static_assert(dit::gemm::TMEM_COLS <= 512 && dit::gemm::pair::TMEM_COLS <= 512 && dit::attn::TMEM_COLS <= 512,
               "TMEM allocation above 512 columns");
-constexpr int kVecPipeSmemMax = 144 * 1024;  // adaLN: 4 warps x 4 weight rows of K <= 4096 bf16 + K fp32
+constexpr int kVecPipeSmemMax = 144 * 1024;
+constexpr int kVecRowsCtasPerSm = 1;  // vec_rows kernels: 512 threads (16 warps) per CTA  // adaLN: 4 warps x 4 weight rows of K <= 4096 bf16 + K fp32
 uint64_t g_wait_limit_ns = 2000000000ull;
 
 // Per-device state, filled once under g_mu.  `init` is published with a
@@ -315,15 +316,15 @@ dit_status dit_vec_linear(const dit_bf16* x, int64_t ldx, const dit_bf16* W, int
   const bf16* xb = reinterpret_cast<const bf16*>(x);
   const bf16* Wb = reinterpret_cast<const bf16*>(W);
   const bf16* bb = reinterpret_cast<const bf16*>(bias);
-  if (B == 1 && (K % 256) == 0 && K <= 4096) {
-    // weight rows in flight through warp-private shared-memory rings (cp.async, 3 rows ahead)
-    const size_t ring_smem = (size_t)dit::kVecPipeWarps * dit::kVecPipeSlots * K * 2 + (size_t)K * 4;
-    int rgrid = (N + dit::kVecPipeWarps - 1) / dit::kVecPipeWarps;
-    const int per_sm = (int)(220 * 1024 / (ring_smem + 1024));
-    if (rgrid > sms * per_sm) rgrid = sms * per_sm;
-#define DIT_VR_CASE(KC_)                                                                                   \
-  case KC_:                                                                                                \
-    dit::vec_linear_pipe_kernel<KC_><<<rgrid, 128, ring_smem, st>>>(xb, Wb, ldw, bb, out, N, K, flags);     \
+  if (B == 1 && (K % 256) == 0 && K <= 3072) {
+    // one warp per weight row, two rows in flight per warp, 16 warps per CTA
+    const int64_t warps = (int64_t)sms * kVecRowsCtasPerSm * 16;
+    int64_t grid = (int64_t)sms * kVecRowsCtasPerSm;
+    if (N < warps) grid = (N + 15) / 16;
+    const size_t xs_smem = (size_t)K * 4;
+#define DIT_VR_CASE(KC_)                                                                                  \
+  case KC_:                                                                                               \
+    dit::vec_rows_kernel<KC_><<<(unsigned)grid, 512, xs_smem, st>>>(xb, Wb, ldw, bb, out, N, K, flags);    \
     return launch_status();
     switch (K / 256) {
       DIT_VR_CASE(1)
@@ -333,11 +334,24 @@ dit_status dit_vec_linear(const dit_bf16* x, int64_t ldx, const dit_bf16* W, int
       DIT_VR_CASE(6)
       DIT_VR_CASE(8)
       DIT_VR_CASE(12)
-      DIT_VR_CASE(16)
       default:
         break;
     }
 #undef DIT_VR_CASE
+  }
+  if (B == 1 && (K % 256) == 0 && K <= 4096) {
+    // weight rows in flight through warp-private shared-memory rings (cp.async, 3 rows ahead)
+    const size_t ring_smem = (size_t)dit::kVecPipeWarps * dit::kVecPipeSlots * K * 2 + (size_t)K * 4;
+    int rgrid = (N + dit::kVecPipeWarps - 1) / dit::kVecPipeWarps;
+    const int per_sm = (int)(220 * 1024 / (ring_smem + 1024));
+    if (rgrid > sms * per_sm) rgrid = sms * per_sm;
+    switch (K / 256) {
+      case 16:
+        dit::vec_linear_pipe_kernel<16><<<rgrid, 128, ring_smem, st>>>(xb, Wb, ldw, bb, out, N, K, flags);
+        return launch_status();
+      default:
+        break;
+    }
   }
   const size_t bulk_smem = smem + (size_t)dit::kRowWarps * 2 * K * 2 + dit::kRowWarps * 2 * 8;
   if (bulk_smem <= (size_t)kRowSmemMax) {
@@ -372,7 +386,8 @@ dit_status dit_vec_linear(const dit_bf16* x, int64_t ldx, const dit_bf16* W, int
 }
 
 // One pass over every matrix of p (batch-1 input x shared by all): see
-// vec_linear_multi_kernel.  K % 256 == 0, K <= 4096; used by the loop.
+// vec_rows_multi_kernel (K <= 3072) and vec_linear_multi_kernel (K = 4096).
+// K % 256 == 0, K <= 4096; used by the loop.
 bool multi_linear_supported(int K) { return (K % 256) == 0 && K <= 4096; }
 
 dit_status multi_linear(const dit_bf16* x, const dit::MultiLinear& p, int flags, cudaStream_t st) {
@@ -381,6 +396,28 @@ dit_status multi_linear(const dit_bf16* x, const dit::MultiLinear& p, int flags,
   dit_status s = device_setup(&sms);
   if (s != DIT_OK) return s;
   const int64_t N = p.row_begin[p.n_mats];
+  if (p.K <= 3072) {
+    int64_t rgrid = (int64_t)sms * kVecRowsCtasPerSm;
+    if (N < rgrid * 16) rgrid = (N + 15) / 16;
+    const size_t xs_smem = (size_t)p.K * 4;
+    const bf16* xr = reinterpret_cast<const bf16*>(x);
+    switch (p.K / 256) {
+#define DIT_VRM_CASE(KC_)                                                                          \
+  case KC_:                                                                                        \
+    dit::vec_rows_multi_kernel<KC_><<<(unsigned)rgrid, 512, xs_smem, st>>>(xr, p, flags);         \
+    return launch_status();
+      DIT_VRM_CASE(1)
+      DIT_VRM_CASE(2)
+      DIT_VRM_CASE(3)
+      DIT_VRM_CASE(4)
+      DIT_VRM_CASE(6)
+      DIT_VRM_CASE(8)
+      DIT_VRM_CASE(12)
+#undef DIT_VRM_CASE
+      default:
+        break;
+    }
+  }
   const size_t smem = (size_t)dit::kVecPipeWarps * dit::kVecPipeSlots * p.K * 2 + (size_t)p.K * 4;
   int64_t grid = (N + dit::kVecPipeWarps - 1) / dit::kVecPipeWarps;
   const int per_sm = (int)(220 * 1024 / (smem + 1024));
@@ -627,22 +664,24 @@ dit_status dit_gemm_epilogue(const dit_gemm_args* a, void* stream) {
     const int tiles = ((a->M + P::BM - 1) / P::BM) * ((a->N + P::BN - 1) / P::BN);
     const int clusters = tiles < sms / 2 ? tiles : sms / 2;
     const int grid = 2 * clusters;
+    // walk the larger operand's panels once: N-fastest when A (M x K) is the larger
+    const int nf = a->M > a->N ? 1 : 0;
     switch (a->epi) {
       case DIT_EPI_NONE:
         P::gemm_pair_kernel<DIT_EPI_NONE><<<grid, P::NUM_THREADS, P::SMEM_BYTES, st>>>(tA, tB, a->M, a->N, a->K, ep,
-                                                                                     g_wait_limit_ns);
+                                                                                     g_wait_limit_ns, nf);
         break;
       case DIT_EPI_BIAS:
         P::gemm_pair_kernel<DIT_EPI_BIAS><<<grid, P::NUM_THREADS, P::SMEM_BYTES, st>>>(tA, tB, a->M, a->N, a->K, ep,
-                                                                                     g_wait_limit_ns);
+                                                                                     g_wait_limit_ns, nf);
         break;
       case DIT_EPI_BIAS_GELU_COLS:
         P::gemm_pair_kernel<DIT_EPI_BIAS_GELU_COLS><<<grid, P::NUM_THREADS, P::SMEM_BYTES, st>>>(
-            tA, tB, a->M, a->N, a->K, ep, g_wait_limit_ns);
+            tA, tB, a->M, a->N, a->K, ep, g_wait_limit_ns, nf);
         break;
       default:
         P::gemm_pair_kernel<DIT_EPI_BIAS_GATED_RESIDUAL><<<grid, P::NUM_THREADS, P::SMEM_BYTES, st>>>(
-            tA, tB, a->M, a->N, a->K, ep, g_wait_limit_ns);
+            tA, tB, a->M, a->N, a->K, ep, g_wait_limit_ns, nf);
         break;
     }
     return launch_status();

@@ -211,6 +211,102 @@ __global__ void __launch_bounds__(256) modulate_norm_row_kernel(const bf16* __re
 }
 
 // ---------------------------------------------------------------------------
+// Vector x weight rows (adaLN modulation, the timestep MLP), batch 1,
+// K = 256 KC: one warp per output row, lane l reading the 16-byte chunks
+// l, l + 32, ... of the row with streaming loads, the (mapped) input vector
+// in shared memory as fp32.  A warp issues the loads of its next row as soon
+// as a row is reduced, and keeps two rows in flight for K <= 1536; rows are
+// dealt to the warps of a persistent grid round robin.  RowFn(n) gives row n's weight
+// pointer, bias and output slot, so the same loop serves one matrix and a
+// list of matrices that share the input (every block's modulation of a step).
+// ---------------------------------------------------------------------------
+struct VecRow {
+  const uint4* w;
+  const bf16* bias;
+  int64_t local;  // index of the row within its matrix
+  int mat;        // which matrix (0 for a single matrix)
+};
+
+template <int KC>
+__device__ __forceinline__ void vr_load(uint4 (&u)[KC], float& bv, const VecRow& rw, bool on, int lane) {
+#pragma unroll
+  for (int c = 0; c < KC; ++c) u[c] = on ? __ldcs(rw.w + c * 32 + lane) : make_uint4(0, 0, 0, 0);
+  bv = (on && lane == 0 && rw.bias != nullptr) ? __bfloat162float(rw.bias[rw.local]) : 0.0f;
+}
+
+template <int KC>
+__device__ __forceinline__ float vr_dot(const uint4 (&u)[KC], const float4* __restrict__ xs, int lane) {
+  float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+  for (int c = 0; c < KC; ++c) {
+    const int k = (c * 32 + lane) * 2;
+    const float4 x0 = xs[k], x1 = xs[k + 1];
+    a0 = fmaf(bf16_lo(u[c].x), x0.x, a0); a1 = fmaf(bf16_hi(u[c].x), x0.y, a1);
+    a0 = fmaf(bf16_lo(u[c].y), x0.z, a0); a1 = fmaf(bf16_hi(u[c].y), x0.w, a1);
+    a0 = fmaf(bf16_lo(u[c].z), x1.x, a0); a1 = fmaf(bf16_hi(u[c].z), x1.y, a1);
+    a0 = fmaf(bf16_lo(u[c].w), x1.z, a0); a1 = fmaf(bf16_hi(u[c].w), x1.w, a1);
+  }
+  return warp_sum(a0 + a1);
+}
+
+template <int KC, typename RowFn, typename OutFn>
+__device__ __forceinline__ void vec_rows_loop(const bf16* __restrict__ x, int K, int flags, int64_t N, RowFn row_of,
+                                              OutFn store) {
+  constexpr bool TWO = KC <= 6;  // two rows in flight per warp while the registers allow it
+  extern __shared__ float4 xs4[];  // the mapped input, K fp32
+  float* xs = reinterpret_cast<float*>(xs4);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t nw = (int64_t)gridDim.x * (blockDim.x >> 5);
+  const int64_t step = TWO ? 2 * nw : nw;
+  int64_t n = (int64_t)blockIdx.x * (blockDim.x >> 5) + warp;
+  uint4 ua[KC], ub[TWO ? KC : 1];
+  float ba = 0.f, bb = 0.f;
+  VecRow ra = row_of(n < N ? n : 0), rb = ra;
+  vr_load<KC>(ua, ba, ra, n < N, lane);
+  if constexpr (TWO) {
+    rb = row_of(n + nw < N ? n + nw : 0);
+    vr_load<KC>(ub, bb, rb, n + nw < N, lane);
+  }
+  for (int k = threadIdx.x; k < K; k += blockDim.x) {
+    float z = __bfloat162float(x[k]);
+    if (flags & DIT_VEC_SILU_IN) z = silu(z);
+    xs[k] = z;
+  }
+  __syncthreads();
+  for (; n < N; n += step) {
+    const float da = vr_dot<KC>(ua, xs4, lane) + ba;
+    if (lane == 0) store(ra, da);
+    const int64_t n2 = n + step;
+    ra = row_of(n2 < N ? n2 : 0);
+    vr_load<KC>(ua, ba, ra, n2 < N, lane);
+    if constexpr (TWO) {
+      if (n + nw < N) {
+        const float db = vr_dot<KC>(ub, xs4, lane) + bb;
+        if (lane == 0) store(rb, db);
+      }
+      const int64_t n3 = n + nw + step;
+      rb = row_of(n3 < N ? n3 : 0);
+      vr_load<KC>(ub, bb, rb, n3 < N, lane);
+    }
+  }
+}
+
+template <int KC>
+__global__ void __launch_bounds__(512, 1) vec_rows_kernel(const bf16* __restrict__ x, const bf16* __restrict__ W,
+                                                       int64_t ldw, const bf16* __restrict__ bias, void* out,
+                                                       int64_t N, int K, int flags) {
+  vec_rows_loop<KC>(
+      x, K, flags, N,
+      [=](int64_t n) { return VecRow{reinterpret_cast<const uint4*>(W + n * ldw), bias, n, 0}; },
+      [=](const VecRow& rw, float v) {
+        if (flags & DIT_VEC_OUT_BF16)
+          reinterpret_cast<bf16*>(out)[rw.local] = __float2bfloat16_rn(v);
+        else
+          reinterpret_cast<float*>(out)[rw.local] = v;
+      });
+}
+
+// ---------------------------------------------------------------------------
 // adaLN / vector x weight, batch 1, with the weight rows in flight through a
 // warp-private shared-memory ring of P row slots.  Lane l copies its KC
 // 16-byte chunks (columns 8(l + 32j) .. +8) of the warp's next rows into the
@@ -398,6 +494,21 @@ __global__ void __launch_bounds__(128) vec_linear_multi_kernel(const bf16* __res
     if (++slot == P) slot = 0;
   }
   cp_async_wait<0>();
+}
+
+// Every matrix of p in one pass with the loop above (one warp per row, two
+// rows in flight); out[j][n - row_begin[j]] = W_j[row] . f(x) + bias_j[row].
+template <int KC>
+__global__ void __launch_bounds__(512, 1) vec_rows_multi_kernel(const bf16* __restrict__ x,
+                                                             const __grid_constant__ MultiLinear p, int flags) {
+  vec_rows_loop<KC>(
+      x, p.K, flags, (int64_t)p.row_begin[p.n_mats],
+      [&](int64_t n) {
+        const int j = multi_find(p, n);
+        const int64_t local = n - p.row_begin[j];
+        return VecRow{reinterpret_cast<const uint4*>(p.W[j] + local * p.K), p.bias[j], local, j};
+      },
+      [&](const VecRow& rw, float v) { p.out[rw.mat][rw.local] = v; });
 }
 
 // ---------------------------------------------------------------------------

@@ -8,7 +8,8 @@
 //
 // Design (sm_100a):
 //   - persistent CTAs, one per SM, tiles of 128 x 256 taken in M-fastest order
-//     so the CTAs running together share B tiles in L2;
+//     so the CTAs running together share B tiles in L2 (the SM-pair kernel
+//     below picks M- or N-fastest per shape);
 //   - warp 0: TMA producer (4-stage ring of 128x64 A and 256x64 B tiles,
 //     128-byte swizzle); warp 1: TMEM allocator + single-thread MMA issuer
 //     (tcgen05.mma 128x256x16, fp32 accumulators in TMEM); warps 2-5: epilogue
@@ -386,6 +387,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 // ---------------------------------------------------------------------------
 namespace pair {
 
+// Tile order.  M-fastest (n_fastest = 0): the clusters running together share
+// B panels, and every wave re-reads the whole A operand, so A should be the
+// smaller operand (it then stays in L2 from wave to wave).  N-fastest: the
+// other way round, for GEMMs whose A is larger than their weight (the output
+// projections: A = [S, D+M], W = [D, D+M]).
+__device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int n_fastest, int& tm, int& tn) {
+  if (n_fastest) {
+    tm = tile / num_n;
+    tn = tile - tm * num_n;
+  } else {
+    tn = tile / num_m;
+    tm = tile - tn * num_m;
+  }
+}
+
 constexpr int BM = 256;      // rows per cluster tile
 constexpr int BM_CTA = 128;  // rows per CTA
 constexpr int BN = 256;
@@ -403,7 +419,7 @@ constexpr uint32_t IDESC = idesc_bf16(BM, BN, 0, 0);
 template <int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M, int N,
-                     int K, Epi ep, uint64_t wait_limit) {
+                     int K, Epi ep, uint64_t wait_limit, int n_fastest) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
@@ -458,8 +474,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       uint32_t phase = 0;
       uint32_t issued_mask = 0, issued_parity = 0;
       bool ok = true;
+      // N-fastest: each A panel is consumed by the clusters of one wave and
+      // not needed again, so it is loaded as evict-first and the weight
+      // panels that every wave re-reads stay in L2
+      const uint64_t a_policy = l2_policy_evict_first();
       for (int tile = cluster_id; tile < num_tiles && ok; tile += n_clusters) {
-        const int tm = tile % num_m, tn = tile / num_m;
+        int tm, tn;
+        tile_coords(tile, num_m, num_n, n_fastest, tm, tn);
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1, wait_limit, abort_flag, SITE_GEMM2_PRODUCER)) {
             ok = false;
@@ -467,7 +488,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
           }
           if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * STAGE_BYTES);
           const uint32_t leader_full = mapa_shared(smem_u32(&full[stage]), 0);
-          tma_load_2d_pair(sA + stage * A_BYTES, &tmA, leader_full, kb * BK, tm * BM + (int)rank * BM_CTA);
+          if (n_fastest)
+            tma_load_2d_pair_hint(sA + stage * A_BYTES, &tmA, leader_full, kb * BK, tm * BM + (int)rank * BM_CTA,
+                                  a_policy);
+          else
+            tma_load_2d_pair(sA + stage * A_BYTES, &tmA, leader_full, kb * BK, tm * BM + (int)rank * BM_CTA);
           tma_load_2d_pair(sB + stage * B_BYTES, &tmB, leader_full, kb * BK, tn * BN + (int)rank * BN_CTA);
           issued_mask |= 1u << stage;
           issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
@@ -540,7 +565,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = cluster_id; tile < num_tiles; tile += n_clusters) {
-      const int tm = tile % num_m, tn = tile / num_m;
+      int tm, tn;
+      tile_coords(tile, num_m, num_n, n_fastest, tm, tn);
       bool ok = mbar_wait(&tfull[acc], acc_phase, wait_limit, abort_flag, SITE_GEMM2_EPILOGUE);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();

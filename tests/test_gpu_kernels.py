@@ -8,7 +8,7 @@ import pytest
 from oracle import dit_oracle as O
 from diffusion_transformer_block_flux_b200 import synth
 import diffusion_transformer_block_flux_b200 as dit
-from helpers import dev_bf16, host_f64, parity
+from helpers import dev_bf16, dev_tree, host_f64, parity
 
 pytestmark = pytest.mark.gpu
 
