@@ -106,27 +106,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64
   return mbar_wait_slow(bar, parity, limit_ns, abort, site);
 }
 
-// The same bounded wait with the slow path inlined, for kernels that give
-// their warpgroups different register counts (setmaxnreg): ptxas cannot
-// allocate a called function that is reached under two register limits.
-__device__ __forceinline__ bool mbar_wait_inl(uint64_t* bar, uint32_t parity, uint64_t limit_ns,
-                                              volatile int* abort, uint32_t site) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  uint32_t n = 0;
-  while (!mbar_try_wait(bar, parity)) {
-    if ((++n & 255u) == 0) {
-      if (abort != nullptr && *abort) return false;
-      if (globaltimer_ns() - t0 > limit_ns) {
-        atomicCAS(&g_dit_error, 0u, (uint32_t)DIT_ERR_TIMEOUT | (site << 8));
-        if (abort != nullptr) *abort = 1;
-        return false;
-      }
-    }
-  }
-  return true;
-}
-
 // ---------------------------------------------------------------------------
 // TMA (cp.async.bulk.tensor), no multicast
 // ---------------------------------------------------------------------------
