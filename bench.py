@@ -645,9 +645,11 @@ def run_video(args):
 def run_ring8(args):
     """One rank's compute in a CP=8 ring over the Flux sequence (4608 tokens
     = 8 x 576 per rank, 24 heads x 128), on one GPU: attention of the 576 local
-    queries against each of the 8 key/value shards plus 7 in-place
-    log-sum-exp merges, captured as one CUDA graph (the transfers between
-    ranks are not part of this single-GPU measurement)."""
+    queries against the 8 key/value shards, each step after the first merged
+    into the running result in its epilogue (dit_attention_accumulate),
+    captured as one CUDA graph (the transfers between ranks are not part of
+    this single-GPU measurement).  G shards per attention step: G = 1 is the
+    ring (8 launches), G = 8 gathers every shard first (1 launch)."""
     import torch
     import diffusion_transformer_block_flux_b200 as dit
     dev = torch.device("cuda", 0)
@@ -658,37 +660,39 @@ def run_ring8(args):
     q = [_rand(torch, g, dev, Sl, D) for _ in range(NB)]
     kv = [_rand(torch, g, dev, 2, S, D) for _ in range(NB)]
     o = torch.empty((Sl, D), dtype=torch.bfloat16, device=dev)
-    part = torch.empty_like(o)
     lse = torch.empty((1, H, Sl), dtype=torch.float32, device=dev)
-    lpart = torch.empty_like(lse)
+    K = max(5, args.steps // 4)
+    flops = 4.0 * Sl * S * H * 128
+    per_g = {}
+    for G in (1, 2, 4, 8):
+        def ring(i, G=G):
+            k, v = kv[i][0], kv[i][1]
+            for j in range(0, N, G):
+                ks, vs = k[j * Sl:(j + G) * Sl], v[j * Sl:(j + G) * Sl]
+                if j == 0:
+                    dit.dit_attention(q[i], ks, vs, o, 1, Sl, G * Sl, H, lse=lse)
+                else:
+                    dit.dit_attention_accumulate(q[i], ks, vs, o, lse, 1, Sl, G * Sl, H)
 
-    def ring(i):
-        k, v = kv[i][0], kv[i][1]
-        for j in range(N):
-            ks, vs = k[j * Sl:(j + 1) * Sl], v[j * Sl:(j + 1) * Sl]
-            if j == 0:
-                dit.dit_attention(q[i], ks, vs, o, 1, Sl, Sl, H, lse=lse)
-            else:
-                dit.dit_attention(q[i], ks, vs, part, 1, Sl, Sl, H, lse=lpart)
-                dit.dit_attention_merge([o, part], [lse, lpart], o, lse, 1, Sl, H)
-
-    for i in range(NB):
-        ring(i)
-    torch.cuda.synchronize()
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph):
         for i in range(NB):
             ring(i)
-    K = max(5, args.steps // 4)
-    ms = _event_time(torch, graph.replay, K, 3, torch.cuda.current_stream()) / NB
-    del graph
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            for i in range(NB):
+                ring(i)
+        ms = _event_time(torch, graph.replay, K, 3, torch.cuda.current_stream()) / NB
+        del graph
+        tf = flops / (ms * 1e-3) / 1e12
+        per_g[G] = {"ms": round(ms, 4), "tflops": round(tf, 1), "frac_of_bf16_peak": round(tf / peaks()["bf16_tflops"], 4),
+                    "launches": N // G}
     st, code = dit.dit_get_device_error()
     if st != 0:
         raise RuntimeError(f"device error word {code:#x}")
-    flops = 4.0 * Sl * S * H * 128
-    return _extra_line("ring_cp8_rank_compute_S4608_576q_24x128", ms, flops, K * NB, 3,
-                       {"us_per_hop": round(ms * 1e3 / N, 2), "hops": N, "merges": N - 1,
-                        "gpu_launches_per_step": 2 * N - 1,
+    ms1 = per_g[1]["ms"]
+    return _extra_line("ring_cp8_rank_compute_S4608_576q_24x128", ms1, flops, K * NB, 3,
+                       {"us_per_hop": round(ms1 * 1e3 / N, 2), "hops": N, "gpu_launches_per_step": N,
+                        "shards_per_step": per_g,
                         "context": "the compile_graph page, section 5: one attention segment of the 8-card ring "
                                    "took 0.073 ms on H20"})
 

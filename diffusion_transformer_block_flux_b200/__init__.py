@@ -128,6 +128,8 @@ _SIGS = {
                                i64, i32, i32, i32, i32, f32, c_void_p]),
     "dit_attention": (i32, [c_void_p, c_void_p, c_void_p, i64, i64, i64, c_void_p, i64, c_void_p, i32, i32,
                             i32, i32, i32, f32, c_void_p]),
+    "dit_attention_accumulate": (i32, [c_void_p, c_void_p, c_void_p, i64, i64, i64, c_void_p, i64, c_void_p, i32,
+                                       i32, i32, i32, i32, f32, c_void_p]),
     "dit_gemm_epilogue": (i32, [ctypes.POINTER(dit_gemm_args), c_void_p]),
     "dit_selftest_exp2_poly": (i32, [c_void_p, c_void_p, i64, c_void_p]),
     "dit_attention_merge": (i32, [i32, ctypes.POINTER(c_void_p), ctypes.POINTER(c_void_p), i64, c_void_p, c_void_p,
@@ -290,6 +292,14 @@ def dit_attention(q, k, v, o, B, Sq, Skv, H, softmax_scale=None, lse=None, strea
     if softmax_scale is None:
         softmax_scale = 128 ** -0.5
     _call("dit_attention", _ptr(q), _ptr(k), _ptr(v), q.stride(0), k.stride(0), v.stride(0), _ptr(o),
+          o.stride(0), _ptr(lse), B, Sq, Skv, H, 128, float(softmax_scale), _stream(stream))
+
+
+def dit_attention_accumulate(q, k, v, o, lse, B, Sq, Skv, H, softmax_scale=None, stream=None):
+    """Merge attention(q, k, v) into the running result (o, lse) in place (one ring hop)."""
+    if softmax_scale is None:
+        softmax_scale = 128 ** -0.5
+    _call("dit_attention_accumulate", _ptr(q), _ptr(k), _ptr(v), q.stride(0), k.stride(0), v.stride(0), _ptr(o),
           o.stride(0), _ptr(lse), B, Sq, Skv, H, 128, float(softmax_scale), _stream(stream))
 
 

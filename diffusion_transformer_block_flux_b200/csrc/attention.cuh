@@ -5,19 +5,22 @@
 // 4608-token text|image sequence, 24 heads x 128, bf16, run by a flash
 // backend; §6.3 — operands laid out (B, S, H, D).  No mask.
 //
-// One CTA = one (batch, head) and two 128-row query tiles Q0, Q1 that
-// ping-pong: while one softmax warpgroup turns its score tile into
-// probabilities, the tensor core computes the other tile's scores and PV.
+// One CTA = one (batch, head) and two 128-row query tiles Q0, Q1.
 //   warps 0-3  softmax + epilogue for Q0 (thread = query row = TMEM lane)
 //   warps 4-7  softmax + epilogue for Q1
 //   warp 8     TMA producer: Q0, Q1 once; K_j, V_j through 2-stage rings
 //   warp 9     TMEM allocator + single-thread MMA issuer
-// TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,384) O1 [384,512).
-// P_k (bf16 pairs) overwrites the first 64 columns of S_k after the softmax
-// has read S_k into registers; the next S_k MMA is issued after the PV MMA
-// that reads P_k, and tcgen05 MMAs of one CTA execute in issue order.
-// A commit after S_k(j+1) therefore also covers PV_k(j): once a softmax
-// warpgroup sees S_k(j+1), O_k is stable and may be rescaled in place.
+// TMEM (512 columns): S [0,128) shared by both tiles, P0 [128,192),
+// P1 [192,256) (bf16 pairs), O0 [256,384), O1 [384,512).
+// The score tile S is the only buffer the two tiles share, and a tile's
+// softmax holds it only until its scores are in registers: it then frees S
+// (s_free) and the MMA issuer computes the other tile's next scores into it
+// while the exponentials run.  P_t has its own columns, so the PV product of
+// step j and the scores of step j + 1 never wait for each other; a tile
+// only waits for its previous PV (p_free) before writing P_t again or
+// rescaling O_t.  Each tile's softmax warps therefore run back to back, and
+// the tensor core works through QK0 QK1 PV0 PV1 per key tile in the order
+//   QK0(j+1), PV0(j), QK1(j+1), PV1(j).
 #pragma once
 
 #include "common.cuh"
@@ -37,6 +40,7 @@ constexpr int OFF_V = 4 * TILE_BYTES;           // V[2]
 constexpr int OFF_BAR = 6 * TILE_BYTES;
 constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;
 constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t COL_S = 0, COL_P = 128, COL_O = 256;  // P_t at COL_P + 64 t, O_t at COL_O + 128 t
 constexpr uint32_t IDESC_QK = idesc_bf16(128, 128, 0, 0);  // Q, K both K-major (d contiguous)
 constexpr uint32_t IDESC_PV = idesc_bf16(128, 128, 0, 1);  // P from TMEM, V MN-major (d contiguous)
 
@@ -46,6 +50,9 @@ struct Params {
   float* lse;
   int Sq, Skv, H;
   float scale_log2;  // softmax_scale * log2(e)
+  // 1: o and lse hold a running result over other keys on entry; this
+  // launch's result is merged into it by log-sum-exp (a ring hop)
+  int accumulate;
 };
 
 __global__ void __launch_bounds__(NUM_THREADS, 1)
@@ -59,11 +66,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* k_empty = bars + 3;  // [2]
   uint64_t* v_full = bars + 5;   // [2]
   uint64_t* v_empty = bars + 7;  // [2]
-  uint64_t* s_full = bars + 9;   // [2]
-  uint64_t* p_full = bars + 11;  // [2]
-  uint64_t* o_full = bars + 13;  // [2]
-  uint64_t* drain = bars + 15;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  uint64_t* s_full = bars + 9;   // [2] scores of tile t are in S
+  uint64_t* s_free = bars + 11;  // the tile that last received S has loaded it
+  uint64_t* p_full = bars + 12;  // [2] P_t written
+  uint64_t* p_free = bars + 14;  // [2] the PV that read P_t is done (O_t stable)
+  uint64_t* o_full = bars + 16;  // [2]
+  uint64_t* drain = bars + 18;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 19);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -82,8 +91,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(&v_empty[s], 1);
       mbar_init(&s_full[s], 1);
       mbar_init(&p_full[s], 4);  // one arrival per softmax warp of the tile
+      mbar_init(&p_free[s], 1);
       mbar_init(&o_full[s], 1);
     }
+    mbar_init(s_free, 4);  // the four warps of the tile that loaded S
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -144,12 +155,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const uint32_t sQ0 = smem_u32(smem + OFF_Q);
       bool ok = true;
       bool issued = false;
+      uint32_t sfree_ph = 0;  // parity of the next s_free phase
       auto issue_qk = [&](int t, int kst) {
         const uint32_t kb = smem_u32(smem + OFF_K + kst * TILE_BYTES);
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
           const uint32_t off = (uint32_t)((kk >> 2) * HALF_BYTES + (kk & 3) * 32);
-          umma_ss(tmem_base + (uint32_t)(t * 128), sdesc_sw128(sQ0 + (uint32_t)(t * TILE_BYTES) + off, 16, 1024),
+          umma_ss(tmem_base + COL_S, sdesc_sw128(sQ0 + (uint32_t)(t * TILE_BYTES) + off, 16, 1024),
                   sdesc_sw128(kb + off, 16, 1024), IDESC_QK, kk > 0 ? 1u : 0u);
         }
       };
@@ -159,20 +171,30 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int kk = 0; kk < BKV / 16; ++kk) {
           // A: P_t in TMEM, 16 keys = 8 columns of bf16 pairs.
           // B: V MN-major; 64-d halves HALF_BYTES apart (LBO), 8-key groups 1024 B apart (SBO).
-          umma_ts(tmem_base + 256u + (uint32_t)(t * 128), tmem_base + (uint32_t)(t * 128 + kk * 8),
+          umma_ts(tmem_base + COL_O + (uint32_t)(t * 128), tmem_base + COL_P + (uint32_t)(t * 64 + kk * 8),
                   sdesc_sw128(vb + (uint32_t)(kk * 2048), HALF_BYTES, 1024), IDESC_PV, (acc || kk > 0) ? 1u : 0u);
         }
       };
+      auto wait_sfree = [&]() -> bool {
+        const bool r = mbar_wait(s_free, sfree_ph, wait_limit, abort_flag, SITE_ATTN_MMA);
+        sfree_ph ^= 1u;
+        return r;
+      };
+      // prologue: S <- Q0 K_0, then (once tile 0 has loaded it) S <- Q1 K_0
       if (!mbar_wait(q_full, 0, wait_limit, abort_flag, SITE_ATTN_MMA)) ok = false;
       if (ok && !mbar_wait(&k_full[0], 0, wait_limit, abort_flag, SITE_ATTN_MMA)) ok = false;
       if (ok) {
         tc_fence_after();
         issue_qk(0, 0);
         umma_commit(&s_full[0]);
+        issued = true;
+      }
+      if (ok && !wait_sfree()) ok = false;
+      if (ok) {
+        tc_fence_after();
         issue_qk(1, 0);
         umma_commit(&s_full[1]);
         umma_commit(&k_empty[0]);
-        issued = true;
       }
       for (int j = 0; j < n_kv && ok; ++j) {
         const int st = j & 1;
@@ -180,25 +202,30 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const bool has_next = j + 1 < n_kv;
         const int nst = (j + 1) & 1;
         const uint32_t nph = ((j + 1) >> 1) & 1;
-        if (!mbar_wait(&v_full[st], ph, wait_limit, abort_flag, SITE_ATTN_MMA)) { ok = false; break; }
-        if (!mbar_wait(&p_full[0], j & 1, wait_limit, abort_flag, SITE_ATTN_MMA)) { ok = false; break; }
-        tc_fence_after();
-        issue_pv(0, st, j > 0);
-        if (has_next) {
+        if (has_next) {  // S <- Q0 K_{j+1} once tile 1 has loaded its scores of key tile j
+          if (!wait_sfree()) { ok = false; break; }
           if (!mbar_wait(&k_full[nst], nph, wait_limit, abort_flag, SITE_ATTN_MMA)) { ok = false; break; }
           tc_fence_after();
           issue_qk(0, nst);
           umma_commit(&s_full[0]);
         }
-        if (!mbar_wait(&p_full[1], j & 1, wait_limit, abort_flag, SITE_ATTN_MMA)) { ok = false; break; }
+        if (!mbar_wait(&v_full[st], ph, wait_limit, abort_flag, SITE_ATTN_MMA)) { ok = false; break; }
+        if (!mbar_wait(&p_full[0], j & 1, wait_limit, abort_flag, SITE_ATTN_MMA)) { ok = false; break; }
         tc_fence_after();
-        issue_pv(1, st, j > 0);
-        umma_commit(&v_empty[st]);
-        if (has_next) {
+        issue_pv(0, st, j > 0);
+        umma_commit(&p_free[0]);
+        if (has_next) {  // S <- Q1 K_{j+1} once tile 0 has loaded its scores of key tile j+1
+          if (!wait_sfree()) { ok = false; break; }
+          tc_fence_after();
           issue_qk(1, nst);
           umma_commit(&s_full[1]);
           umma_commit(&k_empty[nst]);
         }
+        if (!mbar_wait(&p_full[1], j & 1, wait_limit, abort_flag, SITE_ATTN_MMA)) { ok = false; break; }
+        tc_fence_after();
+        issue_pv(1, st, j > 0);
+        umma_commit(&p_free[1]);
+        umma_commit(&v_empty[st]);
       }
       if (ok) {
         umma_commit(&o_full[0]);
@@ -214,8 +241,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int quad = warp & 3;        // TMEM lane quadrant
     const int row = quad * 32 + lane; // query row within the tile
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-    const uint32_t tS = tmem_base + lane_off + (uint32_t)(t * 128);
-    const uint32_t tO = tmem_base + lane_off + 256u + (uint32_t)(t * 128);
+    const uint32_t tS = tmem_base + lane_off + COL_S;
+    const uint32_t tP = tmem_base + lane_off + COL_P + (uint32_t)(t * 64);
+    const uint32_t tO = tmem_base + lane_off + COL_O + (uint32_t)(t * 128);
     const float sl2 = p.scale_log2;
     // Running max of the scaled logits (log2 units).  It is raised lazily:
     // only when a tile's max exceeds it by more than 8, so P stays <= 2^8 and
@@ -238,6 +266,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       reg_fence32(r[1]);
       reg_fence32(r[2]);
       reg_fence32(r[3]);
+      // the scores are in registers: S may take the other tile's next scores
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(s_free);
       const int valid = p.Skv - j * BKV;  // keys of this tile that exist
       if (valid < BKV) {
 #pragma unroll
@@ -262,9 +294,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const uint64_t sl2x2 = f2_pack(sl2, sl2);
       const uint64_t negx2 = f2_pack(-m_new, -m_new);
       uint64_t sum2[2] = {0ull, 0ull};  // packed (even, odd) partial sums, two chains
+      uint32_t pk[4][16];
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           // x = s * scale * log2(e) - m for the pair (2i, 2i+1): one packed FMA
@@ -276,14 +308,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             pp = f2_pack(ex2_fast(f2_lo(x)), ex2_fast(f2_hi(x)));
           }
           sum2[i & 1] = f2_add(sum2[i & 1], pp);
-          pk[i] = pack_bf16x2(f2_lo(pp), f2_hi(pp));
+          pk[c][i] = pack_bf16x2(f2_lo(pp), f2_hi(pp));
         }
-        tmem_st16(tS + (uint32_t)(c * 16), pk);
       }
       const uint64_t st2 = f2_add(sum2[0], sum2[1]);
       l_run = l_run * alpha + (f2_lo(st2) + f2_hi(st2));
-      // Rescale O_t when any row of this warp raised its max (O_t is stable:
-      // the commit we waited on covers the previous PV into O_t).
+      // P_t and O_t are free once the previous PV of this tile is done
+      if (j > 0) {
+        ok = mbar_wait(&p_free[t], (j - 1) & 1, wait_limit, abort_flag, SITE_ATTN_SOFTMAX);
+        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+        tc_fence_after();
+      }
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_st16(tP + (uint32_t)(c * 16), pk[c]);
+      // Rescale O_t when any row of this warp raised its max
       if (j > 0 && __any_sync(0xffffffffu, need)) {
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
@@ -307,27 +345,56 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (ok) {
       tc_fence_after();
       const int qi = q_row0 + t * BQ + row;
-      const float inv_l = 1.0f / l_run;
+      const bool live = qi < p.Sq;
       bf16* orow = p.o + ((int64_t)batch * p.Sq + qi) * p.ldo + head * HD;
+      const int64_t li = ((int64_t)batch * p.H + head) * p.Sq + qi;
+      const float lse_cur = (m_run + __log2f(l_run)) * 0.6931471805599453f;  // natural log
+      // o = w_prev o_prev + w_cur (O / l): w_prev = 0, w_cur = 1 unless accumulating
+      float w_prev = 0.0f, w_cur = 1.0f / l_run, lse_new = lse_cur;
+      if (p.accumulate && live) {
+        const float lse_prev = p.lse[li];  // -inf: nothing accumulated yet
+        const float mx = fmaxf(lse_prev, lse_cur);
+        const float ep = __expf(lse_prev - mx), ec = __expf(lse_cur - mx);
+        const float inv = 1.0f / (ep + ec);
+        lse_new = mx + __logf(ep + ec);
+        w_prev = ep * inv;
+        w_cur *= ec * inv;
+      }
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
         uint32_t r[32];
         tmem_ld32(tO + (uint32_t)(c * 32), r);
-        if (qi < p.Sq) {
+        if (live) {
           uint4* dp = reinterpret_cast<uint4*>(orow + c * 32);
+          float pv[32];
+          if (p.accumulate) {  // this thread's own row: read before it is written
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const uint4 u = dp[q];
+              pv[8 * q + 0] = bf16_lo(u.x); pv[8 * q + 1] = bf16_hi(u.x);
+              pv[8 * q + 2] = bf16_lo(u.y); pv[8 * q + 3] = bf16_hi(u.y);
+              pv[8 * q + 4] = bf16_lo(u.z); pv[8 * q + 5] = bf16_hi(u.z);
+              pv[8 * q + 6] = bf16_lo(u.w); pv[8 * q + 7] = bf16_hi(u.w);
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) pv[i] = 0.0f;
+          }
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
+            float o8[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) o8[i] = fmaf(__uint_as_float(r[8 * q + i]), w_cur, w_prev * pv[8 * q + i]);
             uint4 w;
-            w.x = pack_bf16x2(__uint_as_float(r[8 * q + 0]) * inv_l, __uint_as_float(r[8 * q + 1]) * inv_l);
-            w.y = pack_bf16x2(__uint_as_float(r[8 * q + 2]) * inv_l, __uint_as_float(r[8 * q + 3]) * inv_l);
-            w.z = pack_bf16x2(__uint_as_float(r[8 * q + 4]) * inv_l, __uint_as_float(r[8 * q + 5]) * inv_l);
-            w.w = pack_bf16x2(__uint_as_float(r[8 * q + 6]) * inv_l, __uint_as_float(r[8 * q + 7]) * inv_l);
+            w.x = pack_bf16x2(o8[0], o8[1]);
+            w.y = pack_bf16x2(o8[2], o8[3]);
+            w.z = pack_bf16x2(o8[4], o8[5]);
+            w.w = pack_bf16x2(o8[6], o8[7]);
             dp[q] = w;
           }
         }
       }
-      if (p.lse != nullptr && qi < p.Sq)
-        p.lse[((int64_t)batch * p.H + head) * p.Sq + qi] = (m_run + __log2f(l_run)) * 0.6931471805599453f;
+      if (p.lse != nullptr && live) p.lse[li] = lse_new;
     }
   }
 

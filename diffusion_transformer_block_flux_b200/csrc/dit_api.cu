@@ -316,15 +316,19 @@ dit_status dit_vec_linear(const dit_bf16* x, int64_t ldx, const dit_bf16* W, int
   const bf16* xb = reinterpret_cast<const bf16*>(x);
   const bf16* Wb = reinterpret_cast<const bf16*>(W);
   const bf16* bb = reinterpret_cast<const bf16*>(bias);
-  if (B == 1 && (K % 256) == 0 && K <= 3072) {
-    // one warp per weight row, two rows in flight per warp, 16 warps per CTA
-    const int64_t warps = (int64_t)sms * kVecRowsCtasPerSm * 16;
+  if (B <= 2 && (K % 256) == 0 && K <= 3072) {
+    // one warp per weight row, 16 warps per CTA, one CTA per SM
     int64_t grid = (int64_t)sms * kVecRowsCtasPerSm;
-    if (N < warps) grid = (N + 15) / 16;
-    const size_t xs_smem = (size_t)K * 4;
-#define DIT_VR_CASE(KC_)                                                                                  \
-  case KC_:                                                                                               \
-    dit::vec_rows_kernel<KC_><<<(unsigned)grid, 512, xs_smem, st>>>(xb, Wb, ldw, bb, out, N, K, flags);    \
+    if (N < grid * 16) grid = (N + 15) / 16;
+    const size_t xs_smem = (size_t)B * K * 4;
+#define DIT_VR_CASE(KC_)                                                                                       \
+  case KC_:                                                                                                    \
+    if (B == 1)                                                                                                \
+      dit::vec_rows_kernel<KC_, 1><<<(unsigned)grid, 512, xs_smem, st>>>(xb, ldx, Wb, ldw, bb, out, ldo, N, K, \
+                                                                         flags);                               \
+    else                                                                                                       \
+      dit::vec_rows_kernel<KC_, 2><<<(unsigned)grid, 512, xs_smem, st>>>(xb, ldx, Wb, ldw, bb, out, ldo, N, K, \
+                                                                         flags);                               \
     return launch_status();
     switch (K / 256) {
       DIT_VR_CASE(1)
@@ -525,9 +529,13 @@ dit_status dit_qk_norm_rope(const dit_bf16* q, const dit_bf16* k, int64_t ld_in,
                    (cudaStream_t)stream);
 }
 
-dit_status dit_attention(const dit_bf16* q, const dit_bf16* k, const dit_bf16* v, int64_t ldq, int64_t ldk,
-                         int64_t ldv, dit_bf16* o, int64_t ldo, float* lse, int B, int Sq, int Skv, int H,
-                         int head_dim, float softmax_scale, void* stream) {
+}  // extern "C"
+
+namespace {
+
+dit_status attention_launch(const dit_bf16* q, const dit_bf16* k, const dit_bf16* v, int64_t ldq, int64_t ldk,
+                            int64_t ldv, dit_bf16* o, int64_t ldo, float* lse, int B, int Sq, int Skv, int H,
+                            int head_dim, float softmax_scale, int accumulate, void* stream) {
   if (q == nullptr || k == nullptr || v == nullptr || o == nullptr) return DIT_ERR_INVALID_ARG;
   if (head_dim != 128) return DIT_ERR_UNSUPPORTED;
   if (B < 1 || Sq < 1 || Skv < 1 || H < 1 || B > 65535 || H > 65535) return DIT_ERR_SHAPE;
@@ -550,10 +558,28 @@ dit_status dit_attention(const dit_bf16* q, const dit_bf16* k, const dit_bf16* v
   p.Skv = Skv;
   p.H = H;
   p.scale_log2 = softmax_scale * 1.4426950408889634f;
+  p.accumulate = accumulate;
   dim3 grid((unsigned)((Sq + 2 * dit::attn::BQ - 1) / (2 * dit::attn::BQ)), (unsigned)H, (unsigned)B);
   dit::attn::attention_kernel<<<grid, dit::attn::NUM_THREADS, dit::attn::SMEM_BYTES, (cudaStream_t)stream>>>(
       tq, tk, tv, p, g_wait_limit_ns);
   return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+dit_status dit_attention(const dit_bf16* q, const dit_bf16* k, const dit_bf16* v, int64_t ldq, int64_t ldk,
+                         int64_t ldv, dit_bf16* o, int64_t ldo, float* lse, int B, int Sq, int Skv, int H,
+                         int head_dim, float softmax_scale, void* stream) {
+  return attention_launch(q, k, v, ldq, ldk, ldv, o, ldo, lse, B, Sq, Skv, H, head_dim, softmax_scale, 0, stream);
+}
+
+dit_status dit_attention_accumulate(const dit_bf16* q, const dit_bf16* k, const dit_bf16* v, int64_t ldq,
+                                    int64_t ldk, int64_t ldv, dit_bf16* o, int64_t ldo, float* lse, int B, int Sq,
+                                    int Skv, int H, int head_dim, float softmax_scale, void* stream) {
+  if (lse == nullptr) return DIT_ERR_INVALID_ARG;
+  return attention_launch(q, k, v, ldq, ldk, ldv, o, ldo, lse, B, Sq, Skv, H, head_dim, softmax_scale, 1, stream);
 }
 
 dit_status dit_attention_merge(int n, const dit_bf16* const* o_parts, const float* const* lse_parts, int64_t ld_in,

@@ -211,14 +211,18 @@ __global__ void __launch_bounds__(256) modulate_norm_row_kernel(const bf16* __re
 }
 
 // ---------------------------------------------------------------------------
-// Vector x weight rows (adaLN modulation, the timestep MLP), batch 1,
+// Vector x weight rows (adaLN modulation, the timestep MLP), batch NB <= 2,
 // K = 256 KC: one warp per output row, lane l reading the 16-byte chunks
-// l, l + 32, ... of the row with streaming loads, the (mapped) input vector
-// in shared memory as fp32.  A warp issues the loads of its next row as soon
-// as a row is reduced, and keeps two rows in flight for K <= 1536; rows are
-// dealt to the warps of a persistent grid round robin.  RowFn(n) gives row n's weight
-// pointer, bias and output slot, so the same loop serves one matrix and a
-// list of matrices that share the input (every block's modulation of a step).
+// l, l + 32, ... of the row with streaming loads, the (mapped) input vectors
+// in shared memory as fp32.  They are stored lane-interleaved: the 8 values
+// lane l needs for chunk c sit as float4 [c][l] (first 4) and [c][32 + l]
+// (last 4), so a warp's shared-memory reads are contiguous (no bank
+// conflicts).  A warp issues the loads of its next row as soon as a row is
+// reduced, and keeps two rows in flight while the registers allow it; rows
+// are dealt to the warps of a persistent grid round robin.  RowFn(n) gives
+// row n's weight pointer, bias and output slot, so the same loop serves one
+// matrix and a list of matrices that share the input (every block's
+// modulation of a step).
 // ---------------------------------------------------------------------------
 struct VecRow {
   const uint4* w;
@@ -234,13 +238,13 @@ __device__ __forceinline__ void vr_load(uint4 (&u)[KC], float& bv, const VecRow&
   bv = (on && lane == 0 && rw.bias != nullptr) ? __bfloat162float(rw.bias[rw.local]) : 0.0f;
 }
 
+// dot products of the row held in u with input vector b (interleaved layout, 64 float4 per chunk)
 template <int KC>
 __device__ __forceinline__ float vr_dot(const uint4 (&u)[KC], const float4* __restrict__ xs, int lane) {
   float a0 = 0.f, a1 = 0.f;
 #pragma unroll
   for (int c = 0; c < KC; ++c) {
-    const int k = (c * 32 + lane) * 2;
-    const float4 x0 = xs[k], x1 = xs[k + 1];
+    const float4 x0 = xs[c * 64 + lane], x1 = xs[c * 64 + 32 + lane];
     a0 = fmaf(bf16_lo(u[c].x), x0.x, a0); a1 = fmaf(bf16_hi(u[c].x), x0.y, a1);
     a0 = fmaf(bf16_lo(u[c].y), x0.z, a0); a1 = fmaf(bf16_hi(u[c].y), x0.w, a1);
     a0 = fmaf(bf16_lo(u[c].z), x1.x, a0); a1 = fmaf(bf16_hi(u[c].z), x1.y, a1);
@@ -249,11 +253,11 @@ __device__ __forceinline__ float vr_dot(const uint4 (&u)[KC], const float4* __re
   return warp_sum(a0 + a1);
 }
 
-template <int KC, typename RowFn, typename OutFn>
-__device__ __forceinline__ void vec_rows_loop(const bf16* __restrict__ x, int K, int flags, int64_t N, RowFn row_of,
-                                              OutFn store) {
-  constexpr bool TWO = KC <= 6;  // two rows in flight per warp while the registers allow it
-  extern __shared__ float4 xs4[];  // the mapped input, K fp32
+template <int KC, int NB, typename RowFn, typename OutFn>
+__device__ __forceinline__ void vec_rows_loop(const bf16* __restrict__ x, int64_t ldx, int K, int flags, int64_t N,
+                                              RowFn row_of, OutFn store) {
+  constexpr bool TWO = KC * NB <= 6;  // two rows in flight per warp while the registers allow it
+  extern __shared__ float4 xs4[];  // NB mapped inputs, K fp32 each, lane-interleaved
   float* xs = reinterpret_cast<float*>(xs4);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t nw = (int64_t)gridDim.x * (blockDim.x >> 5);
@@ -267,22 +271,31 @@ __device__ __forceinline__ void vec_rows_loop(const bf16* __restrict__ x, int K,
     rb = row_of(n + nw < N ? n + nw : 0);
     vr_load<KC>(ub, bb, rb, n + nw < N, lane);
   }
-  for (int k = threadIdx.x; k < K; k += blockDim.x) {
-    float z = __bfloat162float(x[k]);
+  for (int i = threadIdx.x; i < NB * K; i += blockDim.x) {
+    const int b = i / K, k = i - b * K;
+    float z = __bfloat162float(x[b * ldx + k]);
     if (flags & DIT_VEC_SILU_IN) z = silu(z);
-    xs[k] = z;
+    // column k = 8 (32 c + l) + j sits in float4 [c][l] (j < 4) or [c][32 + l] (j >= 4)
+    const int c = k >> 8, l = (k >> 3) & 31, j = k & 7;
+    xs[b * K + ((c * 64 + (j >> 2) * 32 + l) << 2) + (j & 3)] = z;
   }
   __syncthreads();
   for (; n < N; n += step) {
-    const float da = vr_dot<KC>(ua, xs4, lane) + ba;
-    if (lane == 0) store(ra, da);
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      const float da = vr_dot<KC>(ua, xs4 + b * (K / 4), lane) + ba;
+      if (lane == 0) store(ra, b, da);
+    }
     const int64_t n2 = n + step;
     ra = row_of(n2 < N ? n2 : 0);
     vr_load<KC>(ua, ba, ra, n2 < N, lane);
     if constexpr (TWO) {
       if (n + nw < N) {
-        const float db = vr_dot<KC>(ub, xs4, lane) + bb;
-        if (lane == 0) store(rb, db);
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+          const float db = vr_dot<KC>(ub, xs4 + b * (K / 4), lane) + bb;
+          if (lane == 0) store(rb, b, db);
+        }
       }
       const int64_t n3 = n + nw + step;
       rb = row_of(n3 < N ? n3 : 0);
@@ -291,18 +304,19 @@ __device__ __forceinline__ void vec_rows_loop(const bf16* __restrict__ x, int K,
   }
 }
 
-template <int KC>
-__global__ void __launch_bounds__(512, 1) vec_rows_kernel(const bf16* __restrict__ x, const bf16* __restrict__ W,
-                                                       int64_t ldw, const bf16* __restrict__ bias, void* out,
-                                                       int64_t N, int K, int flags) {
-  vec_rows_loop<KC>(
-      x, K, flags, N,
+template <int KC, int NB>
+__global__ void __launch_bounds__(512, 1) vec_rows_kernel(const bf16* __restrict__ x, int64_t ldx,
+                                                          const bf16* __restrict__ W, int64_t ldw,
+                                                          const bf16* __restrict__ bias, void* out, int64_t ldo,
+                                                          int64_t N, int K, int flags) {
+  vec_rows_loop<KC, NB>(
+      x, ldx, K, flags, N,
       [=](int64_t n) { return VecRow{reinterpret_cast<const uint4*>(W + n * ldw), bias, n, 0}; },
-      [=](const VecRow& rw, float v) {
+      [=](const VecRow& rw, int b, float v) {
         if (flags & DIT_VEC_OUT_BF16)
-          reinterpret_cast<bf16*>(out)[rw.local] = __float2bfloat16_rn(v);
+          reinterpret_cast<bf16*>(out)[b * ldo + rw.local] = __float2bfloat16_rn(v);
         else
-          reinterpret_cast<float*>(out)[rw.local] = v;
+          reinterpret_cast<float*>(out)[b * ldo + rw.local] = v;
       });
 }
 
@@ -496,19 +510,19 @@ __global__ void __launch_bounds__(128) vec_linear_multi_kernel(const bf16* __res
   cp_async_wait<0>();
 }
 
-// Every matrix of p in one pass with the loop above (one warp per row, two
-// rows in flight); out[j][n - row_begin[j]] = W_j[row] . f(x) + bias_j[row].
+// Every matrix of p in one pass with the loop above (one warp per row);
+// out[j][n - row_begin[j]] = W_j[row] . f(x) + bias_j[row].
 template <int KC>
 __global__ void __launch_bounds__(512, 1) vec_rows_multi_kernel(const bf16* __restrict__ x,
                                                              const __grid_constant__ MultiLinear p, int flags) {
-  vec_rows_loop<KC>(
-      x, p.K, flags, (int64_t)p.row_begin[p.n_mats],
+  vec_rows_loop<KC, 1>(
+      x, 0, p.K, flags, (int64_t)p.row_begin[p.n_mats],
       [&](int64_t n) {
         const int j = multi_find(p, n);
         const int64_t local = n - p.row_begin[j];
         return VecRow{reinterpret_cast<const uint4*>(p.W[j] + local * p.K), p.bias[j], local, j};
       },
-      [&](const VecRow& rw, float v) { p.out[rw.mat][rw.local] = v; });
+      [&](const VecRow& rw, int, float v) { p.out[rw.mat][rw.local] = v; });
 }
 
 // ---------------------------------------------------------------------------

@@ -474,13 +474,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       uint32_t phase = 0;
       uint32_t issued_mask = 0, issued_parity = 0;
       bool ok = true;
-      // N-fastest: each A panel is consumed by the clusters of one wave and
-      // not needed again, so it is loaded as evict-first and the weight
-      // panels that every wave re-reads stay in L2
-      const uint64_t a_policy = l2_policy_evict_first();
-      for (int tile = cluster_id; tile < num_tiles && ok; tile += n_clusters) {
+      int wave = 0;  // this cluster's tile count so far: the same for every cluster of a wave
+      for (int tile = cluster_id; tile < num_tiles && ok; tile += n_clusters, ++wave) {
         int tm, tn;
         tile_coords(tile, num_m, num_n, n_fastest, tm, tn);
+        // N-fastest: every other wave walks K backwards, so that it starts on the
+        // K range whose weight panels the previous wave touched last (still in L2)
+        const bool back = n_fastest && (wave & 1);
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1, wait_limit, abort_flag, SITE_GEMM2_PRODUCER)) {
             ok = false;
@@ -488,12 +488,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
           }
           if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * STAGE_BYTES);
           const uint32_t leader_full = mapa_shared(smem_u32(&full[stage]), 0);
-          if (n_fastest)
-            tma_load_2d_pair_hint(sA + stage * A_BYTES, &tmA, leader_full, kb * BK, tm * BM + (int)rank * BM_CTA,
-                                  a_policy);
-          else
-            tma_load_2d_pair(sA + stage * A_BYTES, &tmA, leader_full, kb * BK, tm * BM + (int)rank * BM_CTA);
-          tma_load_2d_pair(sB + stage * B_BYTES, &tmB, leader_full, kb * BK, tn * BN + (int)rank * BN_CTA);
+          const int kx = (back ? num_kb - 1 - kb : kb) * BK;
+          tma_load_2d_pair(sA + stage * A_BYTES, &tmA, leader_full, kx, tm * BM + (int)rank * BM_CTA);
+          tma_load_2d_pair(sB + stage * B_BYTES, &tmB, leader_full, kx, tn * BN + (int)rank * BN_CTA);
           issued_mask |= 1u << stage;
           issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) {

@@ -39,56 +39,91 @@ def _peer(group, r):
     return r if group is None else dist.get_global_rank(group, r)
 
 
+def _cuda_attn_acc(q, k, v, o, lse, H):
+    from . import dit_attention_accumulate
+    dit_attention_accumulate(q, k, v, o, lse, 1, q.shape[0], k.shape[0], H)
+
+
 class RingAttention:
     """One rank's ring attention with buffers owned by the plan.
 
     Call: out = attention(q, K, V) where K and V are the concatenation of every
-    rank's k and v shards.  The local k and v are copied into slot 0 of a
-    two-slot ring; for N - 1 hops the shard in hand is sent to rank r+1 while
-    the next one is received from rank r-1, and the local attention of the
-    shard in hand runs meanwhile.  Hop 0 writes the running result, later hops
-    a partial result merged into it by log-sum-exp; the last merge writes
-    `out`.  Returns the fp32 log-sum-exp [1, H, S/N] of the local queries over
-    all keys (a buffer of the plan)."""
+    rank's k and v shards.  Shards travel one per hop: at hop h this rank sends
+    the shard it received last (its own at hop 0) to rank r+1 and receives the
+    next one from rank r-1, N - 1 hops in all, each hop's send and receive
+    posted as one batch.  Received shards land in consecutive rows of a
+    staging ring, and every `shards_per_step` shards (G) one attention launch
+    covers them: the first writes `out` and the running log-sum-exp, the
+    later ones merge into both in their epilogue (dit_attention_accumulate),
+    while the next G shards are still arriving.  G = 1 is the ring of the
+    compile_graph page (§5); larger G trades overlap for longer launches
+    (G = N gathers every shard before one launch).  Returns the fp32
+    log-sum-exp [1, H, S/N] of the local queries over all keys (a buffer of
+    the plan).
 
-    def __init__(self, S_loc, H, device, dtype=None, group=None, attn=None, merge=None):
+    With `attn` and `merge` given (the CPU tests' oracle operations), a later
+    step writes its own result to a partial buffer and `merge` folds it in."""
+
+    def __init__(self, S_loc, H, device, dtype=None, group=None, attn=None, merge=None, shards_per_step=1):
         import torch
         import torch.distributed as dist
         dtype = dtype or torch.bfloat16
         self.H, self.S_loc, self.group = H, S_loc, group
         self.N = dist.get_world_size(group)
         self.r = dist.get_rank(group)
+        self.G = max(1, min(int(shards_per_step), self.N))
+        custom = attn is not None or merge is not None
         self.attn = attn or _cuda_attn
         self.merge = merge or _cuda_merge
+        self.acc = None if custom else _cuda_attn_acc
         D = H * 128
-        self.kv = torch.empty((2, 2, S_loc, D), dtype=dtype, device=device)  # slot, (k, v)
-        self.o_acc = torch.empty((S_loc, D), dtype=dtype, device=device)
-        self.part = torch.empty_like(self.o_acc)
+        slots = 2 * self.G if self.N > self.G else self.G  # two stages in flight while more shards follow
+        self.slots = slots
+        self.k = torch.empty((slots * S_loc, D), dtype=dtype, device=device)
+        self.v = torch.empty_like(self.k)
         self.lse = torch.empty((1, H, S_loc), dtype=torch.float32, device=device)
-        self.lse_part = torch.empty_like(self.lse)
+        if self.acc is None:
+            self.part = torch.empty((S_loc, D), dtype=dtype, device=device)
+            self.lse_part = torch.empty_like(self.lse)
         self.nxt = _peer(group, (self.r + 1) % self.N)
         self.prv = _peer(group, (self.r - 1) % self.N)
 
+    def _rows(self, slot, n=1):
+        a = slot * self.S_loc
+        return slice(a, a + n * self.S_loc)
+
+    def _step(self, q, first_slot, n, out, first):
+        H = self.H
+        kk, vv = self.k[self._rows(first_slot, n)], self.v[self._rows(first_slot, n)]
+        if first:
+            self.attn(q, kk, vv, out, self.lse, H)
+        elif self.acc is not None:
+            self.acc(q, kk, vv, out, self.lse, H)
+        else:
+            self.attn(q, kk, vv, self.part, self.lse_part, H)
+            self.merge([out, self.part], [self.lse, self.lse_part], out, self.lse, H)
+
     def __call__(self, q, k, v, out):
         import torch.distributed as dist
-        D, N, H = self.H * 128, self.N, self.H
-        self.kv[0, 0].copy_(k[:, :D])
-        self.kv[0, 1].copy_(v[:, :D])
-        for hop in range(N):
-            cur, nxt = hop & 1, (hop + 1) & 1
+        D, N, G, S = self.H * 128, self.N, self.G, self.slots
+        self.k[self._rows(0)].copy_(k[:, :D])
+        self.v[self._rows(0)].copy_(v[:, :D])
+        step_first = 0  # slot of the current step's first shard
+        for h in range(N):  # shard h (received at hop h - 1, or the local one) sits in slot h % S
             reqs = []
-            if hop < N - 1:
-                # one group for the send and the receive: with NCCL, separate calls
+            if h < N - 1:
+                # one group for the sends and the receives: with NCCL, separate calls
                 # would queue every rank's send ahead of its receive and wait in a cycle
-                reqs = dist.batch_isend_irecv([dist.P2POp(dist.isend, self.kv[cur], self.nxt, self.group),
-                                               dist.P2POp(dist.irecv, self.kv[nxt], self.prv, self.group)])
-            kk, vv = self.kv[cur, 0], self.kv[cur, 1]
-            if hop == 0:
-                self.attn(q, kk, vv, out if N == 1 else self.o_acc, self.lse, H)
-            else:
-                self.attn(q, kk, vv, self.part, self.lse_part, H)
-                self.merge([self.o_acc, self.part], [self.lse, self.lse_part],
-                           out if hop == N - 1 else self.o_acc, self.lse, H)
+                cur, nxt = self._rows(h % S), self._rows((h + 1) % S)
+                reqs = dist.batch_isend_irecv([
+                    dist.P2POp(dist.isend, self.k[cur], self.nxt, self.group),
+                    dist.P2POp(dist.isend, self.v[cur], self.nxt, self.group),
+                    dist.P2POp(dist.irecv, self.k[nxt], self.prv, self.group),
+                    dist.P2POp(dist.irecv, self.v[nxt], self.prv, self.group)])
+            if (h + 1) % G == 0 or h == N - 1:  # the step's last shard is in hand
+                n = h - (h // G) * G + 1
+                self._step(q, step_first, n, out, h < G)
+                step_first = (h + 1) % S
             for req in reqs:
                 req.wait()
         return self.lse
@@ -135,9 +170,9 @@ class UlyssesAttention:
         return out
 
 
-def ring_attention(q, k, v, out, H, group=None, attn=None, merge=None):
+def ring_attention(q, k, v, out, H, group=None, attn=None, merge=None, shards_per_step=1):
     """One-off ring attention (a plan built for this call); see RingAttention."""
-    plan = RingAttention(q.shape[0], H, q.device, q.dtype, group, attn, merge)
+    plan = RingAttention(q.shape[0], H, q.device, q.dtype, group, attn, merge, shards_per_step)
     lse = plan(q, k, v, out)
     return lse[0]
 
@@ -191,7 +226,7 @@ class SequenceParallelSingleBlock:
     [1, D] bf16; rope: this shard's rows of the RoPE table [S/N, 64, 2] fp32."""
 
     def __init__(self, S_loc, D, H, M, device, group=None, mode="ring", ops=None, attn=None, merge=None,
-                 dtype=None, eps=1e-6):
+                 dtype=None, eps=1e-6, shards_per_step=1):
         import torch
         dtype = dtype or torch.bfloat16
         if mode not in ("ring", "ulysses"):
@@ -203,7 +238,7 @@ class SequenceParallelSingleBlock:
         self.qkv = torch.empty((S_loc, 3 * D), dtype=dtype, device=device)
         self.cat = torch.empty((S_loc, D + M), dtype=dtype, device=device)
         if mode == "ring":
-            self.attention = RingAttention(S_loc, H, device, dtype, group, attn, merge)
+            self.attention = RingAttention(S_loc, H, device, dtype, group, attn, merge, shards_per_step)
         else:
             self.attention = UlyssesAttention(S_loc, H, device, dtype, group, attn)
 

@@ -190,6 +190,25 @@ dit_status dit_attention(const dit_bf16* q, const dit_bf16* k, const dit_bf16* v
                          float* lse, int B, int Sq, int Skv, int H, int head_dim,
                          float softmax_scale, void* stream);
 
+/* Attention of q against one more key set, merged into a running result
+ * ([CG] §5: a ring hop adds the attention over the shard in hand to the
+ * result over the shards seen so far, by log-sum-exp).  On entry o (same
+ * layout as dit_attention's output) and lse (required, fp32 [B][H][Sq],
+ * natural log) hold the running result over earlier keys; on return they
+ * hold the result over the union:
+ *   lse' = log(exp(lse) + exp(lse_cur)),
+ *   o'   = exp(lse - lse') o + exp(lse_cur - lse') o_cur,
+ * where (o_cur, lse_cur) is dit_attention over k, v.  A row whose running
+ * lse is -inf (nothing accumulated yet) gets o_cur exactly as dit_attention
+ * would write it (o is then only read, with weight 0, and must be finite).
+ * One launch, no extra buffer: the merge runs in the epilogue, each thread
+ * reading its row of o before writing it.  Arguments and errors as
+ * dit_attention; lse == NULL is DIT_ERR_INVALID_ARG. */
+dit_status dit_attention_accumulate(const dit_bf16* q, const dit_bf16* k, const dit_bf16* v,
+                                    int64_t ldq, int64_t ldk, int64_t ldv, dit_bf16* o, int64_t ldo,
+                                    float* lse, int B, int Sq, int Skv, int H, int head_dim,
+                                    float softmax_scale, void* stream);
+
 /* Merge of attention results over disjoint key sets ([CG] §5: sequence-
  * parallel ring attention merges each hop's partial result by its
  * log-sum-exp):

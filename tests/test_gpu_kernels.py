@@ -242,7 +242,7 @@ def _attn_case(B, Sq, Skv, H, qmul=1.0, seed=0):
     (1, 384, 640, 1, 8.0),     # peaky logits: exercises the online max rescale
     (1, 1000, 512, 2, 1.0),    # cross-attention shape (512 context tokens)
     (1, 1, 1, 1, 1.0),         # single query, single key
-    (1, 129, 127, 1, 3.0),
+    (1, 129, 127, 1, 3.0),     # peaky, ragged
 ])
 def test_attention(B, Sq, Skv, H, qmul):
     import torch
@@ -257,15 +257,17 @@ def test_attention(B, Sq, Skv, H, qmul):
     for b in range(B):
         qs, ks, vs = qf[b * Sq:(b + 1) * Sq], kf[b * Skv:(b + 1) * Skv], vf[b * Skv:(b + 1) * Skv]
         ref = O.attention(qs, ks, vs, H)
-        # Derived max-abs bound for a bf16 attention output: the largest
-        # element carries its own bf16 rounding (<= 2^-9 relative) plus the
-        # bf16 rounding of P that the tensor-core PV product needs (<= 2^-9
-        # relative per term), so allow 2^-7 * max|ref| on top of 3e-2 * RMS
-        # (averaging over many keys makes RMS small next to the largest
-        # element).  rel L2 keeps 1e-2 and must also stay within 2x the error
-        # of the exact result merely rounded to bf16 (+1e-3).
+        # Near-uniform softmax (qmul 1): the stated bound.  Peaky logits
+        # (qmul 3, 8): a few keys dominate each row, so the largest outputs sit
+        # near max|v| while averaging keeps RMS small; such an element carries
+        # its own bf16 rounding (<= 2^-9 relative) plus the bf16 rounding of P
+        # that the tensor-core PV product needs (<= 2^-9 relative per term),
+        # hence the derived bound 3e-2 * RMS + 2^-7 * max|ref| for those cases
+        # only.  rel L2 keeps 1e-2 and must also stay within 2x the error of
+        # the exact result merely rounded to bf16 (+1e-3).
         rms = np.sqrt(np.mean(ref ** 2))
-        parity(got[b], ref, f"attention b={b}", max_abs_frac=3e-2 + 2.0 ** -7 * np.abs(ref).max() / rms)
+        frac = 3e-2 if qmul == 1.0 else 3e-2 + 2.0 ** -7 * np.abs(ref).max() / rms
+        parity(got[b], ref, f"attention b={b}", max_abs_frac=frac)
         ref_b = synth.bf16_bits_to_f64(synth.f32_to_bf16_bits(ref.astype(np.float32)))
         floor = np.linalg.norm(ref_b - ref) / np.linalg.norm(ref)
         assert np.linalg.norm(got[b] - ref) / np.linalg.norm(ref) <= 2 * floor + 1e-3
@@ -374,6 +376,42 @@ def test_ring_schedule_on_one_gpu_equals_full_attention():
     rms = np.sqrt(np.mean(ref ** 2))
     # each hop's output and the merge round to bf16: four roundings of <= 2^-9
     parity(host_f64(o), ref, "ring on one GPU", max_abs_frac=3e-2 + 4 * 2.0 ** -9 * np.abs(ref).max() / rms)
+    ref_lse = O.attention_lse(qf, kf, H)
+    assert np.abs(lse[0].cpu().double().numpy() - ref_lse).max() < 1e-3 * max(1.0, np.abs(ref_lse).max())
+    assert_no_device_error()
+
+
+@pytest.mark.parametrize("cuts", [(0, 256, 512), (0, 100, 333, 576, 600), (0, 577)])
+def test_attention_accumulate_over_key_splits(cuts):
+    """dit_attention_accumulate folds the attention over one more key set into
+    a running (o, lse): started from lse = -inf it equals dit_attention bit
+    for bit, and accumulating over uneven key splits gives the attention over
+    all keys (fp64 oracle) and its log-sum-exp.  Each step rounds the running
+    output to bf16: max abs <= 3e-2 RMS + (steps) 2^-9 max|ref|."""
+    import torch
+    H, Sq = 3, 300
+    D = H * 128
+    Skv = cuts[-1]
+    q, k, v = _attn_case(1, Sq, Skv, H, 2.0, seed=9)
+    dq, dk, dv = dev_bf16(q), dev_bf16(k), dev_bf16(v)
+    o = torch.zeros((Sq, D), dtype=torch.bfloat16, device="cuda")
+    lse = torch.full((1, H, Sq), float("-inf"), dtype=torch.float32, device="cuda")
+    plain = torch.empty_like(o)
+    plain_lse = torch.empty_like(lse)
+    a, b = cuts[0], cuts[1]
+    dit.dit_attention(dq, dk[a:b], dv[a:b], plain, 1, Sq, b - a, H, lse=plain_lse)
+    dit.dit_attention_accumulate(dq, dk[a:b], dv[a:b], o, lse, 1, Sq, b - a, H)
+    torch.cuda.synchronize()
+    assert torch.equal(o, plain) and torch.equal(lse, plain_lse)
+    for a, b in zip(cuts[1:], cuts[2:]):
+        dit.dit_attention_accumulate(dq, dk[a:b], dv[a:b], o, lse, 1, Sq, b - a, H)
+    torch.cuda.synchronize()
+    qf, kf, vf = (synth.bf16_bits_to_f64(t) for t in (q, k, v))
+    ref = O.attention(qf, kf, vf, H)
+    rms = np.sqrt(np.mean(ref ** 2))
+    steps = len(cuts) - 1
+    parity(host_f64(o), ref, "accumulated attention",
+           max_abs_frac=3e-2 + steps * 2.0 ** -9 * np.abs(ref).max() / rms)
     ref_lse = O.attention_lse(qf, kf, H)
     assert np.abs(lse[0].cpu().double().numpy() - ref_lse).max() < 1e-3 * max(1.0, np.abs(ref_lse).max())
     assert_no_device_error()

@@ -58,24 +58,26 @@ def _rank(rank, world, port, S, H, out):
         ref = O.attention(q, k, v, H)[sl]
         ref_lse = O.attention_lse(q, k, H)[:, sl]
         qs, ks, vs = (torch.from_numpy(np.ascontiguousarray(t[sl])) for t in (q, k, v))
-        o_ring = torch.empty_like(qs)
-        lse = sp.ring_attention(qs, ks, vs, o_ring, H, attn=o_attn, merge=o_merge)
+        ring = []
+        for g in range(1, world + 1):  # shards per attention step: 1 (the ring) .. N (gather all)
+            o_ring = torch.empty_like(qs)
+            lse = sp.ring_attention(qs, ks, vs, o_ring, H, attn=o_attn, merge=o_merge, shards_per_step=g)
+            ring.append((float(np.abs(o_ring.numpy() - ref).max()),
+                         float(np.abs(lse.double().numpy() - ref_lse).max() / np.abs(ref_lse).max())))
         o_uly = torch.empty_like(qs)
         sp.ulysses_attention(qs, ks, vs, o_uly, H, attn=o_attn)
-        out[rank] = (float(np.abs(o_ring.numpy() - ref).max()),
-                     float(np.abs(lse.double().numpy() - ref_lse).max() / np.abs(ref_lse).max()),
-                     float(np.abs(o_uly.numpy() - ref).max()))
+        out[rank] = (ring, float(np.abs(o_uly.numpy() - ref).max()))
         dist.barrier()
     finally:
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world", [2, 4])
+@pytest.mark.parametrize("world", [2, 3, 4])
 def test_ring_and_ulysses_schedules_equal_full_attention(world):
     ctx = mp.get_context("spawn")
     mgr = ctx.Manager()
     out = mgr.dict()
-    S, H = 24, 4
+    S, H = 24, (6 if world == 3 else 4)
     port = _free_port()
     procs = [ctx.Process(target=_rank, args=(r, world, port, S, H, out)) for r in range(world)]
     for p in procs:
@@ -84,10 +86,11 @@ def test_ring_and_ulysses_schedules_equal_full_attention(world):
         p.join(timeout=120)
         assert p.exitcode == 0, f"rank exited with {p.exitcode}"
     for r in range(world):
-        ring_err, lse_err, uly_err = out[r]
+        ring, uly_err = out[r]
         # the ring's merge takes the running lse in fp32 (the CUDA contract)
-        assert ring_err < 1e-6, (r, ring_err)
-        assert lse_err < 1e-6, (r, lse_err)
+        for g, (ring_err, lse_err) in enumerate(ring, 1):
+            assert ring_err < 1e-6, (r, g, ring_err)
+            assert lse_err < 1e-6, (r, g, lse_err)
         assert uly_err < 1e-12, (r, uly_err)
 
 
