@@ -411,11 +411,11 @@ def run_ours(args, rank, world, local_rank):
 # (profiles/*.ncu.md), with a hash of the kernel's sources at capture time.
 # A kernel whose sources changed since reports traffic null.
 NCU_TRAFFIC = {
-    "gemm_qkv_mlp_gelu_qknorm_rope": (335648256, ("gemm.cuh", "common.cuh"), "cf20cddbba096d1c"),
-    "gemm_out_gated_residual": (588929792, ("gemm.cuh", "common.cuh"), "cf20cddbba096d1c"),
-    "attention": (95100928, ("attention.cuh", "common.cuh"), "03b6fdd82910cea2"),
-    "modulate_norm": (28414720, ("elementwise.cuh", "common.cuh"), "97ff3e5e07faf2f4"),
-    "adaln_modulation": (56782336, ("elementwise.cuh", "common.cuh"), "97ff3e5e07faf2f4"),
+    "gemm_qkv_mlp_gelu_qknorm_rope": (337409280, ("gemm.cuh", "common.cuh"), "2684d334b04464f6"),
+    "gemm_out_gated_residual": (436414208, ("gemm.cuh", "common.cuh"), "2684d334b04464f6"),
+    "attention": (95543040, ("attention.cuh", "common.cuh"), "e03ff7a4dcb5868e"),
+    "modulate_norm": (28440064, ("elementwise.cuh", "common.cuh"), "bf93bdf9621f448c"),
+    "adaln_modulation": (56678400, ("elementwise.cuh", "common.cuh"), "bf93bdf9621f448c"),
 }
 
 
