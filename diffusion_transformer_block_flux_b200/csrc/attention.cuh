@@ -86,7 +86,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     mbar_init(q_full, 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&k_full[s], 1);
-      mbar_init(&k_empty[s], 1);
+      mbar_init(&k_empty[s], 4);  // the four warps of tile 1, once they hold the scores of the last QK
       mbar_init(&v_full[s], 1);
       mbar_init(&v_empty[s], 1);
       mbar_init(&s_full[s], 1);
@@ -150,90 +150,100 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
     }
   } else if (warp == 9) {
-    if (lane == 0) {
-      // ---------------- MMA issuer ----------------
-      const uint32_t sQ0 = smem_u32(smem + OFF_Q);
-      bool ok = true;
-      bool issued = false;
-      uint32_t sfree_ph = 0;  // parity of the next s_free phase
-      auto issue_qk = [&](int t, int kst) {
-        const uint32_t kb = smem_u32(smem + OFF_K + kst * TILE_BYTES);
+    // ---------------- MMA issuer: the whole warp runs the loop, one elected
+    // lane issues each tcgen05 instruction ----------------
+    const uint32_t sQ0 = smem_u32(smem + OFF_Q);
+    bool ok = true;
+    bool issued = false;
+    uint32_t sfree_ph = 0;  // parity of the next s_free phase
+    // Descriptors are built once: the address field of a shared-memory
+    // descriptor is (address >> 4), so moving to another tile, stage or
+    // 16-deep slice adds (byte offset >> 4) to the base descriptor.
+    const uint64_t dQ = sdesc_sw128(sQ0, 16, 1024);
+    const uint64_t dK = sdesc_sw128(smem_u32(smem + OFF_K), 16, 1024);
+    const uint64_t dV = sdesc_sw128(smem_u32(smem + OFF_V), HALF_BYTES, 1024);
+    const uint32_t tSacc = tmem_base + COL_S;
+    auto issue_qk = [&](int t, int kst) {
+      const uint64_t q = dQ + (uint64_t)((t * TILE_BYTES) >> 4);
+      const uint64_t k = dK + (uint64_t)((kst * TILE_BYTES) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < HD / 16; ++kk) {
-          const uint32_t off = (uint32_t)((kk >> 2) * HALF_BYTES + (kk & 3) * 32);
-          umma_ss(tmem_base + COL_S, sdesc_sw128(sQ0 + (uint32_t)(t * TILE_BYTES) + off, 16, 1024),
-                  sdesc_sw128(kb + off, 16, 1024), IDESC_QK, kk > 0 ? 1u : 0u);
-        }
-      };
-      auto issue_pv = [&](int t, int vst, bool acc) {
-        const uint32_t vb = smem_u32(smem + OFF_V + vst * TILE_BYTES);
+      for (int kk = 0; kk < HD / 16; ++kk) {
+        const uint64_t off = (uint64_t)(((kk >> 2) * HALF_BYTES + (kk & 3) * 32) >> 4);
+        umma_ss_elect(tSacc, q + off, k + off, IDESC_QK, kk > 0 ? 1u : 0u);
+      }
+    };
+    auto issue_pv = [&](int t, int vst, bool acc) {
+      const uint64_t v = dV + (uint64_t)((vst * TILE_BYTES) >> 4);
+      const uint32_t tO = tmem_base + COL_O + (uint32_t)(t * 128);
+      const uint32_t tP = tmem_base + COL_P + (uint32_t)(t * 64);
 #pragma unroll
-        for (int kk = 0; kk < BKV / 16; ++kk) {
-          // A: P_t in TMEM, 16 keys = 8 columns of bf16 pairs.
-          // B: V MN-major; 64-d halves HALF_BYTES apart (LBO), 8-key groups 1024 B apart (SBO).
-          umma_ts(tmem_base + COL_O + (uint32_t)(t * 128), tmem_base + COL_P + (uint32_t)(t * 64 + kk * 8),
-                  sdesc_sw128(vb + (uint32_t)(kk * 2048), HALF_BYTES, 1024), IDESC_PV, (acc || kk > 0) ? 1u : 0u);
-        }
-      };
-      auto wait_sfree = [&]() -> bool {
-        const bool r = mbar_wait(s_free, sfree_ph, wait_limit, abort_flag, SITE_ATTN_MMA);
-        sfree_ph ^= 1u;
-        return r;
-      };
-      // prologue: S <- Q0 K_0, then (once tile 0 has loaded it) S <- Q1 K_0
-      if (!mbar_wait(q_full, 0, wait_limit, abort_flag, SITE_ATTN_MMA)) ok = false;
-      if (ok && !mbar_wait(&k_full[0], 0, wait_limit, abort_flag, SITE_ATTN_MMA)) ok = false;
-      if (ok) {
-        tc_fence_after();
-        issue_qk(0, 0);
-        umma_commit(&s_full[0]);
-        issued = true;
+      for (int kk = 0; kk < BKV / 16; ++kk) {
+        // A: P_t in TMEM, 16 keys = 8 columns of bf16 pairs.
+        // B: V MN-major; 64-d halves HALF_BYTES apart (LBO), 8-key groups 1024 B apart (SBO).
+        umma_ts_elect(tO, tP + (uint32_t)(kk * 8), v + (uint64_t)((kk * 2048) >> 4), IDESC_PV,
+                      (acc || kk > 0) ? 1u : 0u);
       }
-      if (ok && !wait_sfree()) ok = false;
-      if (ok) {
+    };
+    // every lane waits; the warp proceeds only if all of them saw the phase
+    auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity, wait_limit, abort_flag, SITE_ATTN_MMA));
+    };
+    auto wait_sfree = [&]() -> bool {
+      const bool r = wait(s_free, sfree_ph);
+      sfree_ph ^= 1u;
+      return r;
+    };
+    // prologue: S <- Q0 K_0, then (once tile 0 has loaded it) S <- Q1 K_0
+    if (!wait(q_full, 0)) ok = false;
+    if (ok && !wait(&k_full[0], 0)) ok = false;
+    if (ok) {
+      tc_fence_after();
+      issue_qk(0, 0);
+      umma_commit_elect(&s_full[0]);
+      issued = true;
+    }
+    if (ok && !wait_sfree()) ok = false;
+    if (ok) {
+      tc_fence_after();
+      issue_qk(1, 0);
+      umma_commit_elect(&s_full[1]);
+    }
+    for (int j = 0; j < n_kv && ok; ++j) {
+      const int st = j & 1;
+      const uint32_t ph = (j >> 1) & 1;
+      const bool has_next = j + 1 < n_kv;
+      const int nst = (j + 1) & 1;
+      const uint32_t nph = ((j + 1) >> 1) & 1;
+      if (has_next) {  // S <- Q0 K_{j+1} once tile 1 has loaded its scores of key tile j
+        if (!wait_sfree()) { ok = false; break; }
+        if (!wait(&k_full[nst], nph)) { ok = false; break; }
         tc_fence_after();
-        issue_qk(1, 0);
-        umma_commit(&s_full[1]);
-        umma_commit(&k_empty[0]);
+        issue_qk(0, nst);
+        umma_commit_elect(&s_full[0]);
       }
-      for (int j = 0; j < n_kv && ok; ++j) {
-        const int st = j & 1;
-        const uint32_t ph = (j >> 1) & 1;
-        const bool has_next = j + 1 < n_kv;
-        const int nst = (j + 1) & 1;
-        const uint32_t nph = ((j + 1) >> 1) & 1;
-        if (has_next) {  // S <- Q0 K_{j+1} once tile 1 has loaded its scores of key tile j
-          if (!wait_sfree()) { ok = false; break; }
-          if (!mbar_wait(&k_full[nst], nph, wait_limit, abort_flag, SITE_ATTN_MMA)) { ok = false; break; }
-          tc_fence_after();
-          issue_qk(0, nst);
-          umma_commit(&s_full[0]);
-        }
-        if (!mbar_wait(&v_full[st], ph, wait_limit, abort_flag, SITE_ATTN_MMA)) { ok = false; break; }
-        if (!mbar_wait(&p_full[0], j & 1, wait_limit, abort_flag, SITE_ATTN_MMA)) { ok = false; break; }
+      if (!wait(&v_full[st], ph)) { ok = false; break; }
+      if (!wait(&p_full[0], j & 1)) { ok = false; break; }
+      tc_fence_after();
+      issue_pv(0, st, j > 0);
+      umma_commit_elect(&p_free[0]);
+      if (has_next) {  // S <- Q1 K_{j+1} once tile 0 has loaded its scores of key tile j+1
+        if (!wait_sfree()) { ok = false; break; }
         tc_fence_after();
-        issue_pv(0, st, j > 0);
-        umma_commit(&p_free[0]);
-        if (has_next) {  // S <- Q1 K_{j+1} once tile 0 has loaded its scores of key tile j+1
-          if (!wait_sfree()) { ok = false; break; }
-          tc_fence_after();
-          issue_qk(1, nst);
-          umma_commit(&s_full[1]);
-          umma_commit(&k_empty[nst]);
-        }
-        if (!mbar_wait(&p_full[1], j & 1, wait_limit, abort_flag, SITE_ATTN_MMA)) { ok = false; break; }
-        tc_fence_after();
-        issue_pv(1, st, j > 0);
-        umma_commit(&p_free[1]);
-        umma_commit(&v_empty[st]);
+        issue_qk(1, nst);
+        umma_commit_elect(&s_full[1]);
       }
-      if (ok) {
-        umma_commit(&o_full[0]);
-        umma_commit(&o_full[1]);
-      } else if (issued) {
-        umma_commit(drain);
-        (void)mbar_wait(drain, 0, wait_limit, nullptr, SITE_ATTN_DRAIN);
-      }
+      if (!wait(&p_full[1], j & 1)) { ok = false; break; }
+      tc_fence_after();
+      issue_pv(1, st, j > 0);
+      umma_commit_elect(&p_free[1]);
+      umma_commit_elect(&v_empty[st]);
+    }
+    if (ok) {
+      umma_commit_elect(&o_full[0]);
+      umma_commit_elect(&o_full[1]);
+    } else if (issued) {
+      umma_commit_elect(drain);
+      (void)mbar_wait(drain, 0, wait_limit, nullptr, SITE_ATTN_DRAIN);
     }
   } else {
     // ---------------- softmax warpgroups ----------------
@@ -255,6 +265,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     for (int j = 0; j < n_kv; ++j) {
       ok = mbar_wait(&s_full[t], j & 1, wait_limit, abort_flag, SITE_ATTN_SOFTMAX);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+      // QK_1(j) is the last MMA that reads key tile j: once its scores are
+      // complete, tile 1's warps release the K stage (one arrival per warp,
+      // so the issuing thread spends no commit on it)
+      if (t == 1 && lane == 0) mbar_arrive(&k_empty[j & 1]);
       tc_fence_after();
       uint32_t r[4][32];
       tmem_ld32_nowait(tS + 0u, r[0]);

@@ -278,44 +278,44 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ---------------- MMA issuer ----------------
+    {
+      // ---------------- MMA issuer: the whole warp runs the loop, one
+      // elected lane issues each tcgen05 instruction ----------------
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
       bool issued_any = false;
+      const uint64_t dA = sdesc_sw128(smem_u32(sA), 16, 1024);
+      const uint64_t dB = sdesc_sw128(smem_u32(sB), 16, 1024);
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        if (!mbar_wait(&tempty[acc], acc_phase ^ 1, wait_limit, abort_flag, SITE_GEMM_MMA)) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&tempty[acc], acc_phase ^ 1, wait_limit, abort_flag, SITE_GEMM_MMA))) {
           ok = false;
           break;
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
         for (int kb = 0; kb < num_kb; ++kb) {
-          if (!mbar_wait(&full[stage], phase, wait_limit, abort_flag, SITE_GEMM_MMA)) {
+          if (!__all_sync(0xffffffffu, mbar_wait(&full[stage], phase, wait_limit, abort_flag, SITE_GEMM_MMA))) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t a0 = smem_u32(sA + stage * A_BYTES);
-          const uint32_t b0 = smem_u32(sB + stage * B_BYTES);
+          const uint64_t a0 = dA + (uint64_t)((stage * A_BYTES) >> 4);
+          const uint64_t b0 = dB + (uint64_t)((stage * B_BYTES) >> 4);
 #pragma unroll
-          for (int k = 0; k < BK / 16; ++k) {
-            const uint64_t ad = sdesc_sw128(a0 + k * 32, 16, 1024);
-            const uint64_t bd = sdesc_sw128(b0 + k * 32, 16, 1024);
-            umma_ss(d_tmem, ad, bd, IDESC, (kb | k) != 0 ? 1u : 0u);
-          }
+          for (int k = 0; k < BK / 16; ++k)
+            umma_ss_elect(d_tmem, a0 + (uint64_t)(k * 2), b0 + (uint64_t)(k * 2), IDESC, (kb | k) != 0 ? 1u : 0u);
           issued_any = true;
-          umma_commit(&empty[stage]);
+          umma_commit_elect(&empty[stage]);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
           }
         }
         if (!ok) break;
-        umma_commit(&tfull[acc]);
+        umma_commit_elect(&tfull[acc]);
         if (++acc == 2) {
           acc = 0;
           acc_phase ^= 1;
@@ -323,7 +323,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       if (!ok && issued_any) {
         // Make sure no MMA still writes TMEM when it is released.
-        umma_commit(drain);
+        umma_commit_elect(drain);
         (void)mbar_wait(drain, 0, wait_limit, nullptr, SITE_GEMM_DRAIN);
       }
     }
@@ -506,50 +506,52 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0 && rank == 0) {
-      // ---------------- MMA issuer (leader CTA) ----------------
+    if (rank == 0) {
+      // ---------------- MMA issuer (leader CTA): the whole warp runs the
+      // loop, one elected lane issues each tcgen05 instruction ----------------
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
       bool issued_any = false;
+      // descriptor of stage 0's A and B tiles; a stage or a 16-deep slice adds (byte offset >> 4)
+      const uint64_t dA = sdesc_sw128(smem_u32(sA), 16, 1024);
+      const uint64_t dB = sdesc_sw128(smem_u32(sB), 16, 1024);
       for (int tile = cluster_id; tile < num_tiles && ok; tile += n_clusters) {
-        if (!mbar_wait(&tempty[acc], acc_phase ^ 1, wait_limit, abort_flag, SITE_GEMM2_MMA)) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&tempty[acc], acc_phase ^ 1, wait_limit, abort_flag, SITE_GEMM2_MMA))) {
           ok = false;
           break;
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
         for (int kb = 0; kb < num_kb; ++kb) {
-          if (!mbar_wait(&full[stage], phase, wait_limit, abort_flag, SITE_GEMM2_MMA)) {
+          if (!__all_sync(0xffffffffu, mbar_wait(&full[stage], phase, wait_limit, abort_flag, SITE_GEMM2_MMA))) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t a0 = smem_u32(sA + stage * A_BYTES);
-          const uint32_t b0 = smem_u32(sB + stage * B_BYTES);
+          const uint64_t a0 = dA + (uint64_t)((stage * A_BYTES) >> 4);
+          const uint64_t b0 = dB + (uint64_t)((stage * B_BYTES) >> 4);
 #pragma unroll
-          for (int k = 0; k < BK / 16; ++k) {
-            umma_ss_pair(d_tmem, sdesc_sw128(a0 + k * 32, 16, 1024), sdesc_sw128(b0 + k * 32, 16, 1024), IDESC,
-                         (kb | k) != 0 ? 1u : 0u);
-          }
+          for (int k = 0; k < BK / 16; ++k)
+            umma_ss_pair_elect(d_tmem, a0 + (uint64_t)(k * 2), b0 + (uint64_t)(k * 2), IDESC, (kb | k) != 0 ? 1u : 0u);
           issued_any = true;
-          umma_commit_pair(&empty[stage], 0x3);
+          umma_commit_pair_elect(&empty[stage], 0x3);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
           }
         }
         if (!ok) break;
-        umma_commit_pair(&tfull[acc], 0x3);
+        umma_commit_pair_elect(&tfull[acc], 0x3);
         if (++acc == 2) {
           acc = 0;
           acc_phase ^= 1;
         }
       }
       if (!ok && issued_any) {
-        umma_commit(drain);
+        umma_commit_elect(drain);
         (void)mbar_wait(drain, 0, wait_limit, nullptr, SITE_GEMM2_DRAIN);
       }
     }
