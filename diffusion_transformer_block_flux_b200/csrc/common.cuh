@@ -79,6 +79,23 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// The same test, letting the thread sleep until the phase completes or about
+// hint_ns nanoseconds pass: a waiting warp then takes no issue slots from the
+// warps that share its sub-partition.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
+constexpr uint32_t kWaitSleepNs = 20000;
+
 // Waits until the phase with the given parity has completed.  Returns false
 // (after recording a timeout) when the wait exceeds limit_ns or when another
 // thread of the CTA has raised *abort.  abort == nullptr: only the time limit
@@ -87,8 +104,8 @@ __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, uint
                                             volatile int* abort, uint32_t site) {
   const uint64_t t0 = globaltimer_ns();
   uint32_t n = 0;
-  while (!mbar_try_wait(bar, parity)) {
-    if ((++n & 255u) == 0) {
+  while (!mbar_try_wait_sleep(bar, parity, kWaitSleepNs)) {
+    if ((++n & 15u) == 0) {
       if (abort != nullptr && *abort) return false;
       if (globaltimer_ns() - t0 > limit_ns) {
         atomicCAS(&g_dit_error, 0u, (uint32_t)DIT_ERR_TIMEOUT | (site << 8));
