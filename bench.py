@@ -411,11 +411,11 @@ def run_ours(args, rank, world, local_rank):
 # (profiles/*.ncu.md), with a hash of the kernel's sources at capture time.
 # A kernel whose sources changed since reports traffic null.
 NCU_TRAFFIC = {
-    "gemm_qkv_mlp_gelu_qknorm_rope": (337409280, ("gemm.cuh", "common.cuh"), "2684d334b04464f6"),
-    "gemm_out_gated_residual": (436414208, ("gemm.cuh", "common.cuh"), "2684d334b04464f6"),
-    "attention": (95543040, ("attention.cuh", "common.cuh"), "e03ff7a4dcb5868e"),
-    "modulate_norm": (28440064, ("elementwise.cuh", "common.cuh"), "bf93bdf9621f448c"),
-    "adaln_modulation": (56678400, ("elementwise.cuh", "common.cuh"), "bf93bdf9621f448c"),
+    "gemm_qkv_mlp_gelu_qknorm_rope": (336957952, ("gemm.cuh", "common.cuh"), "58798835864e2a01"),
+    "gemm_out_gated_residual": (436787968, ("gemm.cuh", "common.cuh"), "58798835864e2a01"),
+    "attention": (92532224, ("attention.cuh", "common.cuh"), "a9751413b4e054e3"),
+    "modulate_norm": (28440064, ("elementwise.cuh", "common.cuh"), "046c38d671b7c963"),
+    "adaln_modulation": (56678400, ("elementwise.cuh", "common.cuh"), "046c38d671b7c963"),
 }
 
 
