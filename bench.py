@@ -646,12 +646,18 @@ def run_ring8(args):
     """One rank's compute in a CP=8 ring over the Flux sequence (4608 tokens
     = 8 x 576 per rank, 24 heads x 128), on one GPU: attention of the 576 local
     queries against the 8 key/value shards, each step after the first merged
-    into the running result in its epilogue (dit_attention_accumulate),
-    captured as one CUDA graph (the transfers between ranks are not part of
-    this single-GPU measurement).  G shards per attention step: G = 1 is the
-    ring (8 launches), G = 8 gathers every shard first (1 launch)."""
+    into the running result, captured as one CUDA graph (the transfers between
+    ranks are not part of this single-GPU measurement).  G shards per attention
+    step: G = 1 is the ring (8 steps), G = 8 gathers every shard first (1
+    step).  splits = 1: one attention launch per step, merging in its epilogue
+    (dit_attention / dit_attention_accumulate, 72 CTAs); splits = 2, the ring
+    plan's default at this size: the step's keys are cut in two parts computed
+    side by side (144 CTAs) and merged with the running result by
+    log-sum-exp (dit_attention_split).  The headline is the ring (G = 1) as
+    the plan runs it."""
     import torch
     import diffusion_transformer_block_flux_b200 as dit
+    from diffusion_transformer_block_flux_b200.sequence_parallel import auto_key_splits
     dev = torch.device("cuda", 0)
     g = torch.Generator(device=dev)
     g.manual_seed(13)
@@ -661,38 +667,47 @@ def run_ring8(args):
     kv = [_rand(torch, g, dev, 2, S, D) for _ in range(NB)]
     o = torch.empty((Sl, D), dtype=torch.bfloat16, device=dev)
     lse = torch.empty((1, H, Sl), dtype=torch.float32, device=dev)
+    auto = auto_key_splits(Sl, H, dev)
+    ws = torch.empty(max(1, dit.dit_attention_split_workspace(1, Sl, H, max(2, auto))), dtype=torch.uint8,
+                     device=dev)
     K = max(5, args.steps // 4)
     flops = 4.0 * Sl * S * H * 128
     per_g = {}
-    for G in (1, 2, 4, 8):
-        def ring(i, G=G):
-            k, v = kv[i][0], kv[i][1]
-            for j in range(0, N, G):
-                ks, vs = k[j * Sl:(j + G) * Sl], v[j * Sl:(j + G) * Sl]
-                if j == 0:
-                    dit.dit_attention(q[i], ks, vs, o, 1, Sl, G * Sl, H, lse=lse)
-                else:
-                    dit.dit_attention_accumulate(q[i], ks, vs, o, lse, 1, Sl, G * Sl, H)
+    for splits in sorted({1, auto}):
+        for G in (1, 2, 4, 8):
+            def ring(i, G=G, splits=splits):
+                k, v = kv[i][0], kv[i][1]
+                for j in range(0, N, G):
+                    ks, vs = k[j * Sl:(j + G) * Sl], v[j * Sl:(j + G) * Sl]
+                    if splits > 1:
+                        dit.dit_attention_split(q[i], ks, vs, o, 1, Sl, G * Sl, H, splits, ws, lse=lse,
+                                                accumulate=j > 0)
+                    elif j == 0:
+                        dit.dit_attention(q[i], ks, vs, o, 1, Sl, G * Sl, H, lse=lse)
+                    else:
+                        dit.dit_attention_accumulate(q[i], ks, vs, o, lse, 1, Sl, G * Sl, H)
 
-        for i in range(NB):
-            ring(i)
-        torch.cuda.synchronize()
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph):
             for i in range(NB):
                 ring(i)
-        ms = _event_time(torch, graph.replay, K, 3, torch.cuda.current_stream()) / NB
-        del graph
-        tf = flops / (ms * 1e-3) / 1e12
-        per_g[G] = {"ms": round(ms, 4), "tflops": round(tf, 1), "frac_of_bf16_peak": round(tf / peaks()["bf16_tflops"], 4),
-                    "launches": N // G}
+            torch.cuda.synchronize()
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                for i in range(NB):
+                    ring(i)
+            ms = _event_time(torch, graph.replay, K, 3, torch.cuda.current_stream()) / NB
+            del graph
+            tf = flops / (ms * 1e-3) / 1e12
+            per_g[f"G{G}_splits{splits}"] = {"ms": round(ms, 4), "tflops": round(tf, 1),
+                                             "frac_of_bf16_peak": round(tf / peaks()["bf16_tflops"], 4),
+                                             "launches": (N // G) * (2 if splits > 1 else 1)}
     st, code = dit.dit_get_device_error()
     if st != 0:
         raise RuntimeError(f"device error word {code:#x}")
-    ms1 = per_g[1]["ms"]
+    head = per_g[f"G1_splits{auto}"]
+    ms1 = head["ms"]
     return _extra_line("ring_cp8_rank_compute_S4608_576q_24x128", ms1, flops, K * NB, 3,
-                       {"us_per_hop": round(ms1 * 1e3 / N, 2), "hops": N, "gpu_launches_per_step": N,
-                        "shards_per_step": per_g,
+                       {"us_per_hop": round(ms1 * 1e3 / N, 2), "hops": N, "key_splits": auto,
+                        "gpu_launches_per_step": head["launches"], "shards_per_step": per_g,
                         "context": "the compile_graph page, section 5: one attention segment of the 8-card ring "
                                    "took 0.073 ms on H20"})
 

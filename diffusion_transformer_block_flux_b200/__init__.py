@@ -130,6 +130,9 @@ _SIGS = {
                             i32, i32, i32, f32, c_void_p]),
     "dit_attention_accumulate": (i32, [c_void_p, c_void_p, c_void_p, i64, i64, i64, c_void_p, i64, c_void_p, i32,
                                        i32, i32, i32, i32, f32, c_void_p]),
+    "dit_attention_split": (i32, [c_void_p, c_void_p, c_void_p, i64, i64, i64, c_void_p, i64, c_void_p, i32, i32,
+                                  i32, i32, i32, f32, i32, i32, c_void_p, size_t, c_void_p]),
+    "dit_attention_split_workspace": (size_t, [i32, i32, i32, i32]),
     "dit_gemm_epilogue": (i32, [ctypes.POINTER(dit_gemm_args), c_void_p]),
     "dit_selftest_exp2_poly": (i32, [c_void_p, c_void_p, i64, c_void_p]),
     "dit_attention_merge": (i32, [i32, ctypes.POINTER(c_void_p), ctypes.POINTER(c_void_p), i64, c_void_p, c_void_p,
@@ -301,6 +304,24 @@ def dit_attention_accumulate(q, k, v, o, lse, B, Sq, Skv, H, softmax_scale=None,
         softmax_scale = 128 ** -0.5
     _call("dit_attention_accumulate", _ptr(q), _ptr(k), _ptr(v), q.stride(0), k.stride(0), v.stride(0), _ptr(o),
           o.stride(0), _ptr(lse), B, Sq, Skv, H, 128, float(softmax_scale), _stream(stream))
+
+
+def dit_attention_split_workspace(B, Sq, H, n_split):
+    """Bytes of device workspace dit_attention_split needs."""
+    return lib().dit_attention_split_workspace(B, Sq, H, n_split)
+
+
+def dit_attention_split(q, k, v, o, B, Sq, Skv, H, n_split, workspace, lse=None, accumulate=False,
+                        softmax_scale=None, stream=None):
+    """Attention with the keys cut into n_split parts computed side by side
+    and merged by log-sum-exp; accumulate merges into the running (o, lse).
+    workspace: a uint8 device tensor of dit_attention_split_workspace bytes."""
+    if softmax_scale is None:
+        softmax_scale = 128 ** -0.5
+    _call("dit_attention_split", _ptr(q), _ptr(k), _ptr(v), q.stride(0), k.stride(0), v.stride(0), _ptr(o),
+          o.stride(0), _ptr(lse), B, Sq, Skv, H, 128, float(softmax_scale), n_split, int(bool(accumulate)),
+          _ptr(workspace), workspace.numel() * workspace.element_size() if workspace is not None else 0,
+          _stream(stream))
 
 
 def dit_selftest_exp2_poly(x, y, stream=None):

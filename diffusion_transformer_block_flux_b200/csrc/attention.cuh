@@ -26,6 +26,11 @@
 #include "common.cuh"
 
 namespace dit {
+
+// Most key splits one split launch takes (dit_attention_split); with the
+// running result they make at most five parts for the merge.
+constexpr int kAttnMaxSplits = 4;
+
 namespace attn {
 
 constexpr int BQ = 128;
@@ -53,6 +58,14 @@ struct Params {
   // 1: o and lse hold a running result over other keys on entry; this
   // launch's result is merged into it by log-sum-exp (a ring hop)
   int accumulate;
+  // Key split: blockIdx.z = batch * splits + s, and split s attends to keys
+  // [s kv_per_split, min(Skv, (s + 1) kv_per_split)) (never empty), writing
+  // its partial result to o + s o_split_stride and lse + s lse_split_stride.
+  // splits = 1, kv_per_split = Skv: the plain launch.
+  int splits;
+  int kv_per_split;  // a multiple of BKV when splits > 1
+  int64_t o_split_stride;
+  int64_t lse_split_stride;
 };
 
 __global__ void __launch_bounds__(NUM_THREADS, 1)
@@ -78,9 +91,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int head = blockIdx.y;
-  const int batch = blockIdx.z;
+  const int split = (int)blockIdx.z % p.splits;
+  const int batch = (int)blockIdx.z / p.splits;
+  const int kv0 = split * p.kv_per_split;                    // first key of this CTA's range
+  const int kv_len = min(p.Skv - kv0, p.kv_per_split);       // keys in the range (>= 1)
   const int q_row0 = blockIdx.x * 2 * BQ;
-  const int n_kv = (p.Skv + BKV - 1) / BKV;
+  const int n_kv = (kv_len + BKV - 1) / BKV;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -129,14 +145,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         mbar_arrive_expect_tx(&k_full[st], TILE_BYTES);
         for (int hf = 0; hf < 2; ++hf)
           tma_load_3d(smem + OFF_K + st * TILE_BYTES + hf * HALF_BYTES, &tmK, &k_full[st], x0 + hf * 64,
-                      j * BKV, batch);
+                      kv0 + j * BKV, batch);
         k_issued |= 1u << st;
         k_par = (k_par & ~(1u << st)) | (ph << st);
         if (!mbar_wait(&v_empty[st], ph ^ 1, wait_limit, abort_flag, SITE_ATTN_LOAD)) { ok = false; break; }
         mbar_arrive_expect_tx(&v_full[st], TILE_BYTES);
         for (int hf = 0; hf < 2; ++hf)
           tma_load_3d(smem + OFF_V + st * TILE_BYTES + hf * HALF_BYTES, &tmV, &v_full[st], x0 + hf * 64,
-                      j * BKV, batch);
+                      kv0 + j * BKV, batch);
         v_issued |= 1u << st;
         v_par = (v_par & ~(1u << st)) | (ph << st);
       }
@@ -284,7 +300,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(s_free);
-      const int valid = p.Skv - j * BKV;  // keys of this tile that exist
+      const int valid = kv_len - j * BKV;  // keys of this tile in this CTA's range
       if (valid < BKV) {
 #pragma unroll
         for (int c = 0; c < 4; ++c)
@@ -360,8 +376,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_after();
       const int qi = q_row0 + t * BQ + row;
       const bool live = qi < p.Sq;
-      bf16* orow = p.o + ((int64_t)batch * p.Sq + qi) * p.ldo + head * HD;
-      const int64_t li = ((int64_t)batch * p.H + head) * p.Sq + qi;
+      bf16* orow = p.o + split * p.o_split_stride + ((int64_t)batch * p.Sq + qi) * p.ldo + head * HD;
+      const int64_t li = split * p.lse_split_stride + ((int64_t)batch * p.H + head) * p.Sq + qi;
       const float lse_cur = (m_run + __log2f(l_run)) * 0.6931471805599453f;  // natural log
       // o = w_prev o_prev + w_cur (O / l): w_prev = 0, w_cur = 1 unless accumulating
       float w_prev = 0.0f, w_cur = 1.0f / l_run, lse_new = lse_cur;

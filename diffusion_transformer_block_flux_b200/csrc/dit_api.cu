@@ -533,9 +533,13 @@ dit_status dit_qk_norm_rope(const dit_bf16* q, const dit_bf16* k, int64_t ld_in,
 
 namespace {
 
+// splits > 1: o and lse are the partial-result arrays (split s at o + s
+// o_split_stride, lse + s lse_split_stride), kv_per_split a multiple of BKV
+// with every split non-empty; accumulate must be 0.
 dit_status attention_launch(const dit_bf16* q, const dit_bf16* k, const dit_bf16* v, int64_t ldq, int64_t ldk,
                             int64_t ldv, dit_bf16* o, int64_t ldo, float* lse, int B, int Sq, int Skv, int H,
-                            int head_dim, float softmax_scale, int accumulate, void* stream) {
+                            int head_dim, float softmax_scale, int accumulate, void* stream, int splits = 1,
+                            int kv_per_split = 0, int64_t o_split_stride = 0, int64_t lse_split_stride = 0) {
   if (q == nullptr || k == nullptr || v == nullptr || o == nullptr) return DIT_ERR_INVALID_ARG;
   if (head_dim != 128) return DIT_ERR_UNSUPPORTED;
   if (B < 1 || Sq < 1 || Skv < 1 || H < 1 || B > 65535 || H > 65535) return DIT_ERR_SHAPE;
@@ -559,9 +563,51 @@ dit_status attention_launch(const dit_bf16* q, const dit_bf16* k, const dit_bf16
   p.H = H;
   p.scale_log2 = softmax_scale * 1.4426950408889634f;
   p.accumulate = accumulate;
-  dim3 grid((unsigned)((Sq + 2 * dit::attn::BQ - 1) / (2 * dit::attn::BQ)), (unsigned)H, (unsigned)B);
+  p.splits = splits;
+  p.kv_per_split = splits > 1 ? kv_per_split : Skv;
+  p.o_split_stride = o_split_stride;
+  p.lse_split_stride = lse_split_stride;
+  if ((int64_t)B * splits > 65535) return DIT_ERR_SHAPE;
+  dim3 grid((unsigned)((Sq + 2 * dit::attn::BQ - 1) / (2 * dit::attn::BQ)), (unsigned)H, (unsigned)(B * splits));
   dit::attn::attention_kernel<<<grid, dit::attn::NUM_THREADS, dit::attn::SMEM_BYTES, (cudaStream_t)stream>>>(
       tq, tk, tv, p, g_wait_limit_ns);
+  return launch_status();
+}
+
+// Log-sum-exp merge of n parts, part j with row stride lds[j].
+dit_status merge_launch(int n, const dit_bf16* const* o_parts, const float* const* lse_parts, const int64_t* lds,
+                        dit_bf16* o, float* lse_out, int64_t ld_out, int B, int S, int H, void* stream) {
+  if (o == nullptr) return DIT_ERR_INVALID_ARG;
+  if (n < 1 || n > dit::kMergeMaxParts) return DIT_ERR_INVALID_ARG;
+  if (B < 1 || S < 1 || H < 1 || B > 65535 || H > 65535) return DIT_ERR_SHAPE;
+  const int64_t D = (int64_t)H * 128;
+  if (ld_out < D) return DIT_ERR_SHAPE;
+  if ((ld_out % 8) || !aligned16(o)) return DIT_ERR_ALIGNMENT;
+  dit::MergeParams p{};
+  for (int j = 0; j < n; ++j) {
+    if (o_parts[j] == nullptr || lse_parts[j] == nullptr) return DIT_ERR_INVALID_ARG;
+    if (lds[j] < D) return DIT_ERR_SHAPE;
+    if ((lds[j] % 8) || !aligned16(o_parts[j])) return DIT_ERR_ALIGNMENT;
+    p.o[j] = reinterpret_cast<const bf16*>(o_parts[j]);
+    p.lse[j] = lse_parts[j];
+    p.ld[j] = lds[j];
+  }
+  p.out = reinterpret_cast<bf16*>(o);
+  p.lse_out = lse_out;
+  p.ld_out = ld_out;
+  p.n = n;
+  p.B = B;
+  p.S = S;
+  p.H = H;
+  dit_status s = device_setup(nullptr);
+  if (s != DIT_OK) return s;
+  const dim3 grid((unsigned)((S + 15) / 16), (unsigned)H, (unsigned)B);
+  if (n <= 2)
+    dit::attention_merge_kernel<2><<<grid, 256, 0, (cudaStream_t)stream>>>(p);
+  else if (n <= 4)
+    dit::attention_merge_kernel<4><<<grid, 256, 0, (cudaStream_t)stream>>>(p);
+  else
+    dit::attention_merge_kernel<8><<<grid, 256, 0, (cudaStream_t)stream>>>(p);
   return launch_status();
 }
 
@@ -582,39 +628,76 @@ dit_status dit_attention_accumulate(const dit_bf16* q, const dit_bf16* k, const 
   return attention_launch(q, k, v, ldq, ldk, ldv, o, ldo, lse, B, Sq, Skv, H, head_dim, softmax_scale, 1, stream);
 }
 
+// Key ranges of a split launch: whole key tiles per split, every split non-empty.
+static void split_plan(int Skv, int n_split, int* splits, int* kv_per_split) {
+  const int tiles = (Skv + dit::attn::BKV - 1) / dit::attn::BKV;
+  int n = n_split < tiles ? n_split : tiles;
+  if (n < 1) n = 1;
+  const int per = (tiles + n - 1) / n;
+  *splits = (tiles + per - 1) / per;
+  *kv_per_split = per * dit::attn::BKV;
+}
+
+size_t dit_attention_split_workspace(int B, int Sq, int H, int n_split) {
+  if (B < 1 || Sq < 1 || H < 1 || n_split < 1) return 0;
+  const size_t n = (size_t)(n_split > dit::kAttnMaxSplits ? dit::kAttnMaxSplits : n_split);
+  return n * align256((size_t)B * Sq * H * 128 * sizeof(dit_bf16)) + n * align256((size_t)B * H * Sq * sizeof(float));
+}
+
+dit_status dit_attention_split(const dit_bf16* q, const dit_bf16* k, const dit_bf16* v, int64_t ldq, int64_t ldk,
+                               int64_t ldv, dit_bf16* o, int64_t ldo, float* lse, int B, int Sq, int Skv, int H,
+                               int head_dim, float softmax_scale, int n_split, int accumulate, void* workspace,
+                               size_t workspace_bytes, void* stream) {
+  if (n_split < 1 || n_split > dit::kAttnMaxSplits) return DIT_ERR_INVALID_ARG;
+  if (accumulate && lse == nullptr) return DIT_ERR_INVALID_ARG;
+  if (B < 1 || Sq < 1 || Skv < 1 || H < 1) return DIT_ERR_SHAPE;
+  int splits = 1, per = 0;
+  split_plan(Skv, n_split, &splits, &per);
+  if (splits == 1)
+    return attention_launch(q, k, v, ldq, ldk, ldv, o, ldo, lse, B, Sq, Skv, H, head_dim, softmax_scale, accumulate,
+                            stream);
+  if (workspace == nullptr) return DIT_ERR_WORKSPACE;
+  if (workspace_bytes < dit_attention_split_workspace(B, Sq, H, splits)) return DIT_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return DIT_ERR_ALIGNMENT;
+  const int64_t D = (int64_t)H * 128;
+  // the output is checked here because the merge, not the attention, writes it
+  if (o == nullptr) return DIT_ERR_INVALID_ARG;
+  if (ldo < D || B > 65535 || H > 65535) return DIT_ERR_SHAPE;
+  if ((ldo % 8) != 0 || !aligned16(o)) return DIT_ERR_ALIGNMENT;
+  const size_t o_bytes = align256((size_t)B * Sq * D * sizeof(dit_bf16));
+  dit_bf16* o_parts = reinterpret_cast<dit_bf16*>(workspace);
+  float* lse_parts = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(workspace) + (size_t)splits * o_bytes);
+  const size_t lse_bytes = align256((size_t)B * H * Sq * sizeof(float));
+  dit_status s = attention_launch(q, k, v, ldq, ldk, ldv, o_parts, D, lse_parts, B, Sq, Skv, H, head_dim,
+                                  softmax_scale, 0, stream, splits, per, (int64_t)(o_bytes / sizeof(dit_bf16)),
+                                  (int64_t)(lse_bytes / sizeof(float)));
+  if (s != DIT_OK) return s;
+  // merge the splits (and the running result when accumulating) into o, lse
+  const dit_bf16* op[dit::kMergeMaxParts];
+  const float* lp[dit::kMergeMaxParts];
+  int n = 0;
+  if (accumulate) {
+    op[n] = o;
+    lp[n] = lse;
+    ++n;
+  }
+  for (int j = 0; j < splits; ++j, ++n) {
+    op[n] = o_parts + (size_t)j * (o_bytes / sizeof(dit_bf16));
+    lp[n] = reinterpret_cast<const float*>(reinterpret_cast<const uint8_t*>(lse_parts) + (size_t)j * lse_bytes);
+  }
+  int64_t lds[dit::kMergeMaxParts];
+  for (int j = 0; j < n; ++j) lds[j] = D;
+  if (accumulate) lds[0] = ldo;  // the running result is both a part and the output
+  return merge_launch(n, op, lp, lds, o, lse, ldo, B, Sq, H, stream);
+}
+
 dit_status dit_attention_merge(int n, const dit_bf16* const* o_parts, const float* const* lse_parts, int64_t ld_in,
                                dit_bf16* o, float* lse_out, int64_t ld_out, int B, int S, int H, void* stream) {
-  if (o_parts == nullptr || lse_parts == nullptr || o == nullptr) return DIT_ERR_INVALID_ARG;
+  if (o_parts == nullptr || lse_parts == nullptr) return DIT_ERR_INVALID_ARG;
   if (n < 1 || n > dit::kMergeMaxParts) return DIT_ERR_INVALID_ARG;
-  if (B < 1 || S < 1 || H < 1 || B > 65535 || H > 65535) return DIT_ERR_SHAPE;
-  const int64_t D = (int64_t)H * 128;
-  if (ld_in < D || ld_out < D) return DIT_ERR_SHAPE;
-  if ((ld_in % 8) || (ld_out % 8) || !aligned16(o)) return DIT_ERR_ALIGNMENT;
-  dit::MergeParams p{};
-  for (int j = 0; j < n; ++j) {
-    if (o_parts[j] == nullptr || lse_parts[j] == nullptr) return DIT_ERR_INVALID_ARG;
-    if (!aligned16(o_parts[j])) return DIT_ERR_ALIGNMENT;
-    p.o[j] = reinterpret_cast<const bf16*>(o_parts[j]);
-    p.lse[j] = lse_parts[j];
-  }
-  p.out = reinterpret_cast<bf16*>(o);
-  p.lse_out = lse_out;
-  p.ld_in = ld_in;
-  p.ld_out = ld_out;
-  p.n = n;
-  p.B = B;
-  p.S = S;
-  p.H = H;
-  dit_status s = device_setup(nullptr);
-  if (s != DIT_OK) return s;
-  const dim3 grid((unsigned)((S + 15) / 16), (unsigned)H, (unsigned)B);
-  if (n <= 2)
-    dit::attention_merge_kernel<2><<<grid, 256, 0, (cudaStream_t)stream>>>(p);
-  else if (n <= 4)
-    dit::attention_merge_kernel<4><<<grid, 256, 0, (cudaStream_t)stream>>>(p);
-  else
-    dit::attention_merge_kernel<8><<<grid, 256, 0, (cudaStream_t)stream>>>(p);
-  return launch_status();
+  int64_t lds[dit::kMergeMaxParts];
+  for (int j = 0; j < n; ++j) lds[j] = ld_in;
+  return merge_launch(n, o_parts, lse_parts, lds, o, lse_out, ld_out, B, S, H, stream);
 }
 
 dit_status dit_gemm_epilogue(const dit_gemm_args* a, void* stream) {

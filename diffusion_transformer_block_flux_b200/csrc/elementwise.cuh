@@ -631,9 +631,10 @@ constexpr int kMergeMaxParts = 8;
 struct MergeParams {
   const bf16* o[kMergeMaxParts];
   const float* lse[kMergeMaxParts];
+  int64_t ld[kMergeMaxParts];  // row stride of each part, elements
   bf16* out;
   float* lse_out;
-  int64_t ld_in, ld_out;
+  int64_t ld_out;
   int n, B, S, H;
 };
 
@@ -654,7 +655,7 @@ __global__ void __launch_bounds__(256) attention_merge_kernel(const __grid_const
   for (int j = 0; j < NP; ++j) {
     const bool on = valid && j < p.n;
     l[j] = on ? p.lse[j][li] : -INFINITY;
-    u[j] = on ? *reinterpret_cast<const uint4*>(p.o[j] + bs * p.ld_in + col) : make_uint4(0, 0, 0, 0);
+    u[j] = on ? *reinterpret_cast<const uint4*>(p.o[j] + bs * p.ld[j] + col) : make_uint4(0, 0, 0, 0);
   }
   float m = l[0];
 #pragma unroll

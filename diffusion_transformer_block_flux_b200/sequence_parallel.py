@@ -44,6 +44,17 @@ def _cuda_attn_acc(q, k, v, o, lse, H):
     dit_attention_accumulate(q, k, v, o, lse, 1, q.shape[0], k.shape[0], H)
 
 
+def auto_key_splits(S_loc, H, device):
+    """Key splits for the local attention of S_loc queries: the attention
+    kernel runs one CTA per 256 queries and head, so a short local sequence
+    leaves SMs idle (576 queries x 24 heads: 72 CTAs on 148 SMs); splitting the
+    keys into parts merged by log-sum-exp (dit_attention_split) fills them."""
+    import torch
+    sms = torch.cuda.get_device_properties(device).multi_processor_count
+    ctas = -(-S_loc // 256) * H
+    return max(1, min(4, sms // max(1, ctas)))
+
+
 class RingAttention:
     """One rank's ring attention with buffers owned by the plan.
 
@@ -62,9 +73,15 @@ class RingAttention:
     the plan).
 
     With `attn` and `merge` given (the CPU tests' oracle operations), a later
-    step writes its own result to a partial buffer and `merge` folds it in."""
+    step writes its own result to a partial buffer and `merge` folds it in.
 
-    def __init__(self, S_loc, H, device, dtype=None, group=None, attn=None, merge=None, shards_per_step=1):
+    key_splits (CUDA operations only): each step's keys are cut into that many
+    parts computed side by side and merged by log-sum-exp
+    (dit_attention_split), for local query counts too small to fill the GPU;
+    None picks it from the SM count (auto_key_splits)."""
+
+    def __init__(self, S_loc, H, device, dtype=None, group=None, attn=None, merge=None, shards_per_step=1,
+                 key_splits=None):
         import torch
         import torch.distributed as dist
         dtype = dtype or torch.bfloat16
@@ -77,6 +94,13 @@ class RingAttention:
         self.merge = merge or _cuda_merge
         self.acc = None if custom else _cuda_attn_acc
         D = H * 128
+        self.splits = 1
+        if not custom:
+            from . import dit_attention_split_workspace
+            self.splits = int(key_splits) if key_splits is not None else auto_key_splits(S_loc, H, device)
+            if self.splits > 1:
+                self.ws = torch.empty(dit_attention_split_workspace(1, S_loc, H, self.splits), dtype=torch.uint8,
+                                      device=device)
         slots = 2 * self.G if self.N > self.G else self.G  # two stages in flight while more shards follow
         self.slots = slots
         self.k = torch.empty((slots * S_loc, D), dtype=dtype, device=device)
@@ -95,7 +119,11 @@ class RingAttention:
     def _step(self, q, first_slot, n, out, first):
         H = self.H
         kk, vv = self.k[self._rows(first_slot, n)], self.v[self._rows(first_slot, n)]
-        if first:
+        if self.splits > 1:
+            from . import dit_attention_split
+            dit_attention_split(q, kk, vv, out, 1, q.shape[0], kk.shape[0], H, self.splits, self.ws, lse=self.lse,
+                                accumulate=not first)
+        elif first:
             self.attn(q, kk, vv, out, self.lse, H)
         elif self.acc is not None:
             self.acc(q, kk, vv, out, self.lse, H)
@@ -170,9 +198,9 @@ class UlyssesAttention:
         return out
 
 
-def ring_attention(q, k, v, out, H, group=None, attn=None, merge=None, shards_per_step=1):
+def ring_attention(q, k, v, out, H, group=None, attn=None, merge=None, shards_per_step=1, key_splits=None):
     """One-off ring attention (a plan built for this call); see RingAttention."""
-    plan = RingAttention(q.shape[0], H, q.device, q.dtype, group, attn, merge, shards_per_step)
+    plan = RingAttention(q.shape[0], H, q.device, q.dtype, group, attn, merge, shards_per_step, key_splits)
     lse = plan(q, k, v, out)
     return lse[0]
 
@@ -226,7 +254,7 @@ class SequenceParallelSingleBlock:
     [1, D] bf16; rope: this shard's rows of the RoPE table [S/N, 64, 2] fp32."""
 
     def __init__(self, S_loc, D, H, M, device, group=None, mode="ring", ops=None, attn=None, merge=None,
-                 dtype=None, eps=1e-6, shards_per_step=1):
+                 dtype=None, eps=1e-6, shards_per_step=1, key_splits=None):
         import torch
         dtype = dtype or torch.bfloat16
         if mode not in ("ring", "ulysses"):
@@ -238,7 +266,7 @@ class SequenceParallelSingleBlock:
         self.qkv = torch.empty((S_loc, 3 * D), dtype=dtype, device=device)
         self.cat = torch.empty((S_loc, D + M), dtype=dtype, device=device)
         if mode == "ring":
-            self.attention = RingAttention(S_loc, H, device, dtype, group, attn, merge, shards_per_step)
+            self.attention = RingAttention(S_loc, H, device, dtype, group, attn, merge, shards_per_step, key_splits)
         else:
             self.attention = UlyssesAttention(S_loc, H, device, dtype, group, attn)
 

@@ -209,6 +209,32 @@ dit_status dit_attention_accumulate(const dit_bf16* q, const dit_bf16* k, const 
                                     float* lse, int B, int Sq, int Skv, int H, int head_dim,
                                     float softmax_scale, void* stream);
 
+/* Attention with the keys split across CTAs, for query sets too short to fill
+ * the GPU (one rank of a sequence-parallel ring: [CG] §5, 576 queries per GPU
+ * at CP = 8).  The key range is cut into n_split contiguous parts of whole
+ * 128-key tiles (fewer when Skv has fewer tiles); one launch computes the
+ * attention of every query tile over every part, each part's result (bf16)
+ * and lse (fp32) going to the workspace, and the log-sum-exp merge
+ * (dit_attention_merge) combines the parts into o and lse.  accumulate = 0:
+ * the result is dit_attention's over k, v, with one more bf16 rounding of
+ * each part; lse may be NULL.  accumulate = 1: o and lse (required) hold a
+ * running result on entry, as for dit_attention_accumulate, and the merge
+ * includes it.  n_split: 1..4 (1 behaves as dit_attention or
+ * dit_attention_accumulate and needs no workspace).  workspace: device, 256-byte
+ * aligned, at least dit_attention_split_workspace(B, Sq, H, n_split) bytes,
+ * owned by the caller and reusable once the stream has passed this call.
+ * Other arguments and errors as dit_attention; DIT_ERR_WORKSPACE when the
+ * workspace is missing or too small.  Two launches, no synchronisation,
+ * capturable. */
+dit_status dit_attention_split(const dit_bf16* q, const dit_bf16* k, const dit_bf16* v,
+                               int64_t ldq, int64_t ldk, int64_t ldv, dit_bf16* o, int64_t ldo,
+                               float* lse, int B, int Sq, int Skv, int H, int head_dim,
+                               float softmax_scale, int n_split, int accumulate, void* workspace,
+                               size_t workspace_bytes, void* stream);
+
+/* Bytes of workspace dit_attention_split needs (0 for invalid sizes). */
+size_t dit_attention_split_workspace(int B, int Sq, int H, int n_split);
+
 /* Merge of attention results over disjoint key sets ([CG] §5: sequence-
  * parallel ring attention merges each hop's partial result by its
  * log-sum-exp):

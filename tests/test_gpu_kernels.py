@@ -417,6 +417,69 @@ def test_attention_accumulate_over_key_splits(cuts):
     assert_no_device_error()
 
 
+@pytest.mark.parametrize("B,Sq,Skv,H,n_split", [
+    (1, 300, 600, 3, 2),    # 5 key tiles: parts of 3 + 2 tiles, ragged last tile
+    (1, 576, 4608, 2, 2),   # one rank of a CP = 8 ring, all shards at once
+    (2, 130, 1000, 2, 3),   # batch 2, three parts, ragged query and key tails
+    (1, 200, 900, 2, 4),    # 8 tiles in four parts of two
+    (1, 100, 100, 2, 4),    # one key tile: no split, no workspace needed
+])
+def test_attention_split_matches_oracle(B, Sq, Skv, H, n_split):
+    """dit_attention_split cuts the keys into parts computed by separate CTAs
+    of one launch and merges them by log-sum-exp: the result is the attention
+    over all keys (fp64 oracle) with its log-sum-exp.  Each part is rounded to
+    bf16 before the merge rounds once more: max abs <= 3e-2 RMS + 2 x 2^-9
+    max|ref|."""
+    import torch
+    D = H * 128
+    q, k, v = _attn_case(B, Sq, Skv, H, 2.0, seed=21)
+    dq, dk, dv = dev_bf16(q), dev_bf16(k), dev_bf16(v)
+    o = torch.empty((B * Sq, D), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((B, H, Sq), dtype=torch.float32, device="cuda")
+    nbytes = dit.dit_attention_split_workspace(B, Sq, H, n_split)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    dit.dit_attention_split(dq, dk, dv, o, B, Sq, Skv, H, n_split, ws, lse=lse)
+    torch.cuda.synchronize()
+    qf, kf, vf = (synth.bf16_bits_to_f64(t) for t in (q, k, v))
+    got = host_f64(o)
+    for b in range(B):
+        rows = slice(b * Sq, (b + 1) * Sq)
+        kr = slice(b * Skv, (b + 1) * Skv)
+        ref = O.attention(qf[rows], kf[kr], vf[kr], H)
+        rms = np.sqrt(np.mean(ref ** 2))
+        parity(got[rows], ref, f"split attention, batch {b}",
+               max_abs_frac=3e-2 + 2 * 2.0 ** -9 * np.abs(ref).max() / rms)
+        ref_lse = O.attention_lse(qf[rows], kf[kr], H)
+        assert np.abs(lse[b].cpu().double().numpy() - ref_lse).max() < 1e-3 * max(1.0, np.abs(ref_lse).max())
+    assert_no_device_error()
+
+
+def test_attention_split_accumulates_like_a_ring():
+    """A ring over three uneven key shards with two parts per step: the first
+    step writes the running result, the later ones merge into it
+    (accumulate = 1); the result is the attention over all keys."""
+    import torch
+    H, Sq = 2, 256
+    D = H * 128
+    cuts = (0, 700, 1100, 1800)
+    q, k, v = _attn_case(1, Sq, cuts[-1], H, 2.0, seed=23)
+    dq, dk, dv = dev_bf16(q), dev_bf16(k), dev_bf16(v)
+    o = torch.empty((Sq, D), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((1, H, Sq), dtype=torch.float32, device="cuda")
+    ws = torch.empty(dit.dit_attention_split_workspace(1, Sq, H, 2), dtype=torch.uint8, device="cuda")
+    for i, (a, b) in enumerate(zip(cuts, cuts[1:])):
+        dit.dit_attention_split(dq, dk[a:b], dv[a:b], o, 1, Sq, b - a, H, 2, ws, lse=lse, accumulate=i > 0)
+    torch.cuda.synchronize()
+    qf, kf, vf = (synth.bf16_bits_to_f64(t) for t in (q, k, v))
+    ref = O.attention(qf, kf, vf, H)
+    rms = np.sqrt(np.mean(ref ** 2))
+    # each step: the parts and the running result are rounded once more
+    parity(host_f64(o), ref, "split ring", max_abs_frac=3e-2 + 6 * 2.0 ** -9 * np.abs(ref).max() / rms)
+    ref_lse = O.attention_lse(qf, kf, H)
+    assert np.abs(lse[0].cpu().double().numpy() - ref_lse).max() < 1e-3 * max(1.0, np.abs(ref_lse).max())
+    assert_no_device_error()
+
+
 def test_sequence_parallel_drivers_with_cuda_kernels_one_rank():
     """ring_attention and ulysses_attention with their default CUDA local
     operations in a one-rank NCCL group (no transfer; the multi-rank
@@ -440,11 +503,20 @@ def test_sequence_parallel_drivers_with_cuda_kernels_one_rank():
         ref = torch.empty((S, D), dtype=torch.bfloat16, device="cuda")
         dit.dit_attention(dq, dk, dv, ref, 1, S, S, H)
         o_ring = torch.empty_like(ref)
-        sp.ring_attention(dq, dk, dv, o_ring, H)
+        sp.ring_attention(dq, dk, dv, o_ring, H, key_splits=1)
         o_uly = torch.empty_like(ref)
         sp.ulysses_attention(dq, dk, dv, o_uly, H)
+        # the plan's default for so few query tiles cuts the keys (dit_attention_split)
+        o_split = torch.empty_like(ref)
+        sp.ring_attention(dq, dk, dv, o_split, H)
         torch.cuda.synchronize()
         assert torch.equal(o_ring, ref) and torch.equal(o_uly, ref)
+        assert sp.auto_key_splits(S, H, "cuda") > 1
+        qf, kf, vf = (synth.bf16_bits_to_f64(t) for t in (q, k, v))
+        oref = O.attention(qf, kf, vf, H)
+        rms = np.sqrt(np.mean(oref ** 2))
+        parity(host_f64(o_split), oref, "ring with split keys",
+               max_abs_frac=3e-2 + 2 * 2.0 ** -9 * np.abs(oref).max() / rms)
     finally:
         dist.destroy_process_group()
     assert_no_device_error()
@@ -482,7 +554,7 @@ def test_sequence_parallel_block_one_rank_equals_block_and_graph_replays_it(mode
         ws = torch.empty(dit.dit_single_block_workspace(cfg), dtype=torch.uint8, device="cuda")
         ref = torch.empty_like(x)
         dit.dit_single_block_fwd(cfg, dit.single_weights(w), x, vec, rope, ref, ws)
-        blk = sp.SequenceParallelSingleBlock(s.S, s.D, s.H, s.M, "cuda", mode=mode)
+        blk = sp.SequenceParallelSingleBlock(s.S, s.D, s.H, s.M, "cuda", mode=mode, key_splits=1)
         out = torch.empty_like(x)
         blk.forward(w, x, vec, rope, out)
         torch.cuda.synchronize()
