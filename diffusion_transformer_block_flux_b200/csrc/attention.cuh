@@ -286,38 +286,49 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // so the issuing thread spends no commit on it)
       if (t == 1 && lane == 0) mbar_arrive(&k_empty[j & 1]);
       tc_fence_after();
+      // Scores in two halves: the row max of keys 0..63 runs while keys
+      // 64..127 are still on their way from TMEM.
       uint32_t r[4][32];
+      const int valid = kv_len - j * BKV;  // keys of this tile in this CTA's range
+      auto mask = [&](int c) {
+        if (valid < BKV) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (c * 32 + i >= valid) r[c][i] = __float_as_uint(-INFINITY);
+        }
+      };
+      // max of 32 scores: two independent chains of 3-input max
+      auto cmax = [&](int c) -> float {
+        float a = fmaxf(__uint_as_float(r[c][0]), __uint_as_float(r[c][1]));
+        float b = fmaxf(__uint_as_float(r[c][2]), __uint_as_float(r[c][3]));
+#pragma unroll
+        for (int i = 4; i < 32; i += 4) {
+          a = max3f(a, __uint_as_float(r[c][i]), __uint_as_float(r[c][i + 1]));
+          b = max3f(b, __uint_as_float(r[c][i + 2]), __uint_as_float(r[c][i + 3]));
+        }
+        return fmaxf(a, b);
+      };
       tmem_ld32_nowait(tS + 0u, r[0]);
       tmem_ld32_nowait(tS + 32u, r[1]);
-      tmem_ld32_nowait(tS + 64u, r[2]);
-      tmem_ld32_nowait(tS + 96u, r[3]);
       tmem_wait_ld();
       reg_fence32(r[0]);
       reg_fence32(r[1]);
+      tmem_ld32_nowait(tS + 64u, r[2]);
+      tmem_ld32_nowait(tS + 96u, r[3]);
+      mask(0);
+      mask(1);
+      float m01 = fmaxf(cmax(0), cmax(1));
+      asm volatile("" : "+f"(m01));  // computed before the wait below
+      tmem_wait_ld();
       reg_fence32(r[2]);
       reg_fence32(r[3]);
       // the scores are in registers: S may take the other tile's next scores
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(s_free);
-      const int valid = kv_len - j * BKV;  // keys of this tile in this CTA's range
-      if (valid < BKV) {
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (c * 32 + i >= valid) r[c][i] = __float_as_uint(-INFINITY);
-      }
-      // row max: four independent chains of 3-input max
-      float mx[4];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        float a = fmaxf(__uint_as_float(r[c][0]), __uint_as_float(r[c][1]));
-#pragma unroll
-        for (int i = 2; i < 32; i += 2) a = max3f(a, __uint_as_float(r[c][i]), __uint_as_float(r[c][i + 1]));
-        mx[c] = a;
-      }
-      const float m_tile = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2;
+      mask(2);
+      mask(3);
+      const float m_tile = fmaxf(m01, fmaxf(cmax(2), cmax(3))) * sl2;
       const bool need = m_tile > m_run + 8.0f;  // always true on the first tile
       const float m_new = need ? m_tile : m_run;
       const float alpha = need ? ex2_fast(m_run - m_new) : 1.0f;  // 0 on the first tile
