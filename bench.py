@@ -256,6 +256,8 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     dit.lib()  # raises if the CUDA library is missing
+    if args.l2_keep_weights_mb:
+        dit.dit_set_weight_l2_persist(args.l2_keep_weights_mb << 20)
     w, x, vec = make_block(torch, dev, seed=1234 + rank)
     ids = torch.from_numpy(synth.flux_ids(S_TXT, GRID, GRID)).to(dev)
     rope = torch.empty((S, 64, 2), dtype=torch.float32, device=dev)
@@ -395,7 +397,9 @@ def run_ours(args, rank, world, local_rank):
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": WORKLOAD, "global_batch": world, "seq_len": S, "parallelism": f"replicas{world}",
-                   "l2": "inputs larger than L2 (282 MB of block weights + 0.25 GB activations per step)"},
+                   "l2": "inputs larger than L2 (282 MB of block weights + 0.25 GB activations per step)"
+                         + (f"; {args.l2_keep_weights_mb} MB persisting L2 set-aside for the output GEMM's weight"
+                            if args.l2_keep_weights_mb else "")},
         "ms_per_block": round(ms_per_step, 4), "blocks_per_s": round(world * 1e3 / ms_per_step, 1),
         "block_frac_of_bf16_peak": round(block_frac, 4),
         "gpu_launches": len(KERNELS) * K,
@@ -924,6 +928,8 @@ def main():
                     help="loop workload: 'double,single' block counts instead of 19,38 (same width)")
     ap.add_argument("--loop-steps", type=int, default=0,
                     help="loop workload: Euler steps instead of 50")
+    ap.add_argument("--l2-keep-weights-mb", type=int, default=0,
+                    help="persisting L2 set-aside (MB) for the output GEMMs' weights (dit_set_weight_l2_persist); 0 = off")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -130,6 +130,7 @@ _SIGS = {
                             i32, i32, i32, f32, c_void_p]),
     "dit_attention_accumulate": (i32, [c_void_p, c_void_p, c_void_p, i64, i64, i64, c_void_p, i64, c_void_p, i32,
                                        i32, i32, i32, i32, f32, c_void_p]),
+    "dit_set_weight_l2_persist": (i32, [size_t]),
     "dit_attention_split": (i32, [c_void_p, c_void_p, c_void_p, i64, i64, i64, c_void_p, i64, c_void_p, i32, i32,
                                   i32, i32, i32, f32, i32, i32, c_void_p, size_t, c_void_p]),
     "dit_attention_split_workspace": (size_t, [i32, i32, i32, i32]),
@@ -304,6 +305,12 @@ def dit_attention_accumulate(q, k, v, o, lse, B, Sq, Skv, H, softmax_scale=None,
         softmax_scale = 128 ** -0.5
     _call("dit_attention_accumulate", _ptr(q), _ptr(k), _ptr(v), q.stride(0), k.stride(0), v.stride(0), _ptr(o),
           o.stride(0), _ptr(lse), B, Sq, Skv, H, 128, float(softmax_scale), _stream(stream))
+
+
+def dit_set_weight_l2_persist(nbytes):
+    """Opt-in L2 residency of the output GEMMs' weights (a process-wide
+    persisting L2 set-aside of nbytes on the current device; 0 turns it off)."""
+    _call("dit_set_weight_l2_persist", int(nbytes))
 
 
 def dit_attention_split_workspace(B, Sq, H, n_split):

@@ -42,6 +42,9 @@ struct DeviceInfo {
   bool supported = false;
   int num_sms = 0;
   bool attrs_set = false;
+  // dit_set_weight_l2_persist: N-fastest GEMMs keep their weight in the
+  // persisting L2 set-aside
+  std::atomic<bool> keep_weights{false};
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -252,6 +255,19 @@ size_t dit_abi_struct_size(int which) {
     case 7: return sizeof(dit_loop_io);
     default: return 0;
   }
+}
+
+dit_status dit_set_weight_l2_persist(size_t bytes) {
+  int dev = 0;
+  DIT_CUDA_CHECK(cudaGetDevice(&dev));
+  dit_status s = device_setup(nullptr);
+  if (s != DIT_OK) return s;
+  int maxp = 0;
+  DIT_CUDA_CHECK(cudaDeviceGetAttribute(&maxp, cudaDevAttrMaxPersistingL2CacheSize, dev));
+  const size_t want = bytes < (size_t)maxp ? bytes : (size_t)maxp;
+  DIT_CUDA_CHECK(cudaDeviceSetLimit(cudaLimitPersistingL2CacheSize, want));
+  g_dev[dev].keep_weights.store(want > 0, std::memory_order_relaxed);
+  return DIT_OK;
 }
 
 dit_status dit_set_wait_limit_ns(uint64_t limit_ns) {
@@ -767,6 +783,8 @@ dit_status dit_gemm_epilogue(const dit_gemm_args* a, void* stream) {
   ep.k_scale = reinterpret_cast<const bf16*>(a->k_scale);
   ep.rope = reinterpret_cast<const float2*>(a->rope);
   ep.rope_rows = a->rope_rows > 0 ? a->rope_rows : a->M;
+  ep.w_keep = nullptr;
+  ep.w_keep_bytes = 0;
   cudaStream_t st = (cudaStream_t)stream;
   if (use_pair) {
     namespace P = dit::gemm::pair;
@@ -775,6 +793,17 @@ dit_status dit_gemm_epilogue(const dit_gemm_args* a, void* stream) {
     const int grid = 2 * clusters;
     // walk the larger operand's panels once: N-fastest when A (M x K) is the larger
     const int nf = a->M > a->N ? 1 : 0;
+    int dev = 0;
+    if (nf && cudaGetDevice(&dev) == cudaSuccess && g_dev[dev].keep_weights.load(std::memory_order_relaxed)) {
+      // whole 128-byte lines inside the weight: the kernel returns them to normal L2 priority at the end
+      const uintptr_t w0 = reinterpret_cast<uintptr_t>(a->W);
+      const uintptr_t lo = (w0 + 127) & ~(uintptr_t)127;
+      const uintptr_t hi = (w0 + (uintptr_t)a->N * (uintptr_t)a->ldw * 2) & ~(uintptr_t)127;
+      if (hi > lo) {
+        ep.w_keep = reinterpret_cast<const uint8_t*>(lo);
+        ep.w_keep_bytes = (int64_t)(hi - lo);
+      }
+    }
     switch (a->epi) {
       case DIT_EPI_NONE:
         P::gemm_pair_kernel<DIT_EPI_NONE><<<grid, P::NUM_THREADS, P::SMEM_BYTES, st>>>(tA, tB, a->M, a->N, a->K, ep,

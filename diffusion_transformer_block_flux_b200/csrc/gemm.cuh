@@ -58,6 +58,12 @@ struct Epi {
   const bf16* k_scale;
   const float2* rope;  // [rope_rows][64] (cos, sin); row of output row m = m % rope_rows
   int rope_rows;
+  // Weight kept in L2 (pair kernel, N-fastest raster, with a persisting L2
+  // set-aside): the weight's loads take the evict-last policy, and when a CTA
+  // is done it returns its share of [w_keep, w_keep + w_keep_bytes) to normal
+  // priority, so the next kernels get the whole L2 back.  nullptr: off.
+  const uint8_t* w_keep;
+  int64_t w_keep_bytes;
 };
 
 // One 128-column head of q or k for output row m: bias, optional RMSNorm with
@@ -475,6 +481,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       uint32_t issued_mask = 0, issued_parity = 0;
       bool ok = true;
       int wave = 0;  // this cluster's tile count so far: the same for every cluster of a wave
+      const bool keep_b = n_fastest && ep.w_keep != nullptr;
+      const uint64_t b_policy = l2_policy_evict_last();
       for (int tile = cluster_id; tile < num_tiles && ok; tile += n_clusters, ++wave) {
         int tm, tn;
         tile_coords(tile, num_m, num_n, n_fastest, tm, tn);
@@ -490,7 +498,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
           const uint32_t leader_full = mapa_shared(smem_u32(&full[stage]), 0);
           const int kx = (back ? num_kb - 1 - kb : kb) * BK;
           tma_load_2d_pair(sA + stage * A_BYTES, &tmA, leader_full, kx, tm * BM + (int)rank * BM_CTA);
-          tma_load_2d_pair(sB + stage * B_BYTES, &tmB, leader_full, kx, tn * BN + (int)rank * BN_CTA);
+          if (keep_b)
+            tma_load_2d_pair_hint(sB + stage * B_BYTES, &tmB, leader_full, kx, tn * BN + (int)rank * BN_CTA,
+                                  b_policy);
+          else
+            tma_load_2d_pair(sB + stage * B_BYTES, &tmB, leader_full, kx, tn * BN + (int)rank * BN_CTA);
           issued_mask |= 1u << stage;
           issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) {
@@ -598,6 +610,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
   cluster_sync_all();  // no CTA leaves while its peer may still touch its memory
   tc_fence_after();
   if (warp == 1) tmem_dealloc_pair(tmem_base, TMEM_COLS);
+  if (n_fastest && ep.w_keep != nullptr) {
+    // this CTA's share of the kept weight back to normal L2 priority
+    const int64_t lines = ep.w_keep_bytes >> 7;
+    for (int64_t i = (int64_t)blockIdx.x * NUM_THREADS + threadIdx.x; i < lines; i += (int64_t)gridDim.x * NUM_THREADS)
+      l2_priority_normal(ep.w_keep + (i << 7));
+  }
 }
 
 }  // namespace pair

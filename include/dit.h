@@ -96,6 +96,19 @@ dit_status dit_clear_device_error(void* stream);
  * 2e9).  Applies to kernels launched after the call. */
 dit_status dit_set_wait_limit_ns(uint64_t limit_ns);
 
+/* Opt-in L2 residency for the weight of the output GEMMs (the projections
+ * whose activation operand is larger than their weight, e.g. the single-stream
+ * block's [attn | mlp] x W2, 94 MB at the Flux width).  Those GEMMs visit
+ * their tiles N-fastest, so every wave of tiles re-reads the whole weight; with
+ * this set, the weight's loads take the L2 evict-last policy, and at the end of
+ * the GEMM each CTA returns its share of the weight to normal priority.
+ * bytes: size of the persisting L2 set-aside, clipped to the device maximum
+ * (cudaDevAttrMaxPersistingL2CacheSize); 0 turns it off.  This sets
+ * cudaLimitPersistingL2CacheSize, a limit of the calling process's context on
+ * the current device that every kernel of the process shares, until it is set
+ * again or the context ends.  Affects GEMMs launched after the call. */
+dit_status dit_set_weight_l2_persist(size_t bytes);
+
 /* Failure-detection self test: launches one CTA that waits on a barrier that
  * nothing ever arrives on, with the given limit.  The kernel must give up,
  * record DIT_ERR_TIMEOUT in the device error word and exit.  Enqueued on

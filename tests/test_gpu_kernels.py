@@ -226,6 +226,33 @@ def test_gemm_gated_residual(M, rows_per_batch, N, K, inplace):
     parity(host_f64(out_s), xsf + g * y, "gated residual, small residual")
 
 
+def test_weight_l2_persist_changes_no_bits():
+    """With the opt-in L2 residency of the output GEMM's weight, the N-fastest
+    GEMM (M > N) loads its weight with the evict-last policy and demotes it at
+    the end: a caching hint, so the output equals the plain call bit for bit,
+    and the oracle's.  The process-wide set-aside is turned off again."""
+    import torch
+    M, N, K = 1024, 256, 2048
+    A, W, b = _gemm_inputs(M, N, K, seed=17)
+    x = synth.normal_bf16(5, "x", (M, N))
+    gate = synth.bf16_bits_to_f64(synth.normal_bf16(6, "g", (1, N), 0.7))
+    dA, dW, db, dx, dg = dev_bf16(A), dev_bf16(W), dev_bf16(b), dev_bf16(x), f32dev(gate)
+    plain = torch.empty_like(dx)
+    kept = torch.empty_like(dx)
+    dit.dit_gemm_epilogue(dA, dW, plain, dit.DIT_EPI_BIAS_GATED_RESIDUAL, bias=db, gate=dg, gate_stride=N, resid=dx)
+    try:
+        dit.dit_set_weight_l2_persist(64 << 20)
+        dit.dit_gemm_epilogue(dA, dW, kept, dit.DIT_EPI_BIAS_GATED_RESIDUAL, bias=db, gate=dg, gate_stride=N,
+                              resid=dx)
+        torch.cuda.synchronize()
+    finally:
+        dit.dit_set_weight_l2_persist(0)
+    assert torch.equal(plain, kept)
+    y = O.linear(synth.bf16_bits_to_f64(A), synth.bf16_bits_to_f64(W), synth.bf16_bits_to_f64(b))
+    parity(host_f64(kept), synth.bf16_bits_to_f64(x) + gate * y, "gated residual, weight kept in L2")
+    assert_no_device_error()
+
+
 # ---------------------------------------------------------------- attention
 
 def _attn_case(B, Sq, Skv, H, qmul=1.0, seed=0):
