@@ -123,6 +123,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  griddep_wait();  // the prologue above overlaps the previous kernel; everything below follows it
+  griddep_launch_dependents();
 
   if (warp == 8) {
     if (lane == 0) {

@@ -48,6 +48,23 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 }
 
 // ---------------------------------------------------------------------------
+// Programmatic dependent launch.  A kernel launched with the programmatic
+// stream-serialization attribute may start while the previous kernel of the
+// stream is still running; griddep_wait() returns once that kernel (and so,
+// transitively, every earlier one) has completed and its writes are visible.
+// Every kernel here calls it in every CTA before its first global-memory
+// access, so stream order holds for all the data a kernel reads or writes;
+// only its prologue (barrier init, TMEM allocation, descriptor prefetch)
+// overlaps the previous kernel.  Without the attribute both are no-ops.
+// griddep_launch_dependents() lets the next kernel start launching once every
+// CTA of this one has issued it.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------
 // mbarrier
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {

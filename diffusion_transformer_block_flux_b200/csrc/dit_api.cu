@@ -1,3 +1,4 @@
+#include <cstdlib>
 // C ABI of libdit: argument checks, TMA descriptor encoding and kernel
 // launches for every entry point declared in include/dit.h.
 //
@@ -71,6 +72,44 @@ inline dit_status cuda_fail(cudaError_t e) {
 dit_status launch_status() {
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? DIT_OK : cuda_fail(e);
+}
+
+// Kernels of the block path are launched with programmatic stream
+// serialization: a launch may begin while the previous kernel of the stream
+// drains, and each of these kernels holds every global-memory access behind
+// griddep_wait() (common.cuh), so only prologues overlap.  DIT_DISABLE_PDL=1
+// in the environment launches them the plain way.  Errors surface through the
+// caller's launch_status().
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* v = getenv("DIT_DISABLE_PDL");
+    return !(v != nullptr && v[0] == '1');
+  }();
+  return on;
+}
+
+// Set while a profiled call records events between its kernels: those
+// launches go the plain way, so each kernel's interval is its own.
+thread_local bool t_plain_launches = false;
+struct PlainLaunches {
+  bool prev;
+  PlainLaunches() : prev(t_plain_launches) { t_plain_launches = true; }
+  ~PlainLaunches() { t_plain_launches = prev; }
+};
+
+template <typename... KArgs, typename... Args>
+void launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = (pdl_enabled() && !t_plain_launches) ? 1 : 0;
+  (void)cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
 // Per-device setup: SM count, capability check, kernel attributes, driver
@@ -340,10 +379,10 @@ dit_status dit_vec_linear(const dit_bf16* x, int64_t ldx, const dit_bf16* W, int
 #define DIT_VR_CASE(KC_)                                                                                       \
   case KC_:                                                                                                    \
     if (B == 1)                                                                                                \
-      dit::vec_rows_kernel<KC_, 1><<<(unsigned)grid, 512, xs_smem, st>>>(xb, ldx, Wb, ldw, bb, out, ldo, N, K, \
+      launch_pdl(dit::vec_rows_kernel<KC_, 1>, (unsigned)grid, 512, xs_smem, st, xb, ldx, Wb, ldw, bb, out, ldo, N, K, \
                                                                          flags);                               \
     else                                                                                                       \
-      dit::vec_rows_kernel<KC_, 2><<<(unsigned)grid, 512, xs_smem, st>>>(xb, ldx, Wb, ldw, bb, out, ldo, N, K, \
+      launch_pdl(dit::vec_rows_kernel<KC_, 2>, (unsigned)grid, 512, xs_smem, st, xb, ldx, Wb, ldw, bb, out, ldo, N, K, \
                                                                          flags);                               \
     return launch_status();
     switch (K / 256) {
@@ -424,7 +463,7 @@ dit_status multi_linear(const dit_bf16* x, const dit::MultiLinear& p, int flags,
     switch (p.K / 256) {
 #define DIT_VRM_CASE(KC_)                                                                          \
   case KC_:                                                                                        \
-    dit::vec_rows_multi_kernel<KC_><<<(unsigned)rgrid, 512, xs_smem, st>>>(xr, p, flags);         \
+    launch_pdl(dit::vec_rows_multi_kernel<KC_>, (unsigned)rgrid, 512, xs_smem, st, xr, p, flags);         \
     return launch_status();
       DIT_VRM_CASE(1)
       DIT_VRM_CASE(2)
@@ -501,16 +540,16 @@ dit_status dit_modulate_norm(const dit_bf16* x, int64_t ldx, const float* shift,
       const dim3 grid((unsigned)S, (unsigned)B);
       const int threads = D / (8 * NC);
       if (NC == 1)
-        dit::modulate_norm_row_kernel<1><<<grid, threads, 0, st>>>(xb, ldx, shift, scale, mod_stride, yb, ldy, S, D,
+        launch_pdl(dit::modulate_norm_row_kernel<1>, grid, threads, 0, st, xb, ldx, shift, scale, mod_stride, yb, ldy, S, D,
                                                                     eps);
       else if (NC == 2)
-        dit::modulate_norm_row_kernel<2><<<grid, threads, 0, st>>>(xb, ldx, shift, scale, mod_stride, yb, ldy, S, D,
+        launch_pdl(dit::modulate_norm_row_kernel<2>, grid, threads, 0, st, xb, ldx, shift, scale, mod_stride, yb, ldy, S, D,
                                                                     eps);
       else if (NC == 3)
-        dit::modulate_norm_row_kernel<3><<<grid, threads, 0, st>>>(xb, ldx, shift, scale, mod_stride, yb, ldy, S, D,
+        launch_pdl(dit::modulate_norm_row_kernel<3>, grid, threads, 0, st, xb, ldx, shift, scale, mod_stride, yb, ldy, S, D,
                                                                     eps);
       else
-        dit::modulate_norm_row_kernel<4><<<grid, threads, 0, st>>>(xb, ldx, shift, scale, mod_stride, yb, ldy, S, D,
+        launch_pdl(dit::modulate_norm_row_kernel<4>, grid, threads, 0, st, xb, ldx, shift, scale, mod_stride, yb, ldy, S, D,
                                                                     eps);
       return launch_status();
     }
@@ -585,7 +624,7 @@ dit_status attention_launch(const dit_bf16* q, const dit_bf16* k, const dit_bf16
   p.lse_split_stride = lse_split_stride;
   if ((int64_t)B * splits > 65535) return DIT_ERR_SHAPE;
   dim3 grid((unsigned)((Sq + 2 * dit::attn::BQ - 1) / (2 * dit::attn::BQ)), (unsigned)H, (unsigned)(B * splits));
-  dit::attn::attention_kernel<<<grid, dit::attn::NUM_THREADS, dit::attn::SMEM_BYTES, (cudaStream_t)stream>>>(
+  launch_pdl(dit::attn::attention_kernel, grid, dit::attn::NUM_THREADS, dit::attn::SMEM_BYTES, (cudaStream_t)stream, 
       tq, tk, tv, p, g_wait_limit_ns);
   return launch_status();
 }
@@ -619,11 +658,11 @@ dit_status merge_launch(int n, const dit_bf16* const* o_parts, const float* cons
   if (s != DIT_OK) return s;
   const dim3 grid((unsigned)((S + 15) / 16), (unsigned)H, (unsigned)B);
   if (n <= 2)
-    dit::attention_merge_kernel<2><<<grid, 256, 0, (cudaStream_t)stream>>>(p);
+    launch_pdl(dit::attention_merge_kernel<2>, grid, 256, 0, (cudaStream_t)stream, p);
   else if (n <= 4)
-    dit::attention_merge_kernel<4><<<grid, 256, 0, (cudaStream_t)stream>>>(p);
+    launch_pdl(dit::attention_merge_kernel<4>, grid, 256, 0, (cudaStream_t)stream, p);
   else
-    dit::attention_merge_kernel<8><<<grid, 256, 0, (cudaStream_t)stream>>>(p);
+    launch_pdl(dit::attention_merge_kernel<8>, grid, 256, 0, (cudaStream_t)stream, p);
   return launch_status();
 }
 
@@ -806,19 +845,19 @@ dit_status dit_gemm_epilogue(const dit_gemm_args* a, void* stream) {
     }
     switch (a->epi) {
       case DIT_EPI_NONE:
-        P::gemm_pair_kernel<DIT_EPI_NONE><<<grid, P::NUM_THREADS, P::SMEM_BYTES, st>>>(tA, tB, a->M, a->N, a->K, ep,
+        launch_pdl(P::gemm_pair_kernel<DIT_EPI_NONE>, grid, P::NUM_THREADS, P::SMEM_BYTES, st, tA, tB, a->M, a->N, a->K, ep,
                                                                                      g_wait_limit_ns, nf);
         break;
       case DIT_EPI_BIAS:
-        P::gemm_pair_kernel<DIT_EPI_BIAS><<<grid, P::NUM_THREADS, P::SMEM_BYTES, st>>>(tA, tB, a->M, a->N, a->K, ep,
+        launch_pdl(P::gemm_pair_kernel<DIT_EPI_BIAS>, grid, P::NUM_THREADS, P::SMEM_BYTES, st, tA, tB, a->M, a->N, a->K, ep,
                                                                                      g_wait_limit_ns, nf);
         break;
       case DIT_EPI_BIAS_GELU_COLS:
-        P::gemm_pair_kernel<DIT_EPI_BIAS_GELU_COLS><<<grid, P::NUM_THREADS, P::SMEM_BYTES, st>>>(
+        launch_pdl(P::gemm_pair_kernel<DIT_EPI_BIAS_GELU_COLS>, grid, P::NUM_THREADS, P::SMEM_BYTES, st, 
             tA, tB, a->M, a->N, a->K, ep, g_wait_limit_ns, nf);
         break;
       default:
-        P::gemm_pair_kernel<DIT_EPI_BIAS_GATED_RESIDUAL><<<grid, P::NUM_THREADS, P::SMEM_BYTES, st>>>(
+        launch_pdl(P::gemm_pair_kernel<DIT_EPI_BIAS_GATED_RESIDUAL>, grid, P::NUM_THREADS, P::SMEM_BYTES, st, 
             tA, tB, a->M, a->N, a->K, ep, g_wait_limit_ns, nf);
         break;
     }

@@ -120,6 +120,8 @@ __global__ void __launch_bounds__(256) modulate_norm_row_kernel(const bf16* __re
                                                                 int64_t mod_stride, bf16* __restrict__ y,
                                                                 int64_t ldy, int S, int D, float eps) {
   constexpr int E = 8 * NC;
+  griddep_wait();
+  griddep_launch_dependents();
   __shared__ float2 red[8];
   const int T = blockDim.x;
   const int w = threadIdx.x >> 5, l = threadIdx.x & 31, nw = T >> 5;
@@ -257,6 +259,8 @@ template <int KC, int NB, typename RowFn, typename OutFn>
 __device__ __forceinline__ void vec_rows_loop(const bf16* __restrict__ x, int64_t ldx, int K, int flags, int64_t N,
                                               RowFn row_of, OutFn store) {
   constexpr bool TWO = KC * NB <= 6;  // two rows in flight per warp while the registers allow it
+  griddep_wait();
+  griddep_launch_dependents();
   extern __shared__ float4 xs4[];  // NB mapped inputs, K fp32 each, lane-interleaved
   float* xs = reinterpret_cast<float*>(xs4);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -640,6 +644,8 @@ struct MergeParams {
 
 template <int NP>  // bound on the number of parts (2, 4 or 8): every load is issued before any is used
 __global__ void __launch_bounds__(256) attention_merge_kernel(const __grid_constant__ MergeParams p) {
+  griddep_wait();
+  griddep_launch_dependents();
   // grid (tokens / 16, H, B): 16 consecutive tokens of one (batch, head) per
   // CTA, so the lse accesses are contiguous and no index needs a division
   const int s = blockIdx.x * 16 + (threadIdx.x >> 4);

@@ -465,6 +465,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
   cluster_sync_all();  // barrier inits and TMEM allocation visible to both CTAs
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  griddep_wait();  // the prologue above overlaps the previous kernel; everything below follows it
+  griddep_launch_dependents();
 
   const int num_m = (M + BM - 1) / BM;
   const int num_n = (N + BN - 1) / BN;

@@ -29,6 +29,12 @@
  *     synchronise, so they can be captured into a CUDA graph.  Exceptions are
  *     named: dit_get_device_error synchronises, dit_forward_graph_create
  *     captures on a private stream.
+ *   - The block-path kernels (LN-modulate, adaLN, the GEMMs, attention, the
+ *     merge) are launched with programmatic stream serialization: a kernel may
+ *     begin its prologue (barrier setup, TMEM allocation) while the previous
+ *     kernel of the stream drains, and it touches no global memory before
+ *     that kernel has completed, so stream order holds for every buffer.
+ *     DIT_DISABLE_PDL=1 in the environment launches them the plain way.
  *   - No call aborts or traps.  Argument errors return a status before any work
  *     is enqueued.  A kernel that waits longer than the wait limit (default 2 s)
  *     on an internal barrier records DIT_ERR_TIMEOUT in the device error word,
@@ -378,7 +384,9 @@ dit_status dit_single_block_fwd(const dit_block_cfg* cfg, const dit_single_weigh
 /* Same call that additionally records events[i] (cudaEvent_t, may not be NULL)
  * on the stream before kernel i and events[5] after the last of its five
  * kernels (adaLN, LN-modulate, GEMM1 with fused QK-norm+RoPE, attention,
- * GEMM2), so a caller can time every kernel.  n_events must be >= 6. */
+ * GEMM2), so a caller can time every kernel.  n_events must be >= 6.  Its
+ * kernels start only when the previous one has finished (the plain call lets
+ * each kernel's prologue overlap the end of the one before). */
 dit_status dit_single_block_fwd_profiled(const dit_block_cfg* cfg, const dit_single_weights* w,
                                          const dit_bf16* x, const dit_bf16* vec, const float* rope,
                                          dit_bf16* out, void* ws, size_t ws_bytes,
