@@ -338,8 +338,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const uint64_t negx2 = f2_pack(-m_new, -m_new);
       uint64_t sum2[2] = {0ull, 0ull};  // packed (even, odd) partial sums, two chains
       uint32_t pk[4][16];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      auto exps = [&](int c) {
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           // x = s * scale * log2(e) - m for the pair (2i, 2i+1): one packed FMA
@@ -353,17 +352,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           sum2[i & 1] = f2_add(sum2[i & 1], pp);
           pk[c][i] = pack_bf16x2(f2_lo(pp), f2_hi(pp));
         }
-      }
-      const uint64_t st2 = f2_add(sum2[0], sum2[1]);
-      l_run = l_run * alpha + (f2_lo(st2) + f2_hi(st2));
-      // P_t and O_t are free once the previous PV of this tile is done
+      };
+      // P of keys 0..63 goes to TMEM while the exponentials of keys 64..127
+      // run; P_t and O_t are free once the previous PV of this tile is done
+      exps(0);
+      exps(1);
       if (j > 0) {
         ok = mbar_wait(&p_free[t], (j - 1) & 1, wait_limit, abort_flag, SITE_ATTN_SOFTMAX);
         if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
         tc_fence_after();
       }
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_st16(tP + (uint32_t)(c * 16), pk[c]);
+      tmem_st16(tP + 0u, pk[0]);
+      tmem_st16(tP + 16u, pk[1]);
+      exps(2);
+      exps(3);
+      const uint64_t st2 = f2_add(sum2[0], sum2[1]);
+      l_run = l_run * alpha + (f2_lo(st2) + f2_hi(st2));
+      tmem_st16(tP + 32u, pk[2]);
+      tmem_st16(tP + 48u, pk[3]);
       // Rescale O_t when any row of this warp raised its max
       if (j > 0 && __any_sync(0xffffffffu, need)) {
 #pragma unroll 1
