@@ -135,6 +135,7 @@ _SIGS = {
                                   i32, i32, i32, f32, i32, i32, c_void_p, size_t, c_void_p]),
     "dit_attention_split_workspace": (size_t, [i32, i32, i32, i32]),
     "dit_gemm_epilogue": (i32, [ctypes.POINTER(dit_gemm_args), c_void_p]),
+    "dit_gemm_epilogue_grouped": (i32, [ctypes.POINTER(dit_gemm_args), ctypes.POINTER(dit_gemm_args), c_void_p]),
     "dit_selftest_exp2_poly": (i32, [c_void_p, c_void_p, i64, c_void_p]),
     "dit_attention_merge": (i32, [i32, ctypes.POINTER(c_void_p), ctypes.POINTER(c_void_p), i64, c_void_p, c_void_p,
                                   i64, i32, i32, i32, c_void_p]),
@@ -351,21 +352,34 @@ def dit_attention_merge(o_parts, lse_parts, o, lse_out, B, Sq, H, stream=None):
     _call("dit_attention_merge", n, op, lp, ld, _ptr(o), _ptr(lse_out), o.stride(0), B, Sq, H, _stream(stream))
 
 
-def dit_gemm_epilogue(A, W, C, epi=DIT_EPI_NONE, bias=None, C2=None, split_col=0, gelu_col_begin=0,
-                      gate=None, gate_stride=0, resid=None, rows_per_batch=0, K=None, qk_cols=0, qk_norm=1,
-                      qk_eps=1e-6, q_scale=None, k_scale=None, rope=None, rope_rows=0, stream=None):
-    """C[:, :split] (and C2 for the rest) = epilogue(A W^T).  A [M, >=K], W [N, >=K]."""
+def gemm_args(A, W, C, epi=DIT_EPI_NONE, bias=None, C2=None, split_col=0, gelu_col_begin=0,
+              gate=None, gate_stride=0, resid=None, rows_per_batch=0, K=None, qk_cols=0, qk_norm=1,
+              qk_eps=1e-6, q_scale=None, k_scale=None, rope=None, rope_rows=0) -> dit_gemm_args:
+    """The dit_gemm_args of C[:, :split] (and C2 for the rest) = epilogue(A W^T)."""
     M = A.shape[0]
     N = W.shape[0]
     K = A.shape[1] if K is None else K
-    a = dit_gemm_args(
+    return dit_gemm_args(
         A=_ptr(A), lda=A.stride(0), W=_ptr(W), ldw=W.stride(0), bias=_ptr(bias), C=_ptr(C), ldc=C.stride(0),
         C2=_ptr(C2), ldc2=C2.stride(0) if C2 is not None else 0, split_col=split_col, M=M, N=N, K=K, epi=epi,
         gelu_col_begin=gelu_col_begin, gate=_ptr(gate), gate_stride=gate_stride, resid=_ptr(resid),
         ldr=resid.stride(0) if resid is not None else 0, rows_per_batch=rows_per_batch or M,
         qk_cols=qk_cols, qk_norm=qk_norm, qk_eps=qk_eps, q_scale=_ptr(q_scale), k_scale=_ptr(k_scale),
         rope=_ptr(rope), rope_rows=rope_rows or M)
+
+
+def dit_gemm_epilogue(A, W, C, epi=DIT_EPI_NONE, bias=None, C2=None, split_col=0, gelu_col_begin=0,
+                      gate=None, gate_stride=0, resid=None, rows_per_batch=0, K=None, qk_cols=0, qk_norm=1,
+                      qk_eps=1e-6, q_scale=None, k_scale=None, rope=None, rope_rows=0, stream=None):
+    """C[:, :split] (and C2 for the rest) = epilogue(A W^T).  A [M, >=K], W [N, >=K]."""
+    a = gemm_args(A, W, C, epi, bias, C2, split_col, gelu_col_begin, gate, gate_stride, resid, rows_per_batch, K,
+                  qk_cols, qk_norm, qk_eps, q_scale, k_scale, rope, rope_rows)
     _call("dit_gemm_epilogue", ctypes.byref(a), _stream(stream))
+
+
+def dit_gemm_epilogue_grouped(a: dit_gemm_args, b: dit_gemm_args, stream=None):
+    """Two GEMMs (gemm_args) with the same epilogue kind and K in one launch."""
+    _call("dit_gemm_epilogue_grouped", ctypes.byref(a), ctypes.byref(b), _stream(stream))
 
 
 def block_cfg(B, S, D, H, M, n_txt=0, eps=1e-6) -> dit_block_cfg:

@@ -755,7 +755,11 @@ dit_status dit_attention_merge(int n, const dit_bf16* const* o_parts, const floa
   return merge_launch(n, o_parts, lse_parts, lds, o, lse_out, ld_out, B, S, H, stream);
 }
 
-dit_status dit_gemm_epilogue(const dit_gemm_args* a, void* stream) {
+}  // extern "C"
+
+namespace {
+
+dit_status gemm_validate(const dit_gemm_args* a) {
   if (a == nullptr || a->A == nullptr || a->W == nullptr || a->C == nullptr) return DIT_ERR_INVALID_ARG;
   if (a->M < 1 || a->N < 32 || a->K < 8 || (a->N % 32) != 0 || (a->K % 8) != 0) return DIT_ERR_SHAPE;
   if (a->lda < a->K || a->ldw < a->K || (a->lda % 8) || (a->ldw % 8)) return DIT_ERR_SHAPE;
@@ -792,22 +796,15 @@ dit_status dit_gemm_epilogue(const dit_gemm_args* a, void* stream) {
     default:
       return DIT_ERR_INVALID_ARG;
   }
-  int sms = 0;
-  dit_status s = device_setup(&sms);
-  if (s != DIT_OK) return s;
-  // SM-pair kernel (256 x 256 tiles over two CTAs) once there are at least
-  // two 128-row blocks; the one-CTA kernel (128 x 256 tiles) otherwise.
-  const bool use_pair = a->M > dit::gemm::BM && sms >= 2;
-  CUtensorMap tA, tB;
-  if ((s = make_map_2d(&tA, a->A, a->M, a->K, a->lda, dit::gemm::BM)) != DIT_OK) return s;
-  if ((s = make_map_2d(&tB, a->W, a->N, a->K, a->ldw, use_pair ? dit::gemm::pair::BN_CTA : dit::gemm::BN)) != DIT_OK)
-    return s;
-  dit::gemm::Epi ep;
+  return DIT_OK;
+}
+
+void gemm_epi(const dit_gemm_args* a, dit::gemm::Epi& ep) {
   ep.C = reinterpret_cast<bf16*>(a->C);
   ep.ldc = a->ldc;
   ep.C2 = reinterpret_cast<bf16*>(a->C2);
   ep.ldc2 = a->ldc2;
-  ep.split_col = split;
+  ep.split_col = a->C2 ? a->split_col : a->N;
   ep.bias = reinterpret_cast<const bf16*>(a->bias);
   ep.gelu_col_begin = a->gelu_col_begin;
   ep.gate = a->gate;
@@ -824,45 +821,83 @@ dit_status dit_gemm_epilogue(const dit_gemm_args* a, void* stream) {
   ep.rope_rows = a->rope_rows > 0 ? a->rope_rows : a->M;
   ep.w_keep = nullptr;
   ep.w_keep_bytes = 0;
-  cudaStream_t st = (cudaStream_t)stream;
-  if (use_pair) {
-    namespace P = dit::gemm::pair;
-    const int tiles = ((a->M + P::BM - 1) / P::BM) * ((a->N + P::BN - 1) / P::BN);
-    const int clusters = tiles < sms / 2 ? tiles : sms / 2;
-    const int grid = 2 * clusters;
-    // walk the larger operand's panels once: N-fastest when A (M x K) is the larger
-    const int nf = a->M > a->N ? 1 : 0;
-    int dev = 0;
-    if (nf && cudaGetDevice(&dev) == cudaSuccess && g_dev[dev].keep_weights.load(std::memory_order_relaxed)) {
-      // whole 128-byte lines inside the weight: the kernel returns them to normal L2 priority at the end
-      const uintptr_t w0 = reinterpret_cast<uintptr_t>(a->W);
-      const uintptr_t lo = (w0 + 127) & ~(uintptr_t)127;
-      const uintptr_t hi = (w0 + (uintptr_t)a->N * (uintptr_t)a->ldw * 2) & ~(uintptr_t)127;
-      if (hi > lo) {
-        ep.w_keep = reinterpret_cast<const uint8_t*>(lo);
-        ep.w_keep_bytes = (int64_t)(hi - lo);
-      }
+}
+
+// One job of the SM-pair kernel: tensor maps, epilogue and tile order.
+dit_status pair_job(const dit_gemm_args* a, dit::gemm::pair::PairJob& j) {
+  namespace P = dit::gemm::pair;
+  dit_status s;
+  if ((s = make_map_2d(&j.tmA, a->A, a->M, a->K, a->lda, dit::gemm::BM)) != DIT_OK) return s;
+  if ((s = make_map_2d(&j.tmB, a->W, a->N, a->K, a->ldw, P::BN_CTA)) != DIT_OK) return s;
+  gemm_epi(a, j.ep);
+  j.M = a->M;
+  j.N = a->N;
+  // walk the larger operand's panels once: N-fastest when A (M x K) is the larger
+  j.n_fastest = a->M > a->N ? 1 : 0;
+  int dev = 0;
+  if (j.n_fastest && cudaGetDevice(&dev) == cudaSuccess && g_dev[dev].keep_weights.load(std::memory_order_relaxed)) {
+    // whole 128-byte lines inside the weight: the kernel returns them to normal L2 priority at the end
+    const uintptr_t w0 = reinterpret_cast<uintptr_t>(a->W);
+    const uintptr_t lo = (w0 + 127) & ~(uintptr_t)127;
+    const uintptr_t hi = (w0 + (uintptr_t)a->N * (uintptr_t)a->ldw * 2) & ~(uintptr_t)127;
+    if (hi > lo) {
+      j.ep.w_keep = reinterpret_cast<const uint8_t*>(lo);
+      j.ep.w_keep_bytes = (int64_t)(hi - lo);
     }
-    switch (a->epi) {
-      case DIT_EPI_NONE:
-        launch_pdl(P::gemm_pair_kernel<DIT_EPI_NONE>, grid, P::NUM_THREADS, P::SMEM_BYTES, st, tA, tB, a->M, a->N, a->K, ep,
-                                                                                     g_wait_limit_ns, nf);
-        break;
-      case DIT_EPI_BIAS:
-        launch_pdl(P::gemm_pair_kernel<DIT_EPI_BIAS>, grid, P::NUM_THREADS, P::SMEM_BYTES, st, tA, tB, a->M, a->N, a->K, ep,
-                                                                                     g_wait_limit_ns, nf);
-        break;
-      case DIT_EPI_BIAS_GELU_COLS:
-        launch_pdl(P::gemm_pair_kernel<DIT_EPI_BIAS_GELU_COLS>, grid, P::NUM_THREADS, P::SMEM_BYTES, st, 
-            tA, tB, a->M, a->N, a->K, ep, g_wait_limit_ns, nf);
-        break;
-      default:
-        launch_pdl(P::gemm_pair_kernel<DIT_EPI_BIAS_GATED_RESIDUAL>, grid, P::NUM_THREADS, P::SMEM_BYTES, st, 
-            tA, tB, a->M, a->N, a->K, ep, g_wait_limit_ns, nf);
-        break;
-    }
-    return launch_status();
   }
+  return DIT_OK;
+}
+
+dit_status pair_launch(const dit::gemm::pair::PairGroup& G, int epi, int K, int sms, cudaStream_t st) {
+  namespace P = dit::gemm::pair;
+  int tiles = 0;
+  for (int g = 0; g < G.count; ++g)
+    tiles += ((G.job[g].M + P::BM - 1) / P::BM) * ((G.job[g].N + P::BN - 1) / P::BN);
+  const int clusters = tiles < sms / 2 ? tiles : sms / 2;
+  const int grid = 2 * clusters;
+  switch (epi) {
+    case DIT_EPI_NONE:
+      launch_pdl(P::gemm_pair_kernel<DIT_EPI_NONE>, grid, P::NUM_THREADS, P::SMEM_BYTES, st, G, K, g_wait_limit_ns);
+      break;
+    case DIT_EPI_BIAS:
+      launch_pdl(P::gemm_pair_kernel<DIT_EPI_BIAS>, grid, P::NUM_THREADS, P::SMEM_BYTES, st, G, K, g_wait_limit_ns);
+      break;
+    case DIT_EPI_BIAS_GELU_COLS:
+      launch_pdl(P::gemm_pair_kernel<DIT_EPI_BIAS_GELU_COLS>, grid, P::NUM_THREADS, P::SMEM_BYTES, st, G, K,
+                 g_wait_limit_ns);
+      break;
+    default:
+      launch_pdl(P::gemm_pair_kernel<DIT_EPI_BIAS_GATED_RESIDUAL>, grid, P::NUM_THREADS, P::SMEM_BYTES, st, G, K,
+                 g_wait_limit_ns);
+      break;
+  }
+  return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+dit_status dit_gemm_epilogue(const dit_gemm_args* a, void* stream) {
+  dit_status s = gemm_validate(a);
+  if (s != DIT_OK) return s;
+  int sms = 0;
+  if ((s = device_setup(&sms)) != DIT_OK) return s;
+  cudaStream_t st = (cudaStream_t)stream;
+  // SM-pair kernel (256 x 256 tiles over two CTAs) once there are at least
+  // two 128-row blocks; the one-CTA kernel (128 x 256 tiles) otherwise.
+  if (a->M > dit::gemm::BM && sms >= 2) {
+    dit::gemm::pair::PairGroup G;
+    G.count = 1;
+    if ((s = pair_job(a, G.job[0])) != DIT_OK) return s;
+    G.job[1] = G.job[0];
+    return pair_launch(G, a->epi, a->K, sms, st);
+  }
+  CUtensorMap tA, tB;
+  if ((s = make_map_2d(&tA, a->A, a->M, a->K, a->lda, dit::gemm::BM)) != DIT_OK) return s;
+  if ((s = make_map_2d(&tB, a->W, a->N, a->K, a->ldw, dit::gemm::BN)) != DIT_OK) return s;
+  dit::gemm::Epi ep;
+  gemm_epi(a, ep);
   const int tiles = ((a->M + dit::gemm::BM - 1) / dit::gemm::BM) * ((a->N + dit::gemm::BN - 1) / dit::gemm::BN);
   const int grid = tiles < sms ? tiles : sms;
   const int smem = dit::gemm::SMEM_BYTES;
@@ -884,6 +919,25 @@ dit_status dit_gemm_epilogue(const dit_gemm_args* a, void* stream) {
       break;
   }
   return launch_status();
+}
+
+dit_status dit_gemm_epilogue_grouped(const dit_gemm_args* a, const dit_gemm_args* b, void* stream) {
+  dit_status s;
+  if ((s = gemm_validate(a)) != DIT_OK) return s;
+  if ((s = gemm_validate(b)) != DIT_OK) return s;
+  if (a->epi != b->epi || a->K != b->K) return DIT_ERR_INVALID_ARG;
+  int sms = 0;
+  if ((s = device_setup(&sms)) != DIT_OK) return s;
+  if (a->M <= dit::gemm::BM || b->M <= dit::gemm::BM || sms < 2) {
+    // a job this small runs on the one-CTA kernel: two launches
+    if ((s = dit_gemm_epilogue(a, stream)) != DIT_OK) return s;
+    return dit_gemm_epilogue(b, stream);
+  }
+  dit::gemm::pair::PairGroup G;
+  G.count = 2;
+  if ((s = pair_job(a, G.job[0])) != DIT_OK) return s;
+  if ((s = pair_job(b, G.job[1])) != DIT_OK) return s;
+  return pair_launch(G, a->epi, a->K, sms, (cudaStream_t)stream);
 }
 
 }  // extern "C"

@@ -422,10 +422,33 @@ constexpr uint32_t TMEM_COLS = 512;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 256 + 1024;
 constexpr uint32_t IDESC = idesc_bf16(BM, BN, 0, 0);
 
+// One GEMM of a launch: its operands' tensor maps, epilogue, shape and tile
+// order.  A launch runs one job or a group of two with the same K and
+// epilogue kind (the double-stream block's text and image projections): the
+// tiles of job 1 follow those of job 0 in one persistent schedule, so a job
+// with few tiles fills the SMs the other leaves idle.
+struct PairJob {
+  CUtensorMap tmA, tmB;
+  Epi ep;
+  int M, N;
+  int n_fastest;
+};
+struct PairGroup {
+  PairJob job[2];
+  int count;  // 1 or 2
+};
+
+// tile index of the launch -> job and tile coordinates
+__device__ __forceinline__ int group_tile(const PairGroup& G, int tiles0, int tile, int& tm, int& tn) {
+  const int g = (G.count > 1 && tile >= tiles0) ? 1 : 0;
+  const PairJob& J = G.job[g];
+  tile_coords(g ? tile - tiles0 : tile, (J.M + BM - 1) / BM, (J.N + BN - 1) / BN, J.n_fastest, tm, tn);
+  return g;
+}
+
 template <int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
-    gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M, int N,
-                     int K, Epi ep, uint64_t wait_limit, int n_fastest) {
+    gemm_pair_kernel(const __grid_constant__ PairGroup G, int K, uint64_t wait_limit) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
@@ -454,8 +477,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
-    tma_prefetch_desc(&tmA);
-    tma_prefetch_desc(&tmB);
+    for (int g = 0; g < G.count; ++g) {
+      tma_prefetch_desc(&G.job[g].tmA);
+      tma_prefetch_desc(&G.job[g].tmB);
+    }
   }
   if (warp == 1) {
     tmem_alloc_pair(tmem_slot, TMEM_COLS);
@@ -468,9 +493,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
   griddep_wait();  // the prologue above overlaps the previous kernel; everything below follows it
   griddep_launch_dependents();
 
-  const int num_m = (M + BM - 1) / BM;
-  const int num_n = (N + BN - 1) / BN;
-  const int num_tiles = num_m * num_n;
+  const int tiles0 = ((G.job[0].M + BM - 1) / BM) * ((G.job[0].N + BN - 1) / BN);
+  const int num_tiles =
+      tiles0 + (G.count > 1 ? ((G.job[1].M + BM - 1) / BM) * ((G.job[1].N + BN - 1) / BN) : 0);
   const int num_kb = (K + BK - 1) / BK;
   const int cluster_id = blockIdx.x >> 1;
   const int n_clusters = gridDim.x >> 1;
@@ -483,14 +508,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       uint32_t issued_mask = 0, issued_parity = 0;
       bool ok = true;
       int wave = 0;  // this cluster's tile count so far: the same for every cluster of a wave
-      const bool keep_b = n_fastest && ep.w_keep != nullptr;
       const uint64_t b_policy = l2_policy_evict_last();
       for (int tile = cluster_id; tile < num_tiles && ok; tile += n_clusters, ++wave) {
         int tm, tn;
-        tile_coords(tile, num_m, num_n, n_fastest, tm, tn);
+        const PairJob& J = G.job[group_tile(G, tiles0, tile, tm, tn)];
+        const bool keep_b = J.n_fastest && J.ep.w_keep != nullptr;
         // N-fastest: every other wave walks K backwards, so that it starts on the
         // K range whose weight panels the previous wave touched last (still in L2)
-        const bool back = n_fastest && (wave & 1);
+        const bool back = J.n_fastest && (wave & 1);
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1, wait_limit, abort_flag, SITE_GEMM2_PRODUCER)) {
             ok = false;
@@ -499,12 +524,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
           if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * STAGE_BYTES);
           const uint32_t leader_full = mapa_shared(smem_u32(&full[stage]), 0);
           const int kx = (back ? num_kb - 1 - kb : kb) * BK;
-          tma_load_2d_pair(sA + stage * A_BYTES, &tmA, leader_full, kx, tm * BM + (int)rank * BM_CTA);
+          tma_load_2d_pair(sA + stage * A_BYTES, &J.tmA, leader_full, kx, tm * BM + (int)rank * BM_CTA);
           if (keep_b)
-            tma_load_2d_pair_hint(sB + stage * B_BYTES, &tmB, leader_full, kx, tn * BN + (int)rank * BN_CTA,
+            tma_load_2d_pair_hint(sB + stage * B_BYTES, &J.tmB, leader_full, kx, tn * BN + (int)rank * BN_CTA,
                                   b_policy);
           else
-            tma_load_2d_pair(sB + stage * B_BYTES, &tmB, leader_full, kx, tn * BN + (int)rank * BN_CTA);
+            tma_load_2d_pair(sB + stage * B_BYTES, &J.tmB, leader_full, kx, tn * BN + (int)rank * BN_CTA);
           issued_mask |= 1u << stage;
           issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) {
@@ -579,7 +604,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     uint32_t acc_phase = 0;
     for (int tile = cluster_id; tile < num_tiles; tile += n_clusters) {
       int tm, tn;
-      tile_coords(tile, num_m, num_n, n_fastest, tm, tn);
+      const PairJob& J = G.job[group_tile(G, tiles0, tile, tm, tn)];
+      const Epi& ep = J.ep;
+      const int M = J.M, N = J.N;
       bool ok = mbar_wait(&tfull[acc], acc_phase, wait_limit, abort_flag, SITE_GEMM2_EPILOGUE);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
@@ -612,11 +639,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
   cluster_sync_all();  // no CTA leaves while its peer may still touch its memory
   tc_fence_after();
   if (warp == 1) tmem_dealloc_pair(tmem_base, TMEM_COLS);
-  if (n_fastest && ep.w_keep != nullptr) {
-    // this CTA's share of the kept weight back to normal L2 priority
-    const int64_t lines = ep.w_keep_bytes >> 7;
-    for (int64_t i = (int64_t)blockIdx.x * NUM_THREADS + threadIdx.x; i < lines; i += (int64_t)gridDim.x * NUM_THREADS)
-      l2_priority_normal(ep.w_keep + (i << 7));
+  for (int g = 0; g < G.count; ++g) {
+    const PairJob& J = G.job[g];
+    if (J.n_fastest && J.ep.w_keep != nullptr) {
+      // this CTA's share of the kept weight back to normal L2 priority
+      const int64_t lines = J.ep.w_keep_bytes >> 7;
+      for (int64_t i = (int64_t)blockIdx.x * NUM_THREADS + threadIdx.x; i < lines;
+           i += (int64_t)gridDim.x * NUM_THREADS)
+        l2_priority_normal(J.ep.w_keep + (i << 7));
+    }
   }
 }
 

@@ -313,9 +313,21 @@ typedef struct {
   int rope_rows;                    /* output row m uses rope row m % rope_rows */
 } dit_gemm_args;
 
-/* bf16 x bf16 -> fp32 accumulate on tcgen05 (128 x 256 tiles, TMA-fed, TMEM
- * accumulators, persistent CTAs); epilogue rounds to bf16 (nearest-even). */
+/* bf16 x bf16 -> fp32 accumulate on tcgen05 (256 x 256 tiles over SM pairs
+ * when M > 128, else 128 x 256 on one SM; TMA-fed, TMEM accumulators,
+ * persistent CTAs); epilogue rounds to bf16 (nearest-even). */
 dit_status dit_gemm_epilogue(const dit_gemm_args* args, void* stream);
+
+/* Two independent GEMMs with the same epilogue kind and the same K in one
+ * persistent launch ([CG] §3.1: the double-stream block runs the same layer
+ * on the text and the image stream with separate weights).  The tiles of b
+ * follow those of a in one schedule, so a GEMM with few tiles (512 text rows)
+ * fills the SMs the other leaves idle.  Each result is the one
+ * dit_gemm_epilogue gives for its arguments, bit for bit.  a and b are
+ * validated as for dit_gemm_epilogue; a->epi != b->epi or a->K != b->K is
+ * DIT_ERR_INVALID_ARG.  With M <= 128 in either, the two run as two launches.
+ * The outputs must not overlap each other or the other GEMM's inputs. */
+dit_status dit_gemm_epilogue_grouped(const dit_gemm_args* a, const dit_gemm_args* b, void* stream);
 
 /* ------------------------------------------------------------------------
  * Blocks ([CG] §2 single-stream block; §3.1 double-stream blocks; [WAN] §1.1)

@@ -226,6 +226,60 @@ def test_gemm_gated_residual(M, rows_per_batch, N, K, inplace):
     parity(host_f64(out_s), xsf + g * y, "gated residual, small residual")
 
 
+@pytest.mark.parametrize("epi,M1,M2,N,K", [
+    ("gated", 512, 4096, 768, 1536),   # text + image output projections (M1 < N: M-fastest; M2 > N: N-fastest)
+    ("gelu", 512, 1000, 1024, 512),    # MLP-in with GELU, ragged image rows
+    ("qk", 300, 700, 768, 256),        # QKV with the fused per-head RMSNorm + RoPE
+    ("gated", 100, 600, 256, 512),     # M1 <= 128: two launches
+])
+def test_gemm_grouped_equals_two_calls(epi, M1, M2, N, K):
+    """Two GEMMs in one grouped launch (the double-stream block's text and
+    image layers) give exactly what two dit_gemm_epilogue calls give, and the
+    oracle's result within the stated tolerance."""
+    import torch
+    D = 768
+    jobs = []
+    for j, M in enumerate((M1, M2)):
+        A, W, b = _gemm_inputs(M, N, K, seed=31 + 7 * j)
+        t = {"A": dev_bf16(A), "W": dev_bf16(W), "b": dev_bf16(b), "Af": A, "Wf": W, "bf": b, "M": M}
+        kw = dict(bias=t["b"])
+        if epi == "gated":
+            x = synth.normal_bf16(40 + j, "x", (M, N))
+            g = synth.bf16_bits_to_f64(synth.normal_bf16(50 + j, "g", (1, N), 0.7))
+            t["x"], t["g"] = x, g
+            t["resid"] = dev_bf16(x)
+            kw.update(epi=dit.DIT_EPI_BIAS_GATED_RESIDUAL, gate=f32dev(g), gate_stride=0, resid=t["resid"])
+        elif epi == "gelu":
+            kw.update(epi=dit.DIT_EPI_BIAS_GELU_COLS, gelu_col_begin=256)
+        else:
+            ids = torch.from_numpy(synth.flux_ids(16, 16, (M - 16 + 15) // 16)[:M]).cuda()
+            rope = torch.empty((M, 64, 2), dtype=torch.float32, device="cuda")
+            dit.dit_rope_table(ids, (8, 28, 28), 10000.0, rope)
+            t["rope"] = rope
+            kw.update(epi=dit.DIT_EPI_BIAS, qk_cols=2 * (N // 3 // 128) * 128, rope=rope, rope_rows=M)
+        t["kw"] = kw
+        jobs.append(t)
+    sep = [torch.empty((t["M"], N), dtype=torch.bfloat16, device="cuda") for t in jobs]
+    grp = [torch.empty_like(o) for o in sep]
+    for t, o in zip(jobs, sep):
+        dit.dit_gemm_epilogue(t["A"], t["W"], o, **t["kw"])
+    args = [dit.gemm_args(t["A"], t["W"], o, **t["kw"]) for t, o in zip(jobs, grp)]
+    dit.dit_gemm_epilogue_grouped(args[0], args[1])
+    torch.cuda.synchronize()
+    for o_s, o_g in zip(sep, grp):
+        assert torch.equal(o_s, o_g)
+    if epi != "qk":
+        for t, o in zip(jobs, grp):
+            y = O.linear(synth.bf16_bits_to_f64(t["Af"]), synth.bf16_bits_to_f64(t["Wf"]),
+                         synth.bf16_bits_to_f64(t["bf"]))
+            if epi == "gated":
+                ref = synth.bf16_bits_to_f64(t["x"]) + t["g"] * y
+            else:
+                ref = np.concatenate([y[:, :256], O.gelu_tanh(y[:, 256:])], axis=1)
+            parity(host_f64(o), ref, f"grouped {epi}, M={t['M']}")
+    assert_no_device_error()
+
+
 def test_weight_l2_persist_changes_no_bits():
     """With the opt-in L2 residency of the output GEMM's weight, the N-fastest
     GEMM (M > N) loads its weight with the evict-last policy and demotes it at
