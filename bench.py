@@ -415,11 +415,11 @@ def run_ours(args, rank, world, local_rank):
 # (profiles/*.ncu.md), with a hash of the kernel's sources at capture time.
 # A kernel whose sources changed since reports traffic null.
 NCU_TRAFFIC = {
-    "gemm_qkv_mlp_gelu_qknorm_rope": (336957952, ("gemm.cuh", "common.cuh"), "58798835864e2a01"),
-    "gemm_out_gated_residual": (436787968, ("gemm.cuh", "common.cuh"), "58798835864e2a01"),
-    "attention": (92532224, ("attention.cuh", "common.cuh"), "a9751413b4e054e3"),
-    "modulate_norm": (28440064, ("elementwise.cuh", "common.cuh"), "046c38d671b7c963"),
-    "adaln_modulation": (56678400, ("elementwise.cuh", "common.cuh"), "046c38d671b7c963"),
+    "gemm_qkv_mlp_gelu_qknorm_rope": (336224000, ("gemm.cuh", "common.cuh"), "2f431c60dd9c3864"),
+    "gemm_out_gated_residual": (437787904, ("gemm.cuh", "common.cuh"), "2f431c60dd9c3864"),
+    "attention": (95213568, ("attention.cuh", "common.cuh"), "8aa1fbcb8a30f541"),
+    "modulate_norm": (28440064, ("elementwise.cuh", "common.cuh"), "7edddd6c2e584c82"),
+    "adaln_modulation": (56678400, ("elementwise.cuh", "common.cuh"), "7edddd6c2e584c82"),
 }
 
 
