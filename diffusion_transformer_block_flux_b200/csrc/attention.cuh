@@ -344,7 +344,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           // x = s * scale * log2(e) - m for the pair (2i, 2i+1): one packed FMA
           const uint64_t x = f2_fma((uint64_t)r[c][2 * i] | ((uint64_t)r[c][2 * i + 1] << 32), sl2x2, negx2);
           uint64_t pp;
-          if ((i & 3) == 3) {  // a quarter of the exponentials on the FMA pipe
+          if ((i & 7) == 7) {  // an eighth of the exponentials on the FMA pipe
             pp = exp2_poly2(f2_lo(x), f2_hi(x));
           } else {
             pp = f2_pack(ex2_fast(f2_lo(x)), ex2_fast(f2_hi(x)));
