@@ -417,7 +417,7 @@ def run_ours(args, rank, world, local_rank):
 NCU_TRAFFIC = {
     "gemm_qkv_mlp_gelu_qknorm_rope": (336224000, ("gemm.cuh", "common.cuh"), "2f431c60dd9c3864"),
     "gemm_out_gated_residual": (437787904, ("gemm.cuh", "common.cuh"), "2f431c60dd9c3864"),
-    "attention": (95213568, ("attention.cuh", "common.cuh"), "8aa1fbcb8a30f541"),
+    "attention": (94483000, ("attention.cuh", "common.cuh"), "22ee6b04065cf91b"),
     "modulate_norm": (28440064, ("elementwise.cuh", "common.cuh"), "7edddd6c2e584c82"),
     "adaln_modulation": (56678400, ("elementwise.cuh", "common.cuh"), "7edddd6c2e584c82"),
 }

@@ -136,6 +136,52 @@ def test_single_block_in_place_matches_out_of_place():
     assert torch.equal(xi, out)
 
 
+_PDL_CHILD = r"""
+import sys, numpy as np, torch
+sys.path.insert(0, sys.argv[1])
+sys.path.insert(0, sys.argv[1] + "/tests")
+from diffusion_transformer_block_flux_b200 import synth
+import diffusion_transformer_block_flux_b200 as dit
+from helpers import dev_bf16, dev_tree
+shape = synth.BlockShape("pdl_check_S1088_D3072", 64, 16, 64, 3072, 24, 12288)
+w = dev_tree(synth.single_block_weights(shape, bias_std=0.1))
+a = synth.block_activations(shape)
+x = dev_bf16(a["x"]); vec = dev_bf16(a["vec"]).reshape(1, -1)
+rope = torch.empty((shape.S, 64, 2), dtype=torch.float32, device="cuda")
+dit.dit_rope_table(torch.from_numpy(a["ids"]).cuda(), (8, 28, 28), 10000.0, rope)
+cfg = dit.block_cfg(1, shape.S, shape.D, shape.H, shape.M)
+ws = torch.empty(dit.dit_single_block_workspace(cfg), dtype=torch.uint8, device="cuda")
+out = torch.empty_like(x)
+for _ in range(3):
+    dit.dit_single_block_fwd(cfg, dit.single_weights(w), x, vec, rope, out, ws)
+torch.cuda.synchronize()
+np.save(sys.argv[2], out.view(torch.int16).cpu().numpy())
+"""
+
+
+def test_single_block_launch_overlap_changes_no_bits(tmp_path):
+    """The block's kernels start their prologue while the previous kernel
+    drains (programmatic dependent launch) but touch memory only after it has
+    finished: the output equals the one with plain launches
+    (DIT_DISABLE_PDL=1) bit for bit, run back to back in two processes."""
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    outs = []
+    for env_off in (False, True):
+        env = dict(os.environ)
+        env.pop("DIT_DISABLE_PDL", None)
+        if env_off:
+            env["DIT_DISABLE_PDL"] = "1"
+        f = tmp_path / f"out_{int(env_off)}.npy"
+        r = subprocess.run([sys.executable, "-c", _PDL_CHILD, root, str(f)], env=env, capture_output=True,
+                           text=True, timeout=600)
+        assert r.returncode == 0, r.stderr[-2000:]
+        outs.append(np.load(f))
+    assert np.array_equal(outs[0], outs[1])
+
+
 @pytest.mark.parametrize("n", [1, 2, 5])
 def test_single_block_host_pipeline_equals_device_calls_bitwise(n):
     """The host-buffer pipeline runs the same kernels: each request's output
