@@ -5,11 +5,12 @@
 // 4608-token text|image sequence, 24 heads x 128, bf16, run by a flash
 // backend; §6.3 — operands laid out (B, S, H, D).  No mask.
 //
-// One CTA = one (batch, head) and two 128-row query tiles Q0, Q1.
+// One CTA = one (batch, head, key range) and two 128-row query tiles Q0, Q1.
 //   warps 0-3  softmax + epilogue for Q0 (thread = query row = TMEM lane)
 //   warps 4-7  softmax + epilogue for Q1
 //   warp 8     TMA producer: Q0, Q1 once; K_j, V_j through 2-stage rings
-//   warp 9     TMEM allocator + single-thread MMA issuer
+//   warp 9     TMEM allocator + MMA issuer (the whole warp runs the loop,
+//              one elected lane issues each tcgen05 instruction)
 // TMEM (512 columns): S [0,128) shared by both tiles, P0 [128,192),
 // P1 [192,256) (bf16 pairs), O0 [256,384), O1 [384,512).
 // The score tile S is the only buffer the two tiles share, and a tile's

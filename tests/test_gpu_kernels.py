@@ -226,20 +226,21 @@ def test_gemm_gated_residual(M, rows_per_batch, N, K, inplace):
     parity(host_f64(out_s), xsf + g * y, "gated residual, small residual")
 
 
-@pytest.mark.parametrize("epi,M1,M2,N,K", [
-    ("gated", 512, 4096, 768, 1536),   # text + image output projections (M1 < N: M-fastest; M2 > N: N-fastest)
-    ("gelu", 512, 1000, 1024, 512),    # MLP-in with GELU, ragged image rows
-    ("qk", 300, 700, 768, 256),        # QKV with the fused per-head RMSNorm + RoPE
-    ("gated", 100, 600, 256, 512),     # M1 <= 128: two launches
+@pytest.mark.parametrize("epi,M1,M2,N1,N2,K", [
+    ("gated", 512, 4096, 768, 768, 1536),   # text + image output projections (M1 < N: M-fastest; M2 > N: N-fastest)
+    ("gelu", 512, 1000, 1024, 1024, 512),   # MLP-in with GELU, ragged image rows
+    ("qk", 300, 700, 768, 768, 256),        # QKV with the fused per-head RMSNorm + RoPE
+    ("gelu", 600, 300, 512, 1536, 384),     # jobs of different widths
+    ("gated", 100, 600, 256, 256, 512),     # M1 <= 128: two launches
 ])
-def test_gemm_grouped_equals_two_calls(epi, M1, M2, N, K):
+def test_gemm_grouped_equals_two_calls(epi, M1, M2, N1, N2, K):
     """Two GEMMs in one grouped launch (the double-stream block's text and
     image layers) give exactly what two dit_gemm_epilogue calls give, and the
     oracle's result within the stated tolerance."""
     import torch
     D = 768
     jobs = []
-    for j, M in enumerate((M1, M2)):
+    for j, (M, N) in enumerate(((M1, N1), (M2, N2))):
         A, W, b = _gemm_inputs(M, N, K, seed=31 + 7 * j)
         t = {"A": dev_bf16(A), "W": dev_bf16(W), "b": dev_bf16(b), "Af": A, "Wf": W, "bf": b, "M": M}
         kw = dict(bias=t["b"])
@@ -258,8 +259,9 @@ def test_gemm_grouped_equals_two_calls(epi, M1, M2, N, K):
             t["rope"] = rope
             kw.update(epi=dit.DIT_EPI_BIAS, qk_cols=2 * (N // 3 // 128) * 128, rope=rope, rope_rows=M)
         t["kw"] = kw
+        t["N"] = N
         jobs.append(t)
-    sep = [torch.empty((t["M"], N), dtype=torch.bfloat16, device="cuda") for t in jobs]
+    sep = [torch.empty((t["M"], t["N"]), dtype=torch.bfloat16, device="cuda") for t in jobs]
     grp = [torch.empty_like(o) for o in sep]
     for t, o in zip(jobs, sep):
         dit.dit_gemm_epilogue(t["A"], t["W"], o, **t["kw"])
@@ -561,6 +563,34 @@ def test_attention_split_accumulates_like_a_ring():
     assert_no_device_error()
 
 
+def test_attention_split_accumulates_into_a_strided_result():
+    """The running result of a ring step may be a column block of a wider
+    buffer (the block's [attn | mlp] concat, row stride D + M): split parts
+    (row stride D) and the running result (its own stride) merge into it,
+    and the columns beside it are left alone."""
+    import torch
+    H, Sq = 2, 300
+    D = H * 128
+    W = D + 512  # concat row: attention columns, then other columns
+    cuts = (0, 640, 1000)
+    q, k, v = _attn_case(1, Sq, cuts[-1], H, 1.5, seed=29)
+    dq, dk, dv = dev_bf16(q), dev_bf16(k), dev_bf16(v)
+    cat = torch.full((Sq, W), 7.0, dtype=torch.bfloat16, device="cuda")
+    o = cat[:, :D]
+    lse = torch.empty((1, H, Sq), dtype=torch.float32, device="cuda")
+    ws = torch.empty(dit.dit_attention_split_workspace(1, Sq, H, 3), dtype=torch.uint8, device="cuda")
+    for i, (a, b) in enumerate(zip(cuts, cuts[1:])):
+        dit.dit_attention_split(dq, dk[a:b], dv[a:b], o, 1, Sq, b - a, H, 3, ws, lse=lse, accumulate=i > 0)
+    torch.cuda.synchronize()
+    assert bool((cat[:, D:] == 7.0).all())
+    qf, kf, vf = (synth.bf16_bits_to_f64(t) for t in (q, k, v))
+    ref = O.attention(qf, kf, vf, H)
+    rms = np.sqrt(np.mean(ref ** 2))
+    parity(host_f64(o.contiguous()), ref, "split ring into a strided result",
+           max_abs_frac=3e-2 + 4 * 2.0 ** -9 * np.abs(ref).max() / rms)
+    assert_no_device_error()
+
+
 def test_sequence_parallel_drivers_with_cuda_kernels_one_rank():
     """ring_attention and ulysses_attention with their default CUDA local
     operations in a one-rank NCCL group (no transfer; the multi-rank
@@ -652,6 +682,18 @@ def test_sequence_parallel_block_one_rank_equals_block_and_graph_replays_it(mode
         graph.replay()
         torch.cuda.synchronize()
         assert torch.equal(out, ref)
+        if mode == "ring":
+            # the plan's default for so few query tiles cuts the keys
+            # (dit_attention_split into the strided concat buffer): the oracle's
+            # block within the block tolerance
+            assert sp.auto_key_splits(s.S, s.H, "cuda") > 1
+            blk2 = sp.SequenceParallelSingleBlock(s.S, s.D, s.H, s.M, "cuda", mode=mode)
+            out2 = torch.empty_like(x)
+            blk2.forward(w, x, vec, rope, out2)
+            torch.cuda.synchronize()
+            f = synth.to_f64(ab)
+            oref = O.single_block(f["x"], f["vec"], f["ids"], synth.to_f64(wb), s.H)
+            parity(host_f64(out2), oref, "sequence-parallel block, keys split")
     finally:
         del graph  # a graph holding NCCL work is released before the group
         dist.destroy_process_group()
