@@ -35,6 +35,7 @@ enum WaitSite : uint32_t {
   SITE_GEMM2_MMA = 12,
   SITE_GEMM2_EPILOGUE = 13,
   SITE_GEMM2_DRAIN = 14,
+  SITE_NORM_RING = 15,
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -132,6 +133,34 @@ __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, uint
     }
   }
   return true;
+}
+
+// Polls the phase with the non-blocking test (no suspension, so the thread
+// resumes the moment the phase completes), reading the clock every 256 polls.
+// Returns false after recording a timeout once limit_ns has passed.
+__device__ __forceinline__ bool mbar_wait_poll(uint64_t* bar, uint32_t parity, uint64_t limit_ns, uint32_t site) {
+  uint32_t k = 0;
+  uint64_t t0 = 0;
+  for (;;) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    if (ok) return true;
+    if ((++k & 255u) == 0) {
+      const uint64_t now = globaltimer_ns();
+      if (t0 == 0) {
+        t0 = now;
+      } else if (now - t0 > limit_ns) {
+        atomicCAS(&g_dit_error, 0u, (uint32_t)DIT_ERR_TIMEOUT | (site << 8));
+        return false;
+      }
+    }
+  }
 }
 
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns,
@@ -525,6 +554,11 @@ __device__ __forceinline__ float f2_hi(uint64_t v) { return __uint_as_float((uin
 __device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
   uint64_t d;
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
 __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {

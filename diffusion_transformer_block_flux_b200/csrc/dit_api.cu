@@ -236,6 +236,23 @@ dit_status launch_qk(const bf16* q, const bf16* k, int64_t ld_in, const bf16* qs
   return launch_status();
 }
 
+// LayerNorm + modulate row ring: resident CTAs per SM and the shared-memory
+// budget of one CTA's ring of rows.
+constexpr int kNormRingCtasPerSm = 4;
+constexpr int kNormRingBytes = 18432;
+
+template <typename Kern>
+static dit_status ring_launch(Kern kernel, dim3 grid, int threads, int smem, cudaStream_t st, const bf16* x,
+                              int64_t ldx, const float* shift, const float* scale, int64_t mod_stride, bf16* y,
+                              int64_t ldy, int S, int D, float eps, int R) {
+  // dynamic plus static shared memory above 48 KB needs the opt-in
+  if (smem > 40 * 1024 && cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return DIT_ERR_CUDA;
+  launch_pdl(kernel, grid, threads, smem, st, x, ldx, shift, scale, mod_stride, y, ldy, S, D, eps, R,
+             g_wait_limit_ns);
+  return DIT_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -537,20 +554,26 @@ dit_status dit_modulate_norm(const dit_bf16* x, int64_t ldx, const float* shift,
       }
     }
     if (NC != 0 && B <= 65535) {
-      const dim3 grid((unsigned)S, (unsigned)B);
+      // persistent row ring: kNormRingCtasPerSm CTAs per SM in all, each with
+      // R = kNormRingBytes / (2 D) rows (2..8) in flight
       const int threads = D / (8 * NC);
+      const int R = std::max(2, std::min(dit::kNormRingMaxStages, kNormRingBytes / (2 * D)));
+      const int smem = R * 2 * D;
+      const int gx = (int)std::max<int64_t>(1, std::min<int64_t>(S, ((int64_t)kNormRingCtasPerSm * sms + B - 1) / B));
+      const dim3 grid((unsigned)gx, (unsigned)B);
       if (NC == 1)
-        launch_pdl(dit::modulate_norm_row_kernel<1>, grid, threads, 0, st, xb, ldx, shift, scale, mod_stride, yb, ldy, S, D,
-                                                                    eps);
+        s = ring_launch(dit::modulate_norm_ring_kernel<1>, grid, threads, smem, st, xb, ldx, shift, scale, mod_stride, yb,
+                        ldy, S, D, eps, R);
       else if (NC == 2)
-        launch_pdl(dit::modulate_norm_row_kernel<2>, grid, threads, 0, st, xb, ldx, shift, scale, mod_stride, yb, ldy, S, D,
-                                                                    eps);
+        s = ring_launch(dit::modulate_norm_ring_kernel<2>, grid, threads, smem, st, xb, ldx, shift, scale, mod_stride, yb,
+                        ldy, S, D, eps, R);
       else if (NC == 3)
-        launch_pdl(dit::modulate_norm_row_kernel<3>, grid, threads, 0, st, xb, ldx, shift, scale, mod_stride, yb, ldy, S, D,
-                                                                    eps);
+        s = ring_launch(dit::modulate_norm_ring_kernel<3>, grid, threads, smem, st, xb, ldx, shift, scale, mod_stride, yb,
+                        ldy, S, D, eps, R);
       else
-        launch_pdl(dit::modulate_norm_row_kernel<4>, grid, threads, 0, st, xb, ldx, shift, scale, mod_stride, yb, ldy, S, D,
-                                                                    eps);
+        s = ring_launch(dit::modulate_norm_ring_kernel<4>, grid, threads, smem, st, xb, ldx, shift, scale, mod_stride, yb,
+                        ldy, S, D, eps, R);
+      if (s != DIT_OK) return s;
       return launch_status();
     }
     // otherwise (D not a multiple of 256 or 768): persistent row stream, D/8 threads per CTA

@@ -96,6 +96,36 @@ def test_modulate_norm(B, S, D):
     parity(host_f64(y), O.layer_norm(xf).reshape(B * S, D), "layer_norm")
 
 
+def test_modulate_norm_equal_and_offset_rows():
+    """Rows of one repeated value normalise to exactly 0 (then the shift);
+    rows far from zero mean (offset 200, std 1) keep their deviations: the
+    statistics are taken about the mean, not as E[x^2] - E[x]^2.  More rows
+    than resident CTAs, so every CTA's ring of rows wraps."""
+    import torch
+    S, D = 2000, 3072
+    x = synth.normal_bf16(5, "x", (S, D))
+    vals = [0.0, 1.0, -3.5, 1e-3, 448.0, 65536.0]
+    for r, c in enumerate(vals):
+        x[r] = synth.const_bf16((D,), c)
+    off = synth.normal_bf16(6, "off", (8, D), 1.0, 200.0)
+    x[len(vals):len(vals) + 8] = off
+    sh = synth.bf16_bits_to_f64(synth.normal_bf16(7, "sh", (1, D), 0.7))
+    sc = synth.bf16_bits_to_f64(synth.normal_bf16(8, "sc", (1, D), 0.7))
+    y = torch.empty((S, D), dtype=torch.bfloat16, device="cuda")
+    xf = synth.bf16_bits_to_f64(x)
+    dit.dit_modulate_norm(dev_bf16(x), None, None, y, 1, S)
+    got = host_f64(y)
+    assert np.all(got[:len(vals)] == 0.0), "equal rows must normalise to exactly 0"
+    parity(got, O.layer_norm(xf), "layer_norm equal/offset rows")
+    dit.dit_modulate_norm(dev_bf16(x), f32dev(sh), f32dev(sc), y, 1, S, mod_stride=D)
+    got = host_f64(y)
+    ref = O.modulate(O.layer_norm(xf), sh, sc)
+    np.testing.assert_array_equal(got[:len(vals)], host_f64(dev_bf16(synth.f32_to_bf16_bits(
+        np.broadcast_to(sh.astype(np.float32), (len(vals), D))))))
+    parity(got, ref, "modulate_norm equal/offset rows")
+    parity(got[len(vals):len(vals) + 8], ref[len(vals):len(vals) + 8], "modulate_norm offset rows")
+
+
 # ---------------------------------------------------------------- QK RMSNorm + RoPE
 
 @pytest.mark.parametrize("B,nt,gh,gw,H", [(1, 64, 12, 16, 3), (2, 5, 3, 7, 2)])
