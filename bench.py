@@ -415,11 +415,11 @@ def run_ours(args, rank, world, local_rank):
 # (profiles/*.ncu.md), with a hash of the kernel's sources at capture time.
 # A kernel whose sources changed since reports traffic null.
 NCU_TRAFFIC = {
-    "gemm_qkv_mlp_gelu_qknorm_rope": (336224000, ("gemm.cuh", "common.cuh"), "2f431c60dd9c3864"),
-    "gemm_out_gated_residual": (437787904, ("gemm.cuh", "common.cuh"), "2f431c60dd9c3864"),
-    "attention": (94483000, ("attention.cuh", "common.cuh"), "22ee6b04065cf91b"),
-    "modulate_norm": (28440064, ("elementwise.cuh", "common.cuh"), "7edddd6c2e584c82"),
-    "adaln_modulation": (56678400, ("elementwise.cuh", "common.cuh"), "7edddd6c2e584c82"),
+    "gemm_qkv_mlp_gelu_qknorm_rope": (335667712, ("gemm.cuh", "common.cuh"), "a040db127389a835"),
+    "gemm_out_gated_residual": (435962112, ("gemm.cuh", "common.cuh"), "a040db127389a835"),
+    "attention": (94130688, ("attention.cuh", "common.cuh"), "38a153274e62a573"),
+    "modulate_norm": (28391168, ("elementwise.cuh", "common.cuh"), "8fa8fb1c7db5f362"),
+    "adaln_modulation": (56746752, ("elementwise.cuh", "common.cuh"), "8fa8fb1c7db5f362"),
 }
 
 
