@@ -171,6 +171,9 @@ dit_status dit_vec_linear(const dit_bf16* x, int64_t ldx, const dit_bf16* W, int
  * per row r of D elements, b = r / S (rows of batch b are contiguous), biased
  * variance, no LayerNorm affine.  shift/scale: device float, row b at
  * shift + b * mod_stride; pass shift = scale = NULL for a plain LayerNorm.
+ * Mean and variance are taken in fp32 over the row shifted by its first
+ * element (relative error of the variance below about D * 2^-24 for any
+ * row; a row of equal values normalises to exactly 0).
  *   x, y device bf16 [B*S][ld].  y must not alias x.  D % 8 == 0, D <= 8192. */
 dit_status dit_modulate_norm(const dit_bf16* x, int64_t ldx, const float* shift, const float* scale,
                              int64_t mod_stride, dit_bf16* y, int64_t ldy,
