@@ -611,7 +611,7 @@ def run_double(args):
                      args.steps, args.warmup, torch.cuda.current_stream())
     flops = 2.0 * S * D * (3 * D + D + 2 * M) + 4.0 * S * S * H * 128 + 2 * 2.0 * D * 6 * D
     return _extra_line("flux_double_block_T512_I4096_D3072_bf16", ms, flops, args.steps, args.warmup,
-                       {"gpu_launches_per_step": 15})
+                       {"gpu_launches_per_step": 11})
 
 
 def run_video(args):
