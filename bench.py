@@ -643,7 +643,7 @@ def run_video(args):
     flops = (2.0 * Sv * Dv * (3 * Dv + Dv + Dv + Dv + 2 * Mv) + 2.0 * C * Dv * 2 * Dv + 4.0 * Sv * Sv * Hv * 128
              + 4.0 * Sv * C * Hv * 128 + 2.0 * Dv * 6 * Dv)
     return _extra_line("video_block_S28350_D1536_H12_M8960_ctx512_bf16", ms, flops, K, args.warmup,
-                       {"gpu_launches_per_step": 14})
+                       {"gpu_launches_per_step": 13})
 
 
 def run_ring8(args):
