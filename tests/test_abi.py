@@ -235,3 +235,39 @@ def test_noalloc_reports_the_same_status_as_the_workspace_call(L):
     big = dit.block_cfg(1, 4608, 3072, 24, 12288)
     assert L.dit_single_block_fwd_noalloc(ctypes.byref(big), ctypes.byref(weights), None, None, None, None,
                                           None) == dit.DIT_ERR_WORKSPACE
+
+
+def test_split_attention_and_grouped_gemm_validate_on_the_host(L):
+    """The key-split attention's workspace query is plain arithmetic (one bf16
+    partial result and one fp32 lse per split, each 256-byte aligned, at most
+    four splits); bad split counts, a missing or misaligned workspace and
+    mismatched grouped GEMM jobs are rejected before any CUDA call."""
+    def a256(n):
+        return (n + 255) // 256 * 256
+    B, Sq, H = 2, 577, 3
+    for n in (1, 2, 3, 4, 7):
+        k = min(n, 4)
+        assert L.dit_attention_split_workspace(B, Sq, H, n) == k * a256(B * Sq * H * 128 * 2) + k * a256(B * H * Sq * 4)
+    for bad in ((0, Sq, H, 2), (B, 0, H, 2), (B, Sq, 0, 2), (B, Sq, H, 0)):
+        assert L.dit_attention_split_workspace(*bad) == 0
+    p = ctypes.c_void_p(256)
+    ws = L.dit_attention_split_workspace(1, 64, 1, 2)
+
+    def split(n_split, accumulate=0, lse=p, workspace=p, nbytes=ws, Skv=1000, B=1):
+        return L.dit_attention_split(p, p, p, 128, 128, 128, p, 128, lse, B, 64, Skv, 1, 128, 0.1, n_split,
+                                     accumulate, workspace, nbytes, None)
+    assert split(0) == dit.DIT_ERR_INVALID_ARG
+    assert split(5) == dit.DIT_ERR_INVALID_ARG
+    assert split(2, accumulate=1, lse=None) == dit.DIT_ERR_INVALID_ARG
+    assert split(2, B=0) == dit.DIT_ERR_SHAPE
+    # 1000 keys are 8 key tiles: two splits need the workspace
+    assert split(2, workspace=None) == dit.DIT_ERR_WORKSPACE
+    assert split(2, nbytes=ws - 1) == dit.DIT_ERR_WORKSPACE
+    assert split(2, workspace=ctypes.c_void_p(272)) == dit.DIT_ERR_ALIGNMENT
+    # grouped GEMM: both jobs valid, same epilogue and the same K
+    g1 = dit.dit_gemm_args(A=256, lda=64, W=256, ldw=64, C=256, ldc=64, M=256, N=64, K=64)
+    g2 = dit.dit_gemm_args(A=256, lda=128, W=256, ldw=128, C=256, ldc=64, M=256, N=64, K=128)
+    assert L.dit_gemm_epilogue_grouped(None, ctypes.byref(g1), None) == dit.DIT_ERR_INVALID_ARG
+    assert L.dit_gemm_epilogue_grouped(ctypes.byref(g1), ctypes.byref(g2), None) == dit.DIT_ERR_INVALID_ARG
+    bad = dit.dit_gemm_args(A=256, lda=64, W=256, ldw=64, C=256, ldc=64, M=1, N=33, K=64)
+    assert L.dit_gemm_epilogue_grouped(ctypes.byref(g1), ctypes.byref(bad), None) == dit.DIT_ERR_SHAPE
