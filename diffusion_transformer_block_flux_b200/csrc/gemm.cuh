@@ -446,6 +446,35 @@ __device__ __forceinline__ int group_tile(const PairGroup& G, int tiles0, int ti
   return g;
 }
 
+// Work items of the persistent schedule.  The tiles of the complete waves
+// run whole.  When the last, partial wave holds at most half as many tiles as
+// there are clusters, each of its tiles runs as two items of 128 columns
+// (N = 128 MMAs) on two clusters, so that wave takes half a tile's time:
+// the fused QKV|MLP-in GEMM of the single-stream block at S = 4608 has 1512
+// tiles for 74 SM pairs, 20 whole waves and 32 tiles left.
+constexpr int BN_HALF = 128;
+constexpr uint32_t IDESC_HALF = idesc_bf16(BM, BN_HALF, 0, 0);
+
+struct TailPlan {
+  int full;   // tiles that run whole (complete waves, or every tile without a split)
+  int items;  // work items in all
+};
+__device__ __forceinline__ TailPlan tail_plan(int num_tiles, int n_clusters) {
+  const int full = num_tiles / n_clusters * n_clusters;
+  const int rem = num_tiles - full;
+  if (rem > 0 && 2 * rem <= n_clusters) return TailPlan{full, full + 2 * rem};
+  return TailPlan{num_tiles, num_tiles};
+}
+// item -> tile and column half (-1: the whole tile)
+__device__ __forceinline__ int item_tile(const TailPlan& P, int item, int& half) {
+  if (item < P.full) {
+    half = -1;
+    return item;
+  }
+  half = (item - P.full) & 1;
+  return P.full + ((item - P.full) >> 1);
+}
+
 template <int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     gemm_pair_kernel(const __grid_constant__ PairGroup G, int K, uint64_t wait_limit) {
@@ -499,6 +528,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
   const int num_kb = (K + BK - 1) / BK;
   const int cluster_id = blockIdx.x >> 1;
   const int n_clusters = gridDim.x >> 1;
+  const TailPlan plan = tail_plan(num_tiles, n_clusters);
 
   if (warp == 0) {
     if (lane == 0) {
@@ -509,9 +539,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       bool ok = true;
       int wave = 0;  // this cluster's tile count so far: the same for every cluster of a wave
       const uint64_t b_policy = l2_policy_evict_last();
-      for (int tile = cluster_id; tile < num_tiles && ok; tile += n_clusters, ++wave) {
-        int tm, tn;
-        const PairJob& J = G.job[group_tile(G, tiles0, tile, tm, tn)];
+      for (int item = cluster_id; item < plan.items && ok; item += n_clusters, ++wave) {
+        int tm, tn, half;
+        const PairJob& J = G.job[group_tile(G, tiles0, item_tile(plan, item, half), tm, tn)];
+        // B rows of this CTA: its half of the tile's 256 columns, or of the
+        // 128 columns of a half item (the box still loads 128 rows; the MMA
+        // reads the first 64)
+        const int b_row = tn * BN + (half < 0 ? (int)rank * BN_CTA : half * BN_HALF + (int)rank * (BN_HALF / 2));
         const bool keep_b = J.n_fastest && J.ep.w_keep != nullptr;
         // N-fastest: every other wave walks K backwards, so that it starts on the
         // K range whose weight panels the previous wave touched last (still in L2)
@@ -526,10 +560,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
           const int kx = (back ? num_kb - 1 - kb : kb) * BK;
           tma_load_2d_pair(sA + stage * A_BYTES, &J.tmA, leader_full, kx, tm * BM + (int)rank * BM_CTA);
           if (keep_b)
-            tma_load_2d_pair_hint(sB + stage * B_BYTES, &J.tmB, leader_full, kx, tn * BN + (int)rank * BN_CTA,
-                                  b_policy);
+            tma_load_2d_pair_hint(sB + stage * B_BYTES, &J.tmB, leader_full, kx, b_row, b_policy);
           else
-            tma_load_2d_pair(sB + stage * B_BYTES, &J.tmB, leader_full, kx, tn * BN + (int)rank * BN_CTA);
+            tma_load_2d_pair(sB + stage * B_BYTES, &J.tmB, leader_full, kx, b_row);
           issued_mask |= 1u << stage;
           issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) {
@@ -557,7 +590,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       // descriptor of stage 0's A and B tiles; a stage or a 16-deep slice adds (byte offset >> 4)
       const uint64_t dA = sdesc_sw128(smem_u32(sA), 16, 1024);
       const uint64_t dB = sdesc_sw128(smem_u32(sB), 16, 1024);
-      for (int tile = cluster_id; tile < num_tiles && ok; tile += n_clusters) {
+      for (int item = cluster_id; item < plan.items && ok; item += n_clusters) {
+        int half;
+        (void)item_tile(plan, item, half);
+        const uint32_t idesc = half < 0 ? IDESC : IDESC_HALF;
         if (!__all_sync(0xffffffffu, mbar_wait(&tempty[acc], acc_phase ^ 1, wait_limit, abort_flag, SITE_GEMM2_MMA))) {
           ok = false;
           break;
@@ -574,7 +610,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
           const uint64_t b0 = dB + (uint64_t)((stage * B_BYTES) >> 4);
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k)
-            umma_ss_pair_elect(d_tmem, a0 + (uint64_t)(k * 2), b0 + (uint64_t)(k * 2), IDESC, (kb | k) != 0 ? 1u : 0u);
+            umma_ss_pair_elect(d_tmem, a0 + (uint64_t)(k * 2), b0 + (uint64_t)(k * 2), idesc, (kb | k) != 0 ? 1u : 0u);
           issued_any = true;
           umma_commit_pair_elect(&empty[stage], 0x3);
           if (++stage == STAGES) {
@@ -602,9 +638,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     const uint32_t leader_tempty1 = mapa_shared(smem_u32(&tempty[1]), 0);
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int tile = cluster_id; tile < num_tiles; tile += n_clusters) {
-      int tm, tn;
-      const PairJob& J = G.job[group_tile(G, tiles0, tile, tm, tn)];
+    for (int item = cluster_id; item < plan.items; item += n_clusters) {
+      int tm, tn, half;
+      const PairJob& J = G.job[group_tile(G, tiles0, item_tile(plan, item, half), tm, tn)];
+      const int col0 = tn * BN + (half < 0 ? 0 : half * BN_HALF);  // first output column of the item
+      const int chunks = (half < 0 ? BN : BN_HALF) / 32;
       const Epi& ep = J.ep;
       const int M = J.M, N = J.N;
       bool ok = mbar_wait(&tfull[acc], acc_phase, wait_limit, abort_flag, SITE_GEMM2_EPILOGUE);
@@ -613,8 +651,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       const int m = tm * BM + row_in_tile;
       const uint32_t t_row = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * BN);
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        const int n0 = tn * BN + c * 32;
+      for (int c = 0; c < chunks; ++c) {
+        const int n0 = col0 + c * 32;
         if (n0 >= N) break;  // warp-uniform
         if (EPI != DIT_EPI_BIAS_GATED_RESIDUAL && n0 < ep.qk_cols) {
           epilogue_qk_head(t_row + (uint32_t)(c * 32), m, n0, ep, m < M);
